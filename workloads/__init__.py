@@ -1,0 +1,229 @@
+"""Seeded synthetic inputs for the heterogeneous-batch LoRA adapter branch.
+
+This module only draws random data and arranges it; it holds none of the
+method's arithmetic (no shrink, no expand, no scaling).  Both the oracle
+tests and the CUDA path consume what it returns, so that the two sides see
+bit-identical inputs.
+
+Shapes follow the workloads of the pages:
+  * "Multi-LoRA Serving in Production" (llms.blog), section "The Mathematical
+    Anatomy of Heterogeneous Batches": row-vector layout X [T, d_in],
+    A [d_in, r], B [r, d_out].
+  * "Multi-LoRA Serving Architecture ... (2026)" (iotdigitaltwinplm.com),
+    section "The memory arithmetic that makes it work": 7B/8B projection
+    widths 4096 / 11008 / 14336; section "An adapter-cache LRU simulator":
+    Zipf popularity p_i proportional to i^-s over i = 1..n.
+
+Value recipe (all configs): X, A, B ~ N(0,1)/sqrt(fan_in) rounded to bf16 by
+round-to-nearest-even (torch ``.to(bfloat16)``), fan_in = d_in for X and A and
+r for B; Y_base ~ N(0,1) in fp32; alpha = 2r so alpha/r = 2.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import List, Optional
+
+import numpy as np
+import torch
+
+PAGE_ROWS = 16
+MAX_RANK = 64
+
+
+def bf16_round(a: np.ndarray) -> np.ndarray:
+    """Round float data to the nearest bf16 value (RNE); return float32 holding it."""
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    return t.to(torch.bfloat16).to(torch.float32).numpy()
+
+
+def bf16_bits(a: np.ndarray) -> np.ndarray:
+    """Bit patterns (uint16) of float32 data that already holds bf16 values."""
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    return (a.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def zipf_weights(n: int, s: float) -> np.ndarray:
+    """Normalised Zipf popularity, p_i proportional to i^-s for i = 1..n."""
+    w = np.arange(1, n + 1, dtype=np.float64) ** (-float(s))
+    return w / w.sum()
+
+
+@dataclasses.dataclass
+class Adapter:
+    rank: int
+    alpha: float
+    A: np.ndarray  # [d_in, r] float32 holding bf16 values
+    B: np.ndarray  # [r, d_out] float32 holding bf16 values
+
+
+@dataclasses.dataclass
+class Workload:
+    name: str
+    d_in: int
+    d_out: int
+    X: np.ndarray          # [T, d_in] float32 (bf16 values)
+    Y_base: np.ndarray     # [T, d_out] float32
+    ids: np.ndarray        # [T] int32, -1 = base model only
+    adapters: List[Optional[Adapter]]  # one entry per slot; None = empty slot
+    # seeded physical page ids per slot: [S, 2, 4] (unused entries -1)
+    page_ids: np.ndarray
+    pages_a: int           # number of pages needed in the d_in-wide pool
+    pages_b: int           # number of pages needed in the d_out-wide pool
+
+    @property
+    def T(self) -> int:
+        return int(self.X.shape[0])
+
+    @property
+    def S(self) -> int:
+        return len(self.adapters)
+
+    def ranks(self) -> np.ndarray:
+        return np.array([0 if a is None else a.rank for a in self.adapters], dtype=np.int32)
+
+    def scales_f32(self) -> np.ndarray:
+        """alpha/r per slot, rounded once to fp32 (both sides widen this value)."""
+        out = np.zeros(self.S, dtype=np.float32)
+        for i, a in enumerate(self.adapters):
+            if a is not None:
+                out[i] = np.float32(a.alpha) / np.float32(a.rank)
+        return out
+
+
+def _draw_adapter(rng: np.random.Generator, d_in: int, d_out: int, r: int) -> Adapter:
+    A = bf16_round(rng.standard_normal((d_in, r), dtype=np.float32) / np.sqrt(d_in))
+    B = bf16_round(rng.standard_normal((r, d_out), dtype=np.float32) / np.sqrt(r))
+    return Adapter(rank=r, alpha=2.0 * r, A=A, B=B)
+
+
+def _assign_pages(rng: np.random.Generator, ranks: np.ndarray, extra_pages: int = 3):
+    """Shuffled physical page ids for every (slot, matrix, page) of the resident adapters."""
+    S = len(ranks)
+    need = np.array([(int(r) + PAGE_ROWS - 1) // PAGE_ROWS for r in ranks], dtype=np.int64)
+    total = int(need.sum())
+    pid = np.full((S, 2, 4), -1, dtype=np.int32)
+    n_pool = total + extra_pages
+    for m in range(2):
+        order = rng.permutation(n_pool)[:total]
+        k = 0
+        for i in range(S):
+            for p in range(int(need[i])):
+                pid[i, m, p] = order[k]
+                k += 1
+    return pid, n_pool, n_pool
+
+
+def _finish(name, rng, d_in, d_out, T, ids, adapters) -> Workload:
+    X = bf16_round(rng.standard_normal((T, d_in), dtype=np.float32) / np.sqrt(d_in))
+    Y_base = rng.standard_normal((T, d_out), dtype=np.float32)
+    ranks = np.array([0 if a is None else a.rank for a in adapters], dtype=np.int32)
+    pid, na, nb = _assign_pages(rng, ranks)
+    return Workload(name=name, d_in=d_in, d_out=d_out, X=X, Y_base=Y_base,
+                    ids=np.ascontiguousarray(ids, dtype=np.int32), adapters=adapters,
+                    page_ids=pid, pages_a=na, pages_b=nb)
+
+
+# ---------------------------------------------------------------------------
+# The five workload shapes
+# ---------------------------------------------------------------------------
+
+def tiny(seed: int = 0) -> Workload:
+    """d_in = d_out = 256, 8 decode tokens, 3 adapters of rank 4, 8, 16, uniform ids."""
+    rng = np.random.default_rng(seed)
+    d = 256
+    adapters = [_draw_adapter(rng, d, d, r) for r in (4, 8, 16)]
+    ids = rng.integers(0, 3, size=8)
+    return _finish("tiny_d256_T8", rng, d, d, 8, ids, adapters)
+
+
+def decode_q_proj_7b(seed: int = 1, T: int = 64) -> Workload:
+    """d = 4096, one token per sequence, 32 resident rank-16 adapters drawn
+    Zipf(1.0) without replacement from a 1000-adapter catalogue; each token draws
+    a resident adapter with its renormalised Zipf weight."""
+    rng = np.random.default_rng(seed)
+    d = 4096
+    w = zipf_weights(1000, 1.0)
+    cat = rng.choice(1000, size=32, replace=False, p=w)
+    p = w[cat] / w[cat].sum()
+    adapters = [_draw_adapter(rng, d, d, 16) for _ in range(32)]
+    ids = rng.choice(32, size=T, p=p)
+    return _finish(f"decode_q_proj_7b_T{T}", rng, d, d, T, ids, adapters)
+
+
+def mixed_mlp(seed: int = 2, which: str = "up", T: int = 256) -> Workload:
+    """256 decode tokens through the MLP up (4096 -> 11008) or down (11008 -> 4096)
+    projection; 128 resident adapters with ranks uniform over {8,16,32,64};
+    tokens assigned by Zipf(1.1) over the resident slots."""
+    rng = np.random.default_rng(seed)
+    d_in, d_out = (4096, 11008) if which == "up" else (11008, 4096)
+    ranks = rng.choice(np.array([8, 16, 32, 64]), size=128)
+    adapters = [_draw_adapter(rng, d_in, d_out, int(r)) for r in ranks]
+    slot_order = rng.permutation(128)
+    ids = slot_order[rng.choice(128, size=T, p=zipf_weights(128, 1.1))]
+    return _finish(f"mixed_mlp_{which}_T{T}", rng, d_in, d_out, T, ids, adapters)
+
+
+def prefill(seed: int = 3, n_seq: int = 16, len_lo: int = 128, len_hi: int = 2048,
+            d: int = 4096) -> Workload:
+    """16 sequences of length uniform in [128, 2048], each one adapter; 6 distinct
+    adapters with ranks drawn from {8,16,32,64}; tokens of a sequence are contiguous."""
+    rng = np.random.default_rng(seed)
+    n_ad = 6
+    ranks = rng.choice(np.array([8, 16, 32, 64]), size=n_ad)
+    adapters = [_draw_adapter(rng, d, d, int(r)) for r in ranks]
+    lens = rng.integers(len_lo, len_hi + 1, size=n_seq)
+    seq_ad = rng.permutation(np.arange(n_seq) % n_ad)
+    ids = np.concatenate([np.full(int(L), int(a)) for L, a in zip(lens, seq_ad)])
+    T = int(lens.sum())
+    return _finish(f"prefill_{n_seq}seq_T{T}", rng, d, d, T, ids, adapters)
+
+
+def sweep_8b(seed: int = 4, T: int = 64, regime: str = "distinct", pool: int = 512,
+             d_in: int = 4096, d_out: int = 14336, rank: int = 64) -> Workload:
+    """d_in = 4096, d_out = 14336, rank 64, a pool of 512 resident adapters;
+    regime "one": every token on one adapter; "distinct": token t uses
+    perm[t mod 512] so min(T, 512) distinct adapters."""
+    rng = np.random.default_rng(seed)
+    adapters = [_draw_adapter(rng, d_in, d_out, rank) for _ in range(pool)]
+    if regime == "one":
+        ids = np.full(T, int(rng.integers(0, pool)))
+    else:
+        perm = rng.permutation(pool)
+        ids = perm[np.arange(T) % pool]
+    return _finish(f"sweep_8b_{regime}_T{T}", rng, d_in, d_out, T, ids, adapters)
+
+
+def random_small(seed: int, T: int, d_in: int, d_out: int, S: int,
+                 ranks=(1, 4, 8, 16), p_none: float = 0.1, p_empty: float = 0.0) -> Workload:
+    """Random small case: mixed ranks, some id = -1 tokens, optional empty slots."""
+    rng = np.random.default_rng(seed)
+    adapters: List[Optional[Adapter]] = []
+    for _ in range(S):
+        if rng.random() < p_empty:
+            adapters.append(None)
+        else:
+            adapters.append(_draw_adapter(rng, d_in, d_out, int(rng.choice(np.array(ranks)))))
+    ids = rng.integers(0, S, size=T)
+    ids[rng.random(T) < p_none] = -1
+    return _finish(f"random_T{T}_{d_in}x{d_out}_S{S}", rng, d_in, d_out, T, ids, adapters)
+
+
+def by_name(name: str, **kw) -> Workload:
+    table = {
+        "tiny": tiny,
+        "decode_q_proj_7b": decode_q_proj_7b,
+        "mixed_mlp_up": lambda **k: mixed_mlp(which="up", **k),
+        "mixed_mlp_down": lambda **k: mixed_mlp(which="down", **k),
+        "prefill": prefill,
+        "sweep_8b_one": lambda **k: sweep_8b(regime="one", **k),
+        "sweep_8b_distinct": lambda **k: sweep_8b(regime="distinct", **k),
+    }
+    return table[name](**kw)
+
+
+def shard_tokens(T: int, rank: int, world: int):
+    """Contiguous token range [lo, hi) that data-parallel replica `rank` of `world` takes."""
+    base, rem = divmod(T, world)
+    lo = rank * base + min(rank, rem)
+    hi = lo + base + (1 if rank < rem else 0)
+    return lo, hi
