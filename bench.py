@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Benchmark of the heterogeneous-batch LoRA adapter branch on B200.
+
+Metric: LoRA-branch tokens/s per layer.  One step = one batch through the
+whole hot path: the segment plan of the batch (made once, as a model does for
+all of its adapted layers) and the fused shrink + expand-add of every layer
+in a ring of independent layer instances (own pools, page tables, X and Y per
+layer).  The ring's footprint is more than 4x the L2 cache, so every layer's
+weights and activations come from HBM.  The step is captured once in a CUDA
+graph and replayed.  value = tokens x layers x steps / device time.
+
+Default workload: 7B decode q_proj, d_in = d_out = 4096, 64 tokens (one per
+sequence), 32 resident rank-16 adapters with Zipf(1.0) popularity, bf16
+weights in 16-row pages with shuffled page order, fp32 Y_base.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "LoRA-branch tokens/s per layer"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="decode_q_proj_7b",
+                   help="decode_q_proj_7b | mixed_mlp_up | mixed_mlp_down | prefill | sweep_8b_one_T<n> | sweep_8b_distinct_T<n>")
+    p.add_argument("--layers", type=int, default=0, help="ring size (0 = enough for > 4x L2)")
+    p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# Workload description (shapes and ids only; weights are drawn per layer)
+# ---------------------------------------------------------------------------
+
+def workload_spec(name: str):
+    import workloads as W
+    if name == "decode_q_proj_7b":
+        wl = W.decode_q_proj_7b()
+        desc = ("7B decode q_proj: d_in=d_out=4096, 64 tokens (1/seq), 32 resident rank-16 adapters "
+                "drawn Zipf(1.0) from a 1000-adapter catalogue, bf16 weights in 16-row pages, fp32 Y_base")
+    elif name in ("mixed_mlp_up", "mixed_mlp_down"):
+        wl = W.mixed_mlp(which=name.split("_")[-1])
+        desc = f"mixed-rank decode MLP {name.split('_')[-1]}: 256 tokens, 128 resident adapters r in {{8,16,32,64}}, Zipf(1.1)"
+    elif name == "prefill":
+        wl = W.prefill()
+        desc = "prefill: 16 sequences of 128-2048 tokens, d=4096, 6 adapters r in {8,16,32,64}"
+    elif name.startswith("sweep_8b_"):
+        _, _, regime, tt = name.split("_")
+        wl = W.sweep_8b(T=int(tt[1:]), regime=regime)
+        desc = f"8B sweep {regime}: d_in=4096, d_out=14336, rank 64, pool of 512, T={tt[1:]}"
+    else:
+        raise SystemExit(f"unknown workload {name}")
+    return wl, desc
+
+
+def algorithmic_bytes(wl) -> int:
+    """Each distinct adapter read once (A and B, bf16), X read in bf16, Y read and written in fp32."""
+    ids = wl.ids
+    valid = ids[(ids >= 0) & (ids < wl.S)]
+    rk = wl.ranks()
+    distinct = np.unique(valid)
+    w = int(sum(2 * int(rk[i]) * (wl.d_in + wl.d_out) for i in distinct))
+    return w + len(valid) * (2 * wl.d_in + 8 * wl.d_out)
+
+
+def algorithmic_flops(wl) -> int:
+    ids = wl.ids
+    valid = ids[(ids >= 0) & (ids < wl.S)]
+    rk = wl.ranks()
+    return int(sum(2 * int(rk[i]) * (wl.d_in + wl.d_out) for i in valid))
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and --impl reference)
+# ---------------------------------------------------------------------------
+
+def time_oracle(wl, seconds: float):
+    """Run the fp64 C oracle on the workload's batch until `seconds` of work
+    (at least one call); returns (tokens/s per layer, threads, sample text)."""
+    from oracle import build_oracle as OC
+    T = wl.T
+    # bounded sample: whole batch when small, else the first tokens of it
+    n_tok = T
+    est = algorithmic_flops(wl)
+    if est > 4e9:
+        n_tok = max(1, int(T * 4e9 / est))
+    tok = np.arange(n_tok)
+    import workloads as W
+    X, Yb, ids, A, B, sc = W.subset_for_tokens(wl, tok)
+    threads = OC.max_threads()
+    calls = 0
+    t0 = time.perf_counter()
+    while True:
+        OC.lora_apply_c(X, Yb, ids, A, B, sc, nthreads=threads)
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    value = n_tok * calls / el
+    sample = f"{calls} oracle calls of {n_tok} tokens ({wl.name}), {el:.1f} s"
+    return value, threads, sample
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl, desc = workload_spec(args.workload)
+    per_step = []
+    for _ in range(max(args.warmup, 0)):
+        time_oracle(wl, 0.0)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        v, threads, sample = time_oracle(wl, 0.0)
+        per_step.append(v)
+    el = time.perf_counter() - t0
+    value = statistics.median(per_step)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * el / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+class Ring:
+    """L independent layer instances sharing one batch (ids, plan)."""
+
+    def __init__(self, wl, n_layers: int, seed: int, device):
+        import torch
+        import heterogeneous_adapter_batching_b200 as H
+        self.H = H
+        self.wl = wl
+        self.T = wl.T
+        g = torch.Generator(device=device)
+        g.manual_seed(seed)
+        ranks = wl.ranks()
+        self.layers, self.X, self.Y = [], [], []
+        for l in range(n_layers):
+            lay = H.AdapterLayer(wl.d_in, wl.d_out, wl.S, wl.pages_a, wl.pages_b, wl.T, device=device)
+            for i in range(wl.S):
+                r = int(ranks[i])
+                if r <= 0:
+                    continue
+                at = (torch.randn((r, wl.d_in), generator=g, device=device) / math.sqrt(wl.d_in)).to(torch.bfloat16)
+                b = (torch.randn((r, wl.d_out), generator=g, device=device) / math.sqrt(r)).to(torch.bfloat16)
+                lay.load(i, r, 2.0 * r, at, b, page_ids=torch.from_numpy(np.ascontiguousarray(wl.page_ids[i])))
+            self.layers.append(lay)
+            self.X.append((torch.randn((wl.T, wl.d_in), generator=g, device=device) / math.sqrt(wl.d_in)).to(torch.bfloat16))
+            self.Y.append(torch.randn((wl.T, wl.d_out), generator=g, device=device))
+        self.ids = torch.from_numpy(wl.ids.copy()).to(device)
+        self.ws = torch.empty(H.lora_workspace_size(wl.T, wl.S), dtype=torch.uint8, device=device)
+        torch.cuda.synchronize()
+
+    def footprint(self) -> int:
+        lay = self.layers[0]
+        per = (lay.buf_a.numel() * 2 + lay.buf_b.numel() * 2 + self.X[0].numel() * 2 + self.Y[0].numel() * 4)
+        return per * len(self.layers)
+
+    def step(self, stream=None) -> int:
+        """Plan once, apply every layer; returns the number of kernels launched."""
+        H = self.H
+        lay0 = self.layers[0]
+        lay0.plan(self.ids, ws=self.ws, stream=stream)
+        n = H.lora_last_launch_count()
+        for lay, X, Y in zip(self.layers, self.X, self.Y):
+            lay.apply_planned(X, Y, ws=self.ws, stream=stream)
+            n += H.lora_last_launch_count()
+        return n
+
+    def apply_only(self, stream=None) -> int:
+        n = 0
+        for lay, X, Y in zip(self.layers, self.X, self.Y):
+            lay.apply_planned(X, Y, ws=self.ws, stream=stream)
+            n += self.H.lora_last_launch_count()
+        return n
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    import heterogeneous_adapter_batching_b200 as H
+    from heterogeneous_adapter_batching_b200 import build as lib_build
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if rank == 0:
+        lib_build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+        dist.barrier()
+    H.load_library()
+
+    wl, desc = workload_spec(args.workload)
+    per_layer = (wl.pages_a * 16 * wl.d_in * 2 + wl.pages_b * 16 * wl.d_out * 2 + wl.T * (wl.d_in * 2 + wl.d_out * 4))
+    n_layers = args.layers or max(8, min(256, math.ceil(4.2 * L2_BYTES / per_layer)))
+    ring = Ring(wl, n_layers, seed=1234 + rank, device=dev)
+
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+    # capture one step in a CUDA graph
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            ring.step(stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        launches_per_step = ring.step(stream)
+    graph_apply = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_apply, stream=stream):
+        apply_launches = ring.apply_only(stream)
+    torch.cuda.synchronize()
+
+    for _ in range(max(args.warmup, 3)):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream()
+    ev0.record(cur)
+    for _ in range(args.steps):
+        graph.replay()
+    ev1.record(cur)
+    torch.cuda.synchronize()
+    elapsed_ms = ev0.elapsed_time(ev1)
+    # dominant kernel: the fused gather kernel, one launch per layer (plan excluded)
+    for _ in range(3):
+        graph_apply.replay()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    k_apply = max(10, args.steps)
+    a0.record(cur)
+    for _ in range(k_apply):
+        graph_apply.replay()
+    a1.record(cur)
+    torch.cuda.synchronize()
+    apply_ms = a0.elapsed_time(a1)
+    clk = clocks.stop()
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+        dist.barrier()
+
+    T = wl.T
+    tokens_per_step = T * n_layers
+    value = tokens_per_step * world * args.steps / (elapsed_ms / 1000.0)
+    ms_per_step = elapsed_ms / args.steps
+
+    # roofline of the gather kernel (one launch = one layer)
+    per_launch_ms = apply_ms / (k_apply * n_layers)
+    alg = algorithmic_bytes(wl)
+    achieved = alg / (per_launch_ms / 1000.0) / 1e9
+    peak, peak_kind = measured_peaks()
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "traffic": None, "peak_source": peak_kind, "kernel": "gather_kernel<apply>",
+            "kernel_us": per_launch_ms * 1000.0, "algorithmic_bytes_per_launch": alg}
+
+    # end-to-end through the C ABI with host buffers (one layer per step)
+    e2e = None
+    if not args.no_e2e:
+        lay = ring.layers[0]
+        Xh = ring.X[0].cpu().pin_memory()
+        Yh = ring.Y[0].cpu().pin_memory()
+        Ih = ring.ids.cpu().pin_memory()
+        Yout = torch.empty_like(Yh).pin_memory()
+        Xd, Yd, Id = torch.empty_like(ring.X[0]), torch.empty_like(ring.Y[0]), torch.empty_like(ring.ids)
+        with torch.cuda.stream(stream):
+            def e2e_step():
+                Xd.copy_(Xh, non_blocking=True)
+                Yd.copy_(Yh, non_blocking=True)
+                Id.copy_(Ih, non_blocking=True)
+                lay.apply(Xd, Yd, Id, stream=stream)
+                Yout.copy_(Yd, non_blocking=True)
+            for _ in range(5):
+                e2e_step()
+            stream.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            k_e2e = max(20, args.steps)
+            e0.record(stream)
+            for _ in range(k_e2e):
+                e2e_step()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / k_e2e
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = Xh.numel() * 2 + Yh.numel() * 4 + Ih.numel() * 4
+        e2e = {"value": T * world / (e2e_ms / 1000.0), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(Yout.numel() * 4), "ms_per_step": e2e_ms,
+               "path": "pinned H2D of X, Y_base, ids -> lora_apply (plan + fused kernel) -> D2H of Y, one layer"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, threads, sample = time_oracle(wl, args.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample}
+
+    if world > 1:
+        dist.barrier()
+        del graph, graph_apply
+        dist.destroy_process_group()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": desc, "tokens": T, "distinct_adapters": wl.distinct(),
+                       "layers_per_step": n_layers, "plans_per_step": 1,
+                       "l2": f"inputs larger than L2: ring of {n_layers} layer instances, "
+                             f"{ring.footprint() / 1e6:.0f} MB > 4 x 126 MB",
+                       "cuda_graph": True, "parallelism": f"replicas x{world} (no collective)"},
+            "gpu_launches": int(launches_per_step * args.steps),
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

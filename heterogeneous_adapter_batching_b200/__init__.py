@@ -1,0 +1,8 @@
+"""B200-native heterogeneous-batch LoRA adapter branch.
+
+The compute lives in liblora.so (CUDA, sm_100a) behind the C ABI of
+include/lora.h; this package only marshals torch tensors into those calls.
+"""
+from . import _binding
+from ._binding import *  # noqa: F401,F403
+from .layer import AdapterLayer  # noqa: F401

@@ -1,0 +1,228 @@
+"""ctypes binding of liblora (include/lora.h): argument marshalling only.
+
+Every function has the name of the C entry point it calls and takes torch
+tensors (device memory) or plain Python numbers; it passes their pointers
+and sizes through and raises LoraError on a negative return code.  There is
+no fallback: if liblora.so is missing the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblora.so")
+
+LORA_OK = 0
+ERR_NAMES = {
+    -1: "LORA_ERR_INVALID_ARG", -2: "LORA_ERR_BAD_RANK", -3: "LORA_ERR_WIDTH_MISMATCH",
+    -4: "LORA_ERR_POOL_OOM", -5: "LORA_ERR_BAD_SLOT", -6: "LORA_ERR_CUDA", -7: "LORA_ERR_WORKSPACE",
+}
+DEV_ERR_BAD_ID = 1
+DEV_ERR_EMPTY_SLOT = 2
+DEV_ERR_TIMEOUT = 4
+DEV_ERR_BAD_PAGE = 8
+PAGE_ROWS = 16
+MAX_RANK = 64
+MAX_PAGES_PER_MATRIX = 4
+MAX_SLOTS = 4096
+OPT_LONG_SEGMENT = 1
+OPT_DECODE_JOB_TOKENS = 2
+
+EXPORTS = [
+    "lora_pool_create", "lora_pool_destroy", "lora_pool_free_pages", "lora_pool_num_pages",
+    "lora_pool_load", "lora_pool_evict", "lora_pool_read_row", "lora_workspace_size",
+    "lora_plan", "lora_shrink", "lora_expand_add", "lora_apply", "lora_apply_planned",
+    "lora_set_option", "lora_get_option", "lora_last_cuda_error", "lora_last_launch_count",
+]
+
+
+class LoraError(RuntimeError):
+    def __init__(self, name: str, rc: int, detail: str = ""):
+        self.rc = rc
+        super().__init__(f"{name} failed: {ERR_NAMES.get(rc, rc)}{(' (' + detail + ')') if detail else ''}")
+
+
+_lib = None
+V = ctypes.c_void_p
+I = ctypes.c_int
+F = ctypes.c_float
+Z = ctypes.c_size_t
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load liblora.so (raises OSError if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise OSError(f"liblora.so not found at {path}; run heterogeneous_adapter_batching_b200.build.build()")
+    lib = ctypes.CDLL(path)
+    sig = {
+        "lora_pool_create": (I, [V, Z, I, I, ctypes.POINTER(V)]),
+        "lora_pool_destroy": (I, [V]),
+        "lora_pool_free_pages": (I, [V]),
+        "lora_pool_num_pages": (I, [V]),
+        "lora_pool_load": (I, [V, V, I, I, I, F, V, V, V, V, V, V, V]),
+        "lora_pool_evict": (I, [V, V, I, I, V, V, V, V]),
+        "lora_pool_read_row": (I, [V, V, I, I, I, I, V, V]),
+        "lora_workspace_size": (Z, [I, I]),
+        "lora_plan": (I, [V, I, V, I, V, V, V, Z, V, V]),
+        "lora_shrink": (I, [V, I, I, V, I, V, V, V, V, V, Z, V, V]),
+        "lora_expand_add": (I, [V, V, I, I, V, I, V, V, V, V, V, Z, V, V]),
+        "lora_apply": (I, [V, V, I, I, I, V, I, V, V, V, V, V, V, Z, V, V]),
+        "lora_apply_planned": (I, [V, V, I, I, I, I, V, V, V, V, V, V, Z, V, V]),
+        "lora_set_option": (I, [I, I]),
+        "lora_get_option": (I, [I]),
+        "lora_last_cuda_error": (ctypes.c_char_p, []),
+        "lora_last_launch_count": (I, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(name: str, rc: int):
+    if rc != LORA_OK:
+        detail = lora_last_cuda_error() if rc == -6 else ""
+        raise LoraError(name, rc, detail)
+    return rc
+
+
+class Pool:
+    """Host handle of one page pool over a caller-owned device buffer."""
+
+    def __init__(self, handle: int, buf: torch.Tensor, width: int):
+        self.handle = handle
+        self.buf = buf          # keeps the device memory alive
+        self.width = width
+
+    def __del__(self):
+        try:
+            if self.handle and _lib is not None:
+                _lib.lora_pool_destroy(ctypes.c_void_p(self.handle))
+                self.handle = 0
+        except Exception:
+            pass
+
+    @property
+    def _h(self):
+        return ctypes.c_void_p(self.handle)
+
+
+def lora_pool_create(dev_buf: torch.Tensor, width: int, page_rows: int = PAGE_ROWS) -> Pool:
+    lib = load_library()
+    out = ctypes.c_void_p()
+    nbytes = dev_buf.numel() * dev_buf.element_size()
+    _check("lora_pool_create", lib.lora_pool_create(_p(dev_buf), nbytes, width, page_rows, ctypes.byref(out)))
+    return Pool(out.value, dev_buf, width)
+
+
+def lora_pool_destroy(pool: Pool) -> None:
+    if pool.handle:
+        load_library().lora_pool_destroy(pool._h)
+        pool.handle = 0
+
+
+def lora_pool_free_pages(pool: Pool) -> int:
+    return load_library().lora_pool_free_pages(pool._h)
+
+
+def lora_pool_num_pages(pool: Pool) -> int:
+    return load_library().lora_pool_num_pages(pool._h)
+
+
+def lora_pool_load(pa: Pool, pb: Pool, slot: int, num_slots: int, rank: int, alpha: float,
+                   a_t: torch.Tensor, b: torch.Tensor, page_ids: Optional[torch.Tensor],
+                   page_table: torch.Tensor, scales: torch.Tensor, ranks: torch.Tensor, stream=None) -> None:
+    """a_t: [rank, d_in] bf16 (host or device), b: [rank, d_out] bf16; page_ids: host int32 [2, 4] or None."""
+    if page_ids is not None:
+        assert page_ids.device.type == "cpu" and page_ids.dtype == torch.int32 and page_ids.is_contiguous()
+    _check("lora_pool_load", load_library().lora_pool_load(
+        pa._h, pb._h, slot, num_slots, rank, alpha, _p(a_t), _p(b), _p(page_ids),
+        _p(page_table), _p(scales), _p(ranks), _s(stream)))
+
+
+def lora_pool_evict(pa: Pool, pb: Pool, slot: int, num_slots: int, page_table: torch.Tensor,
+                    scales: torch.Tensor, ranks: torch.Tensor, stream=None) -> None:
+    _check("lora_pool_evict", load_library().lora_pool_evict(
+        pa._h, pb._h, slot, num_slots, _p(page_table), _p(scales), _p(ranks), _s(stream)))
+
+
+def lora_pool_read_row(pool: Pool, page_table: torch.Tensor, num_slots: int, slot: int, m: int, k: int,
+                       out: torch.Tensor, stream=None) -> None:
+    _check("lora_pool_read_row", load_library().lora_pool_read_row(
+        pool._h, _p(page_table), num_slots, slot, m, k, _p(out), _s(stream)))
+
+
+def lora_workspace_size(T: int, num_slots: int) -> int:
+    return int(load_library().lora_workspace_size(T, num_slots))
+
+
+def lora_plan(ids, T, ranks, num_slots, perm_out, seg_start_out, ws, err=None, stream=None) -> None:
+    _check("lora_plan", load_library().lora_plan(
+        _p(ids), T, _p(ranks), num_slots, _p(perm_out), _p(seg_start_out), _p(ws),
+        ws.numel() * ws.element_size(), _p(err), _s(stream)))
+
+
+def lora_shrink(X, T, d_in, ids, num_slots, ranks, page_table, pa: Pool, V, ws, err=None, stream=None) -> None:
+    _check("lora_shrink", load_library().lora_shrink(
+        _p(X), T, d_in, _p(ids), num_slots, _p(ranks), _p(page_table), pa._h, _p(V), _p(ws),
+        ws.numel() * ws.element_size(), _p(err), _s(stream)))
+
+
+def lora_expand_add(V, Y, T, d_out, ids, num_slots, ranks, scales, page_table, pb: Pool, ws, err=None,
+                    stream=None) -> None:
+    _check("lora_expand_add", load_library().lora_expand_add(
+        _p(V), _p(Y), T, d_out, _p(ids), num_slots, _p(ranks), _p(scales), _p(page_table), pb._h, _p(ws),
+        ws.numel() * ws.element_size(), _p(err), _s(stream)))
+
+
+def lora_apply(X, Y, T, d_in, d_out, ids, num_slots, ranks, scales, page_table, pa: Pool, pb: Pool, ws,
+               err=None, stream=None) -> None:
+    _check("lora_apply", load_library().lora_apply(
+        _p(X), _p(Y), T, d_in, d_out, _p(ids), num_slots, _p(ranks), _p(scales), _p(page_table),
+        pa._h, pb._h, _p(ws), ws.numel() * ws.element_size(), _p(err), _s(stream)))
+
+
+def lora_apply_planned(X, Y, T, d_in, d_out, num_slots, ranks, scales, page_table, pa: Pool, pb: Pool, ws,
+                       err=None, stream=None) -> None:
+    _check("lora_apply_planned", load_library().lora_apply_planned(
+        _p(X), _p(Y), T, d_in, d_out, num_slots, _p(ranks), _p(scales), _p(page_table),
+        pa._h, pb._h, _p(ws), ws.numel() * ws.element_size(), _p(err), _s(stream)))
+
+
+def lora_set_option(key: int, value: int) -> None:
+    _check("lora_set_option", load_library().lora_set_option(key, value))
+
+
+def lora_get_option(key: int) -> int:
+    return int(load_library().lora_get_option(key))
+
+
+def lora_last_cuda_error() -> str:
+    return load_library().lora_last_cuda_error().decode()
+
+
+def lora_last_launch_count() -> int:
+    return int(load_library().lora_last_launch_count())

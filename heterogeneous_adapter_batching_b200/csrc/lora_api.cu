@@ -1,0 +1,400 @@
+// C-ABI entry points of liblora: page pools, argument validation, workspace
+// layout and the launch sequence of each call.  See include/lora.h for the
+// contract of every function.
+#include <atomic>
+#include <cstring>
+
+#include "lora_internal.cuh"
+
+namespace lora {
+
+namespace {
+std::atomic<int> g_long_segment{16};
+std::atomic<int> g_job_tokens{4};
+thread_local int t_launches = 0;
+thread_local const char *t_last_cuda_error = "no error";
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Writes one slot's table row: page ids of A and B, scale and rank.
+__global__ void set_slot_kernel(int32_t *pt, float *scale, int32_t *rank, int slot, int4 pa, int4 pb,
+                                float s, int r) {
+    if (threadIdx.x == 0) {
+        int32_t *row = pt + (size_t)slot * 2 * LORA_MAX_PAGES_PER_MATRIX;
+        row[0] = pa.x; row[1] = pa.y; row[2] = pa.z; row[3] = pa.w;
+        row[4] = pb.x; row[5] = pb.y; row[6] = pb.z; row[7] = pb.w;
+        scale[slot] = s;
+        rank[slot] = r;
+    }
+}
+
+// Resolves (slot, matrix, rank-row) through the page table and copies the row.
+__global__ void read_row_kernel(const uint16_t *pool, int width, const int32_t *pt, int slot, int m, int k,
+                                uint16_t *out) {
+    const int page = pt[((size_t)slot * 2 + m) * LORA_MAX_PAGES_PER_MATRIX + k / LORA_PAGE_ROWS];
+    const uint16_t *row = pool + ((size_t)page * LORA_PAGE_ROWS + (k % LORA_PAGE_ROWS)) * width;
+    for (int c = threadIdx.x + blockIdx.x * blockDim.x; c < width; c += blockDim.x * gridDim.x) out[c] = row[c];
+}
+}  // namespace
+
+int opt_long_segment() { return g_long_segment.load(); }
+int opt_job_tokens() { return g_job_tokens.load(); }
+
+int cuda_check(cudaError_t e) {
+    if (e == cudaSuccess) return LORA_OK;
+    t_last_cuda_error = cudaGetErrorString(e);
+    return LORA_ERR_CUDA;
+}
+void count_launch(int n) { t_launches += n; }
+void reset_launch_count() { t_launches = 0; }
+
+// Page allocation helpers (caller holds the pool mutex).
+static int take_pages(lora_pool_s *p, int n, const int32_t *want, std::vector<int> &got) {
+    got.clear();
+    if (want) {
+        for (int i = 0; i < n; ++i) {
+            const int id = want[i];
+            if (id < 0 || id >= p->num_pages || p->used[id]) return LORA_ERR_BAD_SLOT;
+            for (int j = 0; j < i; ++j)
+                if (want[j] == id) return LORA_ERR_BAD_SLOT;
+        }
+        for (int i = 0; i < n; ++i) {
+            p->used[want[i]] = 1;
+            got.push_back(want[i]);
+        }
+        // drop the taken ids from the free stack
+        std::vector<int> keep;
+        keep.reserve(p->free_stack.size());
+        for (int id : p->free_stack)
+            if (!p->used[id]) keep.push_back(id);
+        p->free_stack.swap(keep);
+        return LORA_OK;
+    }
+    if ((int)p->free_stack.size() < n) return LORA_ERR_POOL_OOM;
+    for (int i = 0; i < n; ++i) {
+        const int id = p->free_stack.back();
+        p->free_stack.pop_back();
+        p->used[id] = 1;
+        got.push_back(id);
+    }
+    return LORA_OK;
+}
+
+static void give_pages(lora_pool_s *p, const std::vector<int> &pages) {
+    for (int id : pages) {
+        if (id >= 0 && id < p->num_pages && p->used[id]) {
+            p->used[id] = 0;
+            p->free_stack.push_back(id);
+        }
+    }
+}
+
+}  // namespace lora
+
+using namespace lora;
+
+extern "C" {
+
+int lora_pool_create(void *dev_buf, size_t bytes, int width, int page_rows, lora_pool_t *out) {
+    if (!out || !dev_buf || width <= 0 || (width % 8) != 0 || page_rows != LORA_PAGE_ROWS) return LORA_ERR_INVALID_ARG;
+    if (!aligned(dev_buf, 256)) return LORA_ERR_INVALID_ARG;
+    const size_t page_bytes = (size_t)page_rows * width * 2;
+    const size_t np = bytes / page_bytes;
+    if (np < 1 || np > (size_t)INT32_MAX / LORA_PAGE_ROWS) return LORA_ERR_INVALID_ARG;
+    lora_pool_s *p = new lora_pool_s();
+    p->base = static_cast<uint16_t *>(dev_buf);
+    p->bytes = bytes;
+    p->width = width;
+    p->page_rows = page_rows;
+    p->num_pages = (int)np;
+    p->used.assign(np, 0);
+    p->free_stack.reserve(np);
+    for (int i = (int)np - 1; i >= 0; --i) p->free_stack.push_back(i);  // pop order 0, 1, 2, ...
+    *out = p;
+    return LORA_OK;
+}
+
+int lora_pool_destroy(lora_pool_t pool) {
+    delete pool;
+    return LORA_OK;
+}
+
+int lora_pool_free_pages(lora_pool_t pool) {
+    if (!pool) return -1;
+    std::lock_guard<std::mutex> g(pool->mu);
+    return (int)pool->free_stack.size();
+}
+
+int lora_pool_num_pages(lora_pool_t pool) { return pool ? pool->num_pages : -1; }
+
+int lora_pool_load(lora_pool_t pa, lora_pool_t pb, int slot, int num_slots, int rank, float alpha,
+                   const uint16_t *a_t, const uint16_t *b, const int32_t *page_ids,
+                   int32_t *page_table_dev, float *scale_dev, int32_t *rank_dev, lora_stream_t stream) {
+    if (!pa || !pb || !a_t || !b || !page_table_dev || !scale_dev || !rank_dev) return LORA_ERR_INVALID_ARG;
+    if (num_slots < 1 || num_slots > LORA_MAX_SLOTS) return LORA_ERR_INVALID_ARG;
+    if (slot < 0 || slot >= num_slots) return LORA_ERR_BAD_SLOT;
+    if (rank < 1 || rank > LORA_MAX_RANK) return LORA_ERR_BAD_RANK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int np = (rank + LORA_PAGE_ROWS - 1) / LORA_PAGE_ROWS;
+    lora_pool_s *pools[2] = {pa, pb};
+    const uint16_t *src[2] = {a_t, b};
+    std::vector<int> got[2];
+    // Lock both pools (in address order when distinct) for the allocation.
+    std::unique_lock<std::mutex> l1, l2;
+    if (pa == pb) {
+        l1 = std::unique_lock<std::mutex>(pa->mu);
+    } else if (pa < pb) {
+        l1 = std::unique_lock<std::mutex>(pa->mu);
+        l2 = std::unique_lock<std::mutex>(pb->mu);
+    } else {
+        l1 = std::unique_lock<std::mutex>(pb->mu);
+        l2 = std::unique_lock<std::mutex>(pa->mu);
+    }
+    for (int m = 0; m < 2; ++m)
+        if (pools[m]->owners.count(std::make_tuple((const void *)page_table_dev, slot, m))) return LORA_ERR_BAD_SLOT;
+    for (int m = 0; m < 2; ++m) {
+        int rc = take_pages(pools[m], np, page_ids ? page_ids + m * LORA_MAX_PAGES_PER_MATRIX : nullptr, got[m]);
+        if (rc) {
+            if (m == 1) give_pages(pools[0], got[0]);
+            return rc;
+        }
+    }
+    int rc = LORA_OK;
+    for (int m = 0; m < 2 && rc == LORA_OK; ++m) {
+        lora_pool_s *p = pools[m];
+        const size_t row_bytes = (size_t)p->width * 2;
+        for (int q = 0; q < np && rc == LORA_OK; ++q) {
+            const int rows = (rank - q * LORA_PAGE_ROWS) < LORA_PAGE_ROWS ? (rank - q * LORA_PAGE_ROWS) : LORA_PAGE_ROWS;
+            char *dst = reinterpret_cast<char *>(p->base) + (size_t)got[m][q] * LORA_PAGE_ROWS * row_bytes;
+            const char *s = reinterpret_cast<const char *>(src[m]) + (size_t)q * LORA_PAGE_ROWS * row_bytes;
+            rc = cuda_check(cudaMemcpyAsync(dst, s, rows * row_bytes, cudaMemcpyDefault, st));
+            if (rc == LORA_OK && rows < LORA_PAGE_ROWS)
+                rc = cuda_check(cudaMemsetAsync(dst + rows * row_bytes, 0, (LORA_PAGE_ROWS - rows) * row_bytes, st));
+        }
+    }
+    if (rc != LORA_OK) {
+        give_pages(pools[0], got[0]);
+        give_pages(pools[1], got[1]);
+        return rc;
+    }
+    int32_t ids[2][4] = {{-1, -1, -1, -1}, {-1, -1, -1, -1}};
+    for (int m = 0; m < 2; ++m)
+        for (int q = 0; q < np; ++q) ids[m][q] = got[m][q];
+    set_slot_kernel<<<1, 32, 0, st>>>(page_table_dev, scale_dev, rank_dev, slot,
+                                      make_int4(ids[0][0], ids[0][1], ids[0][2], ids[0][3]),
+                                      make_int4(ids[1][0], ids[1][1], ids[1][2], ids[1][3]),
+                                      alpha / (float)rank, rank);
+    rc = cuda_check(cudaGetLastError());
+    if (rc != LORA_OK) {
+        give_pages(pools[0], got[0]);
+        give_pages(pools[1], got[1]);
+        return rc;
+    }
+    for (int m = 0; m < 2; ++m) pools[m]->owners[std::make_tuple((const void *)page_table_dev, slot, m)] = got[m];
+    return LORA_OK;
+}
+
+int lora_pool_evict(lora_pool_t pa, lora_pool_t pb, int slot, int num_slots, int32_t *page_table_dev,
+                    float *scale_dev, int32_t *rank_dev, lora_stream_t stream) {
+    if (!pa || !pb || !page_table_dev || !scale_dev || !rank_dev) return LORA_ERR_INVALID_ARG;
+    if (num_slots < 1 || num_slots > LORA_MAX_SLOTS) return LORA_ERR_INVALID_ARG;
+    if (slot < 0 || slot >= num_slots) return LORA_ERR_BAD_SLOT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    lora_pool_s *pools[2] = {pa, pb};
+    std::unique_lock<std::mutex> l1, l2;
+    if (pa == pb) {
+        l1 = std::unique_lock<std::mutex>(pa->mu);
+    } else if (pa < pb) {
+        l1 = std::unique_lock<std::mutex>(pa->mu);
+        l2 = std::unique_lock<std::mutex>(pb->mu);
+    } else {
+        l1 = std::unique_lock<std::mutex>(pb->mu);
+        l2 = std::unique_lock<std::mutex>(pa->mu);
+    }
+    bool found = false;
+    for (int m = 0; m < 2; ++m) {
+        auto key = std::make_tuple((const void *)page_table_dev, slot, m);
+        auto it = pools[m]->owners.find(key);
+        if (it != pools[m]->owners.end()) {
+            found = true;
+            give_pages(pools[m], it->second);
+            pools[m]->owners.erase(it);
+        }
+    }
+    if (!found) return LORA_ERR_BAD_SLOT;
+    set_slot_kernel<<<1, 32, 0, st>>>(page_table_dev, scale_dev, rank_dev, slot, make_int4(-1, -1, -1, -1),
+                                      make_int4(-1, -1, -1, -1), 0.f, 0);
+    return cuda_check(cudaGetLastError());
+}
+
+int lora_pool_read_row(lora_pool_t pool, const int32_t *page_table_dev, int num_slots, int slot, int m, int k,
+                       uint16_t *out_dev, lora_stream_t stream) {
+    if (!pool || !page_table_dev || !out_dev || m < 0 || m > 1 || k < 0 || k >= LORA_MAX_RANK) return LORA_ERR_INVALID_ARG;
+    if (slot < 0 || slot >= num_slots) return LORA_ERR_BAD_SLOT;
+    {
+        std::lock_guard<std::mutex> g(pool->mu);
+        auto it = pool->owners.find(std::make_tuple((const void *)page_table_dev, slot, m));
+        if (it == pool->owners.end() || k >= (int)it->second.size() * LORA_PAGE_ROWS) return LORA_ERR_BAD_SLOT;
+    }
+    read_row_kernel<<<4, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(pool->base, pool->width, page_table_dev,
+                                                                           slot, m, k, out_dev);
+    return cuda_check(cudaGetLastError());
+}
+
+size_t lora_workspace_size(int T, int num_slots) {
+    if (T < 0 || num_slots < 1) return 0;
+    return ws_layout(T, num_slots).total;
+}
+
+static int check_common(int T, int num_slots, const int32_t *ids, const int32_t *ranks, void *ws, size_t ws_bytes) {
+    if (T < 0 || num_slots < 1 || num_slots > LORA_MAX_SLOTS) return LORA_ERR_INVALID_ARG;
+    if (T > 0 && (!ids || !ranks)) return LORA_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < ws_layout(T, num_slots).total || !aligned(ws, 256)) return LORA_ERR_WORKSPACE;
+    return LORA_OK;
+}
+
+static PlanOut plan_out(void *ws, int T, int S, int32_t *perm_out, int32_t *seg_out) {
+    const WsLayout l = ws_layout(T, S);
+    char *b = static_cast<char *>(ws);
+    PlanOut o;
+    o.header = reinterpret_cast<PlanHeader *>(b + l.header);
+    o.seg_start = reinterpret_cast<int32_t *>(b + l.seg_start);
+    o.perm = reinterpret_cast<int32_t *>(b + l.perm);
+    o.jobs = reinterpret_cast<int4 *>(b + l.jobs);
+    o.tiles = reinterpret_cast<int4 *>(b + l.tiles);
+    o.perm_copy = perm_out;
+    o.seg_start_copy = seg_out;
+    return o;
+}
+
+static bool plan_uses_tiles(int T) {
+    return tiles_supported() && opt_long_segment() > 0 && T >= opt_long_segment();
+}
+
+static int run_planned(const uint16_t *X, float *Y, int T, int d_in, int d_out, int num_slots,
+                       const int32_t *ranks, const float *scales, const int32_t *page_table, lora_pool_t pa,
+                       lora_pool_t pb, void *ws, int32_t *err_dev, cudaStream_t st) {
+    const PlanOut o = plan_out(ws, T, num_slots, nullptr, nullptr);
+    GatherArgs a = {};
+    a.X = X; a.Y = Y; a.T = T; a.d_in = d_in; a.d_out = d_out;
+    a.ranks = ranks; a.scales = scales; a.pt = page_table; a.poolA = pa->base; a.poolB = pb->base;
+    a.perm = o.perm; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
+    a.rowsA = (long long)pa->num_pages * LORA_PAGE_ROWS; a.rowsB = (long long)pb->num_pages * LORA_PAGE_ROWS;
+    if (int rc = launch_gather(kApply, a, st, true)) return rc;
+    if (plan_uses_tiles(T)) {
+        TileArgs ta = {};
+        ta.X = X; ta.Y = Y; ta.T = T; ta.d_in = d_in; ta.d_out = d_out;
+        ta.ranks = ranks; ta.scales = scales; ta.pt = page_table; ta.pa = pa; ta.pb = pb;
+        ta.tiles = o.tiles; ta.hdr = o.header; ta.err = err_dev;
+        ta.rowsA = a.rowsA; ta.rowsB = a.rowsB; ta.long_thresh = opt_long_segment();
+        if (int rc = launch_tiles(ta, st, true)) return rc;
+    }
+    return LORA_OK;
+}
+
+int lora_plan(const int32_t *ids, int T, const int32_t *ranks, int num_slots, int32_t *perm_out,
+              int32_t *seg_start_out, void *ws, size_t ws_bytes, int32_t *err_dev, lora_stream_t stream) {
+    reset_launch_count();
+    if (int rc = check_common(T, num_slots, ids, ranks, ws, ws_bytes)) return rc;
+    const PlanOut o = plan_out(ws, T, num_slots, perm_out, seg_start_out);
+    return launch_plan(ids, T, ranks, num_slots, plan_uses_tiles(T) ? opt_long_segment() : 0, opt_job_tokens(),
+                       o, err_dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int lora_apply_planned(const uint16_t *X, float *Y, int T, int d_in, int d_out, int num_slots, const int32_t *ranks,
+                       const float *scales, const int32_t *page_table, lora_pool_t pa, lora_pool_t pb, void *ws,
+                       size_t ws_bytes, int32_t *err_dev, lora_stream_t stream) {
+    reset_launch_count();
+    if (T < 0 || num_slots < 1 || num_slots > LORA_MAX_SLOTS || !ranks) return LORA_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < ws_layout(T, num_slots).total || !aligned(ws, 256)) return LORA_ERR_WORKSPACE;
+    if (!pa || !pb) return LORA_ERR_INVALID_ARG;
+    if (pa->width != d_in || pb->width != d_out) return LORA_ERR_WIDTH_MISMATCH;
+    if (T == 0) return LORA_OK;
+    if (!X || !Y || !scales || !page_table || !aligned(X, 16) || !aligned(Y, 16)) return LORA_ERR_INVALID_ARG;
+    return run_planned(X, Y, T, d_in, d_out, num_slots, ranks, scales, page_table, pa, pb, ws, err_dev,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int lora_shrink(const uint16_t *X, int T, int d_in, const int32_t *ids, int num_slots, const int32_t *ranks,
+                const int32_t *page_table, lora_pool_t pa, float *V, void *ws, size_t ws_bytes, int32_t *err_dev,
+                lora_stream_t stream) {
+    reset_launch_count();
+    if (int rc = check_common(T, num_slots, ids, ranks, ws, ws_bytes)) return rc;
+    if (!pa) return LORA_ERR_INVALID_ARG;
+    if (pa->width != d_in) return LORA_ERR_WIDTH_MISMATCH;
+    if (T == 0) return LORA_OK;
+    if (!X || !V || !page_table || !aligned(X, 16)) return LORA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const PlanOut o = plan_out(ws, T, num_slots, nullptr, nullptr);
+    if (int rc = launch_plan(ids, T, ranks, num_slots, 0, opt_job_tokens(), o, err_dev, st)) return rc;
+    GatherArgs a = {};
+    a.X = X; a.V = V; a.T = T; a.d_in = d_in; a.d_out = 8;
+    a.ranks = ranks; a.pt = page_table; a.poolA = pa->base;
+    a.perm = o.perm; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
+    a.rowsA = (long long)pa->num_pages * LORA_PAGE_ROWS;
+    return launch_gather(kShrink, a, st, true);
+}
+
+int lora_expand_add(const float *V, float *Y, int T, int d_out, const int32_t *ids, int num_slots,
+                    const int32_t *ranks, const float *scales, const int32_t *page_table, lora_pool_t pb, void *ws,
+                    size_t ws_bytes, int32_t *err_dev, lora_stream_t stream) {
+    reset_launch_count();
+    if (int rc = check_common(T, num_slots, ids, ranks, ws, ws_bytes)) return rc;
+    if (!pb) return LORA_ERR_INVALID_ARG;
+    if (pb->width != d_out) return LORA_ERR_WIDTH_MISMATCH;
+    if (T == 0) return LORA_OK;
+    if (!V || !Y || !scales || !page_table || !aligned(Y, 16)) return LORA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const PlanOut o = plan_out(ws, T, num_slots, nullptr, nullptr);
+    if (int rc = launch_plan(ids, T, ranks, num_slots, 0, opt_job_tokens(), o, err_dev, st)) return rc;
+    GatherArgs a = {};
+    a.V = const_cast<float *>(V); a.Y = Y; a.T = T; a.d_in = 8; a.d_out = d_out;
+    a.ranks = ranks; a.scales = scales; a.pt = page_table; a.poolB = pb->base;
+    a.perm = o.perm; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
+    a.rowsB = (long long)pb->num_pages * LORA_PAGE_ROWS;
+    return launch_gather(kExpand, a, st, true);
+}
+
+int lora_apply(const uint16_t *X, float *Y, int T, int d_in, int d_out, const int32_t *ids, int num_slots,
+               const int32_t *ranks, const float *scales, const int32_t *page_table, lora_pool_t pa, lora_pool_t pb,
+               void *ws, size_t ws_bytes, int32_t *err_dev, lora_stream_t stream) {
+    reset_launch_count();
+    if (int rc = check_common(T, num_slots, ids, ranks, ws, ws_bytes)) return rc;
+    if (!pa || !pb) return LORA_ERR_INVALID_ARG;
+    if (pa->width != d_in || pb->width != d_out) return LORA_ERR_WIDTH_MISMATCH;
+    if (T == 0) return LORA_OK;
+    if (!X || !Y || !scales || !page_table || !aligned(X, 16) || !aligned(Y, 16)) return LORA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const PlanOut o = plan_out(ws, T, num_slots, nullptr, nullptr);
+    const int long_thresh = plan_uses_tiles(T) ? opt_long_segment() : 0;
+    if (int rc = launch_plan(ids, T, ranks, num_slots, long_thresh, opt_job_tokens(), o, err_dev, st)) return rc;
+    return run_planned(X, Y, T, d_in, d_out, num_slots, ranks, scales, page_table, pa, pb, ws, err_dev, st);
+}
+
+int lora_set_option(int key, int value) {
+    switch (key) {
+        case LORA_OPT_LONG_SEGMENT:
+            if (value < 0) return LORA_ERR_INVALID_ARG;
+            g_long_segment.store(value);
+            return LORA_OK;
+        case LORA_OPT_DECODE_JOB_TOKENS:
+            if (value < 1 || value > 4) return LORA_ERR_INVALID_ARG;
+            g_job_tokens.store(value);
+            return LORA_OK;
+    }
+    return LORA_ERR_INVALID_ARG;
+}
+
+int lora_get_option(int key) {
+    switch (key) {
+        case LORA_OPT_LONG_SEGMENT: return g_long_segment.load();
+        case LORA_OPT_DECODE_JOB_TOKENS: return g_job_tokens.load();
+    }
+    return LORA_ERR_INVALID_ARG;
+}
+
+const char *lora_last_cuda_error(void) { return t_last_cuda_error; }
+
+int lora_last_launch_count(void) { return t_launches; }
+
+}  // extern "C"

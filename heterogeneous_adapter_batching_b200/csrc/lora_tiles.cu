@@ -1,0 +1,462 @@
+// Tensor-core path for long contiguous segments (prefill).
+//
+// Page "Multi-LoRA Serving in Production" (llms.blog), section "Multi-Size
+// Batched Gather Kernels (MBGMV and MBGMM)": in prefill a sequence brings a
+// variable-length chunk of tokens that all use one adapter, and the kernel
+// indexes that adapter's rank-specific weights dynamically.  Section
+// "Segmented Gather Matrix-Vector Multiplication (SGMV)": shrink v = x A on
+// the tensor cores, then expand v B scaled by alpha/r into the base output.
+//
+// Work unit = (tile, part): a tile is up to 128 consecutive tokens of one
+// segment (from the plan kernel) and a part is a slice of d_out in units of
+// 64 columns; the parts of one tile run on different CTAs when there are too
+// few tiles to fill the GPU (each recomputes the small shrink of its tile).
+// One CTA per SM, persistent over the units, warp-specialised:
+//   warp 0     TMA producer of the shrink operands: X tile [128 x 64] and the
+//              adapter's A^T pages [16 x 64] per page, 128-byte swizzled;
+//   warp 1     TMA producer of the expand operands: B pages [16 x 64] of the
+//              current 64-column n-tile and the Y tile [128 x 64] fp32;
+//   warp 2     allocates tensor memory and issues tcgen05.mma:
+//                shrink  D1[128 x N1] = X[128 x d_in] A[d_in x N1]   (N1 = r rounded up to 16)
+//                expand  D2[128 x 64] = V[128 x N1] B[N1 x 64]        (B read MN-major)
+//   warps 4-7  epilogue: read D1 from tensor memory, round v to bf16 into a
+//              swizzled shared tile (the A operand of the expand), then per
+//              n-tile read D2, add s * D2 to the Y tile and write it back with
+//              a TMA store (or row stores for a tile with fewer than 128 tokens).
+// Pages hold 16 rank-rows; ranks that are not a multiple of 16 read the
+// zero-filled rows of their last page, so padding exists only inside the
+// page and in shared memory, never in the pool.  Every mbarrier wait is
+// bounded (LORA_DEV_ERR_TIMEOUT).  No cluster multicast is used.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "lora_internal.cuh"
+
+namespace lora {
+namespace {
+
+constexpr int kM = 128;              // tokens per tile (MMA M)
+constexpr int kKB = 64;              // shrink K block: one 128-byte swizzle row of bf16
+constexpr int kNB = 64;              // expand n-tile width (MMA N)
+constexpr int kStages = 4;           // shrink pipeline depth
+constexpr int kThreads = 256;
+constexpr uint32_t kTmemCols = 256;  // D1 [0,64), D2[0] [64,128), D2[1] [128,192)
+constexpr long long kWaitLimit = 2000000000LL;
+
+struct TileSmem {
+    __nv_bfloat16 xs[kStages][kM * kKB];      // 16 KB each, K-major SW128
+    __nv_bfloat16 as[kStages][64 * kKB];      //  8 KB each, up to 4 pages x 16 rows
+    __nv_bfloat16 vs[kM * 64];                // 16 KB, V (expand A operand), K-major SW128
+    __nv_bfloat16 bs[2][64 * kNB];            //  8 KB each, B n-tile, rank rows x 64 cols (MN-major SW128)
+    float ys[2][kM * kNB];                    // 32 KB each, two SW128 boxes of [128 rows x 32 cols]
+    uint64_t full[kStages], empty[kStages];
+    uint64_t bfull[2], bempty[2], yfull[2], yempty[2], accfull[2], accempty[2];
+    uint64_t shrink_done, d1_empty, v_ready, v_empty;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ uint32_t su32(const void *p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+
+__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t n) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(n));
+}
+__device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t par) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(a), "r"(par) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ void mbar_wait(uint64_t *b, uint32_t par, TileSmem &sm, int32_t *err) {
+    const uint32_t a = su32(b);
+    if (mbar_try(a, par)) return;
+    const long long t0 = clock64();
+    while (!mbar_try(a, par)) {
+        if (*(volatile int *)&sm.abort) return;
+        if (clock64() - t0 > kWaitLimit) {
+            *(volatile int *)&sm.abort = 1;
+            if (err) atomicOr(err, LORA_DEV_ERR_TIMEOUT);
+            return;
+        }
+    }
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void tma_load(void *dst, const CUtensorMap *m, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(su32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(su32(bar)) : "memory");
+}
+__device__ __forceinline__ void tma_store(const CUtensorMap *m, int x, int y, const void *src) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];"
+                 ::"l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(su32(src)) : "memory");
+}
+
+// tcgen05 shared-memory matrix descriptor, 128-byte swizzle (layout type 2),
+// descriptor version 1, base offset 0 (atoms are 1024-byte aligned).
+__device__ __forceinline__ uint64_t sdesc(const void *p, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((su32(p) >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// Instruction descriptor of kind::f16: bf16 x bf16 -> fp32.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar)) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+#define TMEM_LD16(taddr, r)                                                                                   \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];" \
+                 : "=f"(r[0]), "=f"(r[1]), "=f"(r[2]), "=f"(r[3]), "=f"(r[4]), "=f"(r[5]), "=f"(r[6]), "=f"(r[7]),     \
+                   "=f"(r[8]), "=f"(r[9]), "=f"(r[10]), "=f"(r[11]), "=f"(r[12]), "=f"(r[13]), "=f"(r[14]), "=f"(r[15]) \
+                 : "r"(taddr))
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+struct UnitInfo {
+    int slot, row0, ntok, r, n1, np, j0, j1;
+    bool skip;
+};
+
+__device__ __forceinline__ UnitInfo unit_info(const TileArgs &a, int u, int P, int nj) {
+    UnitInfo ui;
+    const int tile = u / P, part = u - tile * P;
+    const int4 t = a.tiles[tile];
+    ui.slot = t.x;
+    ui.row0 = t.y;
+    ui.ntok = t.z;
+    ui.j0 = (int)((long long)nj * part / P);
+    ui.j1 = (int)((long long)nj * (part + 1) / P);
+    int r = a.ranks[ui.slot];
+    bool bad = r <= 0 || r > LORA_MAX_RANK;
+    const int np = bad ? 0 : (r + 15) >> 4;
+    for (int p = 0; p < np; ++p) {
+        const int pa = a.pt[ui.slot * 8 + p], pb = a.pt[ui.slot * 8 + 4 + p];
+        if (pa < 0 || (long long)(pa + 1) * LORA_PAGE_ROWS > a.rowsA) bad = true;
+        if (pb < 0 || (long long)(pb + 1) * LORA_PAGE_ROWS > a.rowsB) bad = true;
+    }
+    ui.skip = bad || ui.j0 >= ui.j1;
+    ui.r = bad ? 0 : r;
+    ui.np = bad ? 0 : np;
+    ui.n1 = ui.np * 16;
+    return ui;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmA,
+             const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmY, TileArgs a) {
+    extern __shared__ unsigned char smem_raw[];
+    TileSmem &sm = *reinterpret_cast<TileSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], 1); }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.bfull[b], 1); mbar_init(&sm.bempty[b], 1);
+            mbar_init(&sm.yfull[b], 1); mbar_init(&sm.yempty[b], 1);
+            mbar_init(&sm.accfull[b], 1); mbar_init(&sm.accempty[b], 128);
+        }
+        mbar_init(&sm.shrink_done, 1);
+        mbar_init(&sm.d1_empty, 128);
+        mbar_init(&sm.v_ready, 128);
+        mbar_init(&sm.v_empty, 1);
+        sm.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 2) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&sm.tmem_base)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    // The kernels before this one on the stream produce the plan.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    const int n_tiles = a.hdr->n_tiles;
+    const int nj = (a.d_out + kNB - 1) / kNB;
+    const int nkb = (a.d_in + kKB - 1) / kKB;
+    int P = n_tiles > 0 ? (int)((gridDim.x + n_tiles - 1) / n_tiles) : 1;
+    P = P < 1 ? 1 : (P > nj ? nj : P);
+    const int n_units = n_tiles * P;
+
+    if (warp == 0 && lane == 0) {
+        // ---------------- shrink operand producer ----------------
+        int it = 0;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+            const UnitInfo ui = unit_info(a, u, P, nj);
+            if (ui.skip) continue;
+            int pg[4];
+            for (int p = 0; p < 4; ++p) pg[p] = p < ui.np ? a.pt[ui.slot * 8 + p] : 0;
+            for (int kb = 0; kb < nkb; ++kb, ++it) {
+                const int s = it % kStages;
+                mbar_wait(&sm.empty[s], ((it / kStages) & 1) ^ 1, sm, a.err);
+                mbar_expect_tx(&sm.full[s], (uint32_t)(kM * kKB * 2 + ui.np * 16 * kKB * 2));
+                tma_load(sm.xs[s], &tmX, kb * kKB, ui.row0, &sm.full[s]);
+                for (int p = 0; p < ui.np; ++p)
+                    tma_load(&sm.as[s][p * 16 * kKB], &tmA, kb * kKB, pg[p] * LORA_PAGE_ROWS, &sm.full[s]);
+            }
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ---------------- expand operand producer ----------------
+        int it = 0;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+            const UnitInfo ui = unit_info(a, u, P, nj);
+            if (ui.skip) continue;
+            int pg[4];
+            for (int p = 0; p < 4; ++p) pg[p] = p < ui.np ? a.pt[ui.slot * 8 + 4 + p] : 0;
+            for (int j = ui.j0; j < ui.j1; ++j, ++it) {
+                const int b = it & 1;
+                const uint32_t par = ((it >> 1) & 1) ^ 1;
+                mbar_wait(&sm.bempty[b], par, sm, a.err);
+                mbar_expect_tx(&sm.bfull[b], (uint32_t)(ui.np * 16 * kNB * 2));
+                for (int p = 0; p < ui.np; ++p)
+                    tma_load(&sm.bs[b][p * 16 * kNB], &tmB, j * kNB, pg[p] * LORA_PAGE_ROWS, &sm.bfull[b]);
+                mbar_wait(&sm.yempty[b], par, sm, a.err);
+                mbar_expect_tx(&sm.yfull[b], (uint32_t)(kM * kNB * 4));
+                tma_load(&sm.ys[b][0], &tmY, j * kNB, ui.row0, &sm.yfull[b]);
+                tma_load(&sm.ys[b][kM * 32], &tmY, j * kNB + 32, ui.row0, &sm.yfull[b]);
+            }
+        }
+    } else if (warp == 2 && lane == 0) {
+        // ---------------- MMA issuer ----------------
+        int it = 0, ite = 0, itt = 0;
+        const uint32_t idesc2 = idesc_bf16(kM, kNB, 0, 1);
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+            const UnitInfo ui = unit_info(a, u, P, nj);
+            if (ui.skip) continue;
+            const uint32_t idesc1 = idesc_bf16(kM, ui.n1, 0, 0);
+            // shrink: D1 = X A over all K blocks
+            mbar_wait(&sm.d1_empty, (itt & 1) ^ 1, sm, a.err);
+            tc_fence_after();
+            for (int kb = 0; kb < nkb; ++kb, ++it) {
+                const int s = it % kStages;
+                mbar_wait(&sm.full[s], (it / kStages) & 1, sm, a.err);
+                tc_fence_after();
+                const uint64_t da = sdesc(sm.xs[s], 16, 1024);
+                const uint64_t db = sdesc(sm.as[s], 16, 1024);
+#pragma unroll
+                for (int k = 0; k < kKB / 16; ++k)
+                    mma_bf16(tmem, da + (uint64_t)(k * 2), db + (uint64_t)(k * 2), idesc1, (kb | k) != 0);
+                mma_commit(&sm.empty[s]);
+            }
+            mma_commit(&sm.shrink_done);
+            // expand: one 64-column n-tile at a time into a double-buffered accumulator
+            mbar_wait(&sm.v_ready, itt & 1, sm, a.err);
+            tc_fence_after();
+            const uint64_t dv = sdesc(sm.vs, 16, 1024);
+            for (int j = ui.j0; j < ui.j1; ++j, ++ite) {
+                const int b = ite & 1;
+                const uint32_t par = (ite >> 1) & 1;
+                mbar_wait(&sm.accempty[b], par ^ 1, sm, a.err);
+                mbar_wait(&sm.bfull[b], par, sm, a.err);
+                tc_fence_after();
+                const uint64_t dbb = sdesc(sm.bs[b], (uint32_t)(ui.n1 * 128), 1024);
+                for (int k = 0; k < ui.np; ++k)
+                    mma_bf16(tmem + 64 + 64 * b, dv + (uint64_t)(k * 2), dbb + (uint64_t)(k * (2048 >> 4)), idesc2,
+                             k != 0);
+                mma_commit(&sm.bempty[b]);
+                mma_commit(&sm.accfull[b]);
+            }
+            mma_commit(&sm.v_empty);
+            ++itt;
+        }
+    } else if (warp >= 4) {
+        // ---------------- epilogue ----------------
+        const int q = warp & 3;              // tensor-memory lane quarter of this warp
+        const int m = q * 32 + lane;         // tile row = accumulator lane
+        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+        const bool leader = (warp == 4 && lane == 0);
+        int ite = 0, itt = 0;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+            const UnitInfo ui = unit_info(a, u, P, nj);
+            if (ui.skip) continue;
+            const float sc = a.scales[ui.slot];
+            // v = D1 row m, rounded to bf16 into the swizzled V tile
+            mbar_wait(&sm.shrink_done, itt & 1, sm, a.err);
+            tc_fence_after();
+            float d1[64];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if (c < ui.np) TMEM_LD16(trow + c * 16, (&d1[c * 16]));
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&sm.d1_empty);
+            mbar_wait(&sm.v_empty, (itt & 1) ^ 1, sm, a.err);
+            unsigned char *vrow = reinterpret_cast<unsigned char *>(sm.vs) + m * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                if (c < ui.np * 2) {
+                    uint4 pk;
+                    __nv_bfloat162 h0 = __floats2bfloat162_rn(d1[c * 8 + 0], d1[c * 8 + 1]);
+                    __nv_bfloat162 h1 = __floats2bfloat162_rn(d1[c * 8 + 2], d1[c * 8 + 3]);
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(d1[c * 8 + 4], d1[c * 8 + 5]);
+                    __nv_bfloat162 h3 = __floats2bfloat162_rn(d1[c * 8 + 6], d1[c * 8 + 7]);
+                    pk.x = *reinterpret_cast<uint32_t *>(&h0);
+                    pk.y = *reinterpret_cast<uint32_t *>(&h1);
+                    pk.z = *reinterpret_cast<uint32_t *>(&h2);
+                    pk.w = *reinterpret_cast<uint32_t *>(&h3);
+                    *reinterpret_cast<uint4 *>(vrow + ((c ^ (m & 7)) << 4)) = pk;
+                }
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive(&sm.v_ready);
+            // n-tiles
+            for (int j = ui.j0; j < ui.j1; ++j, ++ite) {
+                const int b = ite & 1;
+                const uint32_t par = (ite >> 1) & 1;
+                mbar_wait(&sm.accfull[b], par, sm, a.err);
+                mbar_wait(&sm.yfull[b], par, sm, a.err);
+                tc_fence_after();
+                float acc[64];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) TMEM_LD16(trow + 64 + 64 * b + c * 16, (&acc[c * 16]));
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(&sm.accempty[b]);
+                const bool full_tile = ui.ntok == kM;
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const int h = c >> 3, cc = c & 7;
+                    float4 *yp = reinterpret_cast<float4 *>(reinterpret_cast<unsigned char *>(&sm.ys[b][h * kM * 32]) +
+                                                            m * 128 + ((cc ^ (m & 7)) << 4));
+                    float4 y = *yp;
+                    y.x = fmaf(sc, acc[c * 4 + 0], y.x);
+                    y.y = fmaf(sc, acc[c * 4 + 1], y.y);
+                    y.z = fmaf(sc, acc[c * 4 + 2], y.z);
+                    y.w = fmaf(sc, acc[c * 4 + 3], y.w);
+                    if (full_tile) {
+                        *yp = y;
+                    } else if (m < ui.ntok) {
+                        const int col = j * kNB + c * 4;
+                        if (col < a.d_out)
+                            *reinterpret_cast<float4 *>(a.Y + (size_t)(ui.row0 + m) * a.d_out + col) = y;
+                    }
+                }
+                if (full_tile) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                epi_sync();
+                if (leader) {
+                    if (full_tile) {
+                        tma_store(&tmY, j * kNB, ui.row0, &sm.ys[b][0]);
+                        tma_store(&tmY, j * kNB + 32, ui.row0, &sm.ys[b][kM * 32]);
+                        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                    }
+                    mbar_arrive(&sm.yempty[b]);
+                }
+            }
+            ++itt;
+        }
+        if (leader) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 2) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+int make_map(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, uint64_t cols, uint64_t rows,
+             uint32_t box_cols, uint32_t box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return LORA_ERR_CUDA;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * (uint64_t)esize};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? LORA_OK : LORA_ERR_CUDA;
+}
+
+}  // namespace
+
+bool tiles_supported() { return encode_fn() != nullptr; }
+
+int launch_tiles(const TileArgs &a, cudaStream_t st, bool pdl) {
+    static int num_sms[64] = {};
+    int dev = 0;
+    if (int rc = cuda_check(cudaGetDevice(&dev))) return rc;
+    if (dev < 0 || dev >= 64) return LORA_ERR_INVALID_ARG;
+    const size_t smem = sizeof(TileSmem) + 1024;
+    if (num_sms[dev] == 0) {
+        if (int rc = cuda_check(cudaFuncSetAttribute(tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+            return rc;
+        int n = 0;
+        if (int rc = cuda_check(cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev))) return rc;
+        num_sms[dev] = n > 0 ? n : 1;
+    }
+    CUtensorMap mx, ma, mb, my;
+    if (make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.X, (uint64_t)a.d_in, (uint64_t)a.T, kKB, kM) ||
+        make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.pa->base, (uint64_t)a.d_in, (uint64_t)a.rowsA, kKB, 16) ||
+        make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.pb->base, (uint64_t)a.d_out, (uint64_t)a.rowsB, kNB, 16) ||
+        make_map(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.Y, (uint64_t)a.d_out, (uint64_t)a.T, 32, kM))
+        return LORA_ERR_CUDA;
+    // upper bound of units: every tile of every long segment times the d_out split
+    const int max_tiles = (a.T + kM - 1) / kM + (a.long_thresh > 0 ? a.T / a.long_thresh : 0);
+    int grid = num_sms[dev];
+    if (grid > max_tiles * ((a.d_out + kNB - 1) / kNB)) grid = max_tiles * ((a.d_out + kNB - 1) / kNB);
+    if (grid < 1) grid = 1;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (int rc = cuda_check(cudaLaunchKernelEx(&cfg, tiles_kernel, mx, ma, mb, my, a))) return rc;
+    count_launch();
+    return LORA_OK;
+}
+
+}  // namespace lora

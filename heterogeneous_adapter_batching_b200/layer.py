@@ -1,0 +1,76 @@
+"""Device state of one adapted projection: two page pools, the slot tables and
+the workspace, held in torch tensors (device memory only; every computation
+goes through the C-ABI calls in _binding)."""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _binding as B
+
+
+class AdapterLayer:
+    """Pools, page table [S, 2, 4], ranks [S], scales [S], error word and workspace.
+
+    pool_a holds A^T rows (width d_in), pool_b holds B rows (width d_out); when
+    d_in == d_out and `shared_pool` is set, one pool serves both.
+    """
+
+    def __init__(self, d_in: int, d_out: int, num_slots: int, pages_a: int, pages_b: int,
+                 max_tokens: int, device="cuda", shared_pool: bool = False):
+        self.d_in, self.d_out, self.S = d_in, d_out, num_slots
+        self.device = torch.device(device)
+        rows_a = pages_a * B.PAGE_ROWS
+        self.buf_a = torch.empty((rows_a, d_in), dtype=torch.bfloat16, device=self.device)
+        self.pool_a = B.lora_pool_create(self.buf_a, d_in)
+        if shared_pool and d_in == d_out:
+            self.buf_b, self.pool_b = self.buf_a, self.pool_a
+        else:
+            rows_b = pages_b * B.PAGE_ROWS
+            self.buf_b = torch.empty((rows_b, d_out), dtype=torch.bfloat16, device=self.device)
+            self.pool_b = B.lora_pool_create(self.buf_b, d_out)
+        self.page_table = torch.full((num_slots, 2, B.MAX_PAGES_PER_MATRIX), -1, dtype=torch.int32,
+                                     device=self.device)
+        self.ranks = torch.zeros(num_slots, dtype=torch.int32, device=self.device)
+        self.scales = torch.zeros(num_slots, dtype=torch.float32, device=self.device)
+        self.err = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self.max_tokens = max_tokens
+        nbytes = B.lora_workspace_size(max_tokens, num_slots)
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+
+    def load(self, slot: int, rank: int, alpha: float, a_t_bits: torch.Tensor, b_bits: torch.Tensor,
+             page_ids: Optional[torch.Tensor] = None, stream=None) -> None:
+        """a_t_bits [rank, d_in], b_bits [rank, d_out]: bf16 tensors (host or device)."""
+        B.lora_pool_load(self.pool_a, self.pool_b, slot, self.S, rank, alpha, a_t_bits.contiguous(),
+                         b_bits.contiguous(), page_ids, self.page_table, self.scales, self.ranks, stream)
+
+    def evict(self, slot: int, stream=None) -> None:
+        B.lora_pool_evict(self.pool_a, self.pool_b, slot, self.S, self.page_table, self.scales, self.ranks,
+                          stream)
+
+    def apply(self, X: torch.Tensor, Y: torch.Tensor, ids: torch.Tensor, stream=None) -> None:
+        T = X.shape[0]
+        assert T <= self.max_tokens
+        B.lora_apply(X, Y, T, self.d_in, self.d_out, ids, self.S, self.ranks, self.scales, self.page_table,
+                     self.pool_a, self.pool_b, self.ws, self.err, stream)
+
+    def apply_planned(self, X: torch.Tensor, Y: torch.Tensor, ws: Optional[torch.Tensor] = None,
+                      stream=None) -> None:
+        """Compute half only, with the plan already in `ws` (default: this layer's workspace)."""
+        B.lora_apply_planned(X, Y, X.shape[0], self.d_in, self.d_out, self.S, self.ranks, self.scales,
+                             self.page_table, self.pool_a, self.pool_b, self.ws if ws is None else ws,
+                             self.err, stream)
+
+    def shrink(self, X: torch.Tensor, ids: torch.Tensor, V: torch.Tensor, stream=None) -> None:
+        B.lora_shrink(X, X.shape[0], self.d_in, ids, self.S, self.ranks, self.page_table, self.pool_a, V,
+                      self.ws, self.err, stream)
+
+    def expand_add(self, V: torch.Tensor, Y: torch.Tensor, ids: torch.Tensor, stream=None) -> None:
+        B.lora_expand_add(V, Y, V.shape[0], self.d_out, ids, self.S, self.ranks, self.scales,
+                          self.page_table, self.pool_b, self.ws, self.err, stream)
+
+    def plan(self, ids: torch.Tensor, perm: Optional[torch.Tensor] = None, seg_start: Optional[torch.Tensor] = None,
+             ws: Optional[torch.Tensor] = None, stream=None) -> None:
+        B.lora_plan(ids, ids.shape[0], self.ranks, self.S, perm, seg_start, self.ws if ws is None else ws,
+                    self.err, stream)

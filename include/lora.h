@@ -1,0 +1,212 @@
+/*
+ * liblora — heterogeneous-batch LoRA adapter branch on one B200 (sm_100a).
+ *
+ * Computes, for every token t of a batch whose adapter id is i = ids[t]:
+ *
+ *     Y[t, :] += (alpha_i / r_i) * (X[t, :] A_i) B_i
+ *
+ * with A_i [d_in x r_i] and B_i [r_i x d_out] taken from a paged GPU pool.
+ * Page "Multi-LoRA Serving in Production" (llms.blog), section "The
+ * Mathematical Anatomy of Heterogeneous Batches", gives the formula and the
+ * per-sequence adapters; section "Segmented Gather Matrix-Vector
+ * Multiplication (SGMV)" gives the shrink (v = x A) and the scaled expand
+ * (y += (alpha/r) v B) steps and the grouping of tokens by adapter; sections
+ * "Multi-Size Batched Gather Kernels (MBGMV and MBGMM)" and "Unified Paging
+ * Architecture" give mixed ranks without padding to the maximum rank and
+ * weights gathered from non-contiguous pages through physical page indices.
+ *
+ * Conventions for every call below
+ *  - Return value: LORA_OK (0) or a negative LORA_ERR_* code.  A call that
+ *    returns an error has enqueued no work.
+ *  - Every compute call is asynchronous on the given stream and does no
+ *    host synchronisation.  Pointers named *_dev, and X, Y, V, ids, ranks,
+ *    scales, page_table and ws, are device pointers; everything else is host.
+ *  - bf16 data is passed as uint16_t bit patterns.  Matrices are row-major.
+ *  - Inputs are never modified, except Y (updated in place) and the outputs
+ *    named in each call.
+ *  - The device error word err_dev (may be NULL) receives an OR of
+ *    LORA_DEV_ERR_* bits.  A token whose id is outside [-1, S) or names an
+ *    empty slot (rank 0) is skipped: its Y row is left untouched.  id = -1
+ *    means "base model only" and is not an error.  Kernels never trap.
+ *  - The library keeps no device memory of its own: scratch space comes
+ *    from the caller's workspace (ws, ws_bytes).
+ */
+#ifndef LORA_H_
+#define LORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *lora_stream_t;      /* a cudaStream_t; NULL = legacy default stream */
+typedef struct lora_pool_s *lora_pool_t;        /* opaque host handle of one page pool */
+
+/* Host return codes. */
+#define LORA_OK                  0
+#define LORA_ERR_INVALID_ARG    -1   /* NULL pointer, negative size, misaligned buffer, unknown option */
+#define LORA_ERR_BAD_RANK       -2   /* rank outside [1, LORA_MAX_RANK] */
+#define LORA_ERR_WIDTH_MISMATCH -3   /* pool row width differs from d_in / d_out */
+#define LORA_ERR_POOL_OOM       -4   /* not enough free pages */
+#define LORA_ERR_BAD_SLOT       -5   /* slot outside [0, num_slots), or page id not free / out of range */
+#define LORA_ERR_CUDA           -6   /* a CUDA runtime call failed; see lora_last_cuda_error() */
+#define LORA_ERR_WORKSPACE      -7   /* ws is NULL or ws_bytes < lora_workspace_size(...) */
+
+/* Device error word bits. */
+#define LORA_DEV_ERR_BAD_ID      1   /* some id < -1 or id >= num_slots */
+#define LORA_DEV_ERR_EMPTY_SLOT  2   /* some id names a slot with rank 0 */
+#define LORA_DEV_ERR_TIMEOUT     4   /* a kernel's bounded wait ran out (results of that call are undefined) */
+#define LORA_DEV_ERR_BAD_PAGE    8   /* a used slot's rank exceeds 64 or its page table names a page outside the
+                                        pool; its tokens are skipped */
+
+/* Fixed geometry. */
+#define LORA_PAGE_ROWS            16   /* rank-rows per page */
+#define LORA_MAX_RANK             64
+#define LORA_MAX_PAGES_PER_MATRIX 4    /* LORA_MAX_RANK / LORA_PAGE_ROWS */
+#define LORA_MAX_SLOTS            4096
+
+/* ------------------------------------------------------------------------ */
+/* Page pool (page "Multi-LoRA Serving in Production", section "Unified     */
+/* Paging Architecture": fixed-size physical pages, adapter weights sliced  */
+/* along the rank dimension, logical page tables naming physical pages).   */
+/* ------------------------------------------------------------------------ */
+
+/* Wrap caller-owned device memory dev_buf[bytes] as a pool of pages of
+ * page_rows (must be LORA_PAGE_ROWS) rows of `width` bf16 values each.
+ * num_pages = bytes / (page_rows * width * 2).  dev_buf must be 256-byte
+ * aligned and width a positive multiple of 8.  The caller keeps ownership of
+ * dev_buf and must keep it alive until lora_pool_destroy; the library owns
+ * the host-side free list.  Physical row p*page_rows + j of the pool is the
+ * bf16 row at dev_buf + (p*page_rows + j) * width * 2 bytes. */
+int lora_pool_create(void *dev_buf, size_t bytes, int width, int page_rows, lora_pool_t *out);
+
+/* Free the host handle (not the device memory).  NULL is accepted. */
+int lora_pool_destroy(lora_pool_t pool);
+
+/* Pages currently free / in total; -1 for a NULL handle. */
+int lora_pool_free_pages(lora_pool_t pool);
+int lora_pool_num_pages(lora_pool_t pool);
+
+/* Load adapter (A, B) of rank `rank` into slot `slot` of the page table
+ * page_table_dev [num_slots][2][LORA_MAX_PAGES_PER_MATRIX] (int32; matrix 0 =
+ * A, 1 = B; unused entries are written as -1).
+ *  a_t  : A transposed, [rank][d_in] bf16 (row k = column k of A), d_in = pa's width
+ *  b    : B, [rank][d_out] bf16, d_out = pb's width
+ *  a_t and b may be host (pinned or pageable) or device pointers.
+ * ceil(rank/16) pages are taken from each pool's free list, or, when
+ * page_ids (host, [2][LORA_MAX_PAGES_PER_MATRIX]) is not NULL, exactly those
+ * pages (which must be free).  The rows are copied with cudaMemcpyAsync on
+ * `stream` (page "Multi-LoRA Serving in Production", section "Asynchronous
+ * Prefetching and Request Queuing"); the unused rows of a partly filled last
+ * page are zeroed.  The slot's page-table row, scale_dev[slot] = alpha/rank
+ * (fp32) and rank_dev[slot] = rank are written on the same stream.
+ * The slot must be empty (load into an occupied slot returns
+ * LORA_ERR_BAD_SLOT; evict it first).  Validation (page "Multi-LoRA
+ * Serving Architecture ... (2026)", section "Trade-offs, Gotchas": validate
+ * shape and rank before admission): rank in [1, 64] else LORA_ERR_BAD_RANK.
+ * The pools record which pages belong to (page_table_dev, slot). */
+int lora_pool_load(lora_pool_t pa, lora_pool_t pb, int slot, int num_slots, int rank, float alpha,
+                   const uint16_t *a_t, const uint16_t *b, const int32_t *page_ids,
+                   int32_t *page_table_dev, float *scale_dev, int32_t *rank_dev,
+                   lora_stream_t stream);
+
+/* Return the pages of (page_table_dev, slot) to the free lists and mark the
+ * slot empty on the device (rank 0, scale 0, page entries -1) on `stream`.
+ * Pages are reused in stream order: a later load on the same stream is safe;
+ * a caller using several streams must order them itself. */
+int lora_pool_evict(lora_pool_t pa, lora_pool_t pb, int slot, int num_slots,
+                    int32_t *page_table_dev, float *scale_dev, int32_t *rank_dev,
+                    lora_stream_t stream);
+
+/* Copy rank-row k of matrix m (0 = A^T, 1 = B) of a loaded slot back into
+ * out_dev (device, width bf16) by resolving the page table on the device:
+ * physical row = page_table[slot][m][k / 16] * 16 + k % 16 (used to verify
+ * the paging round trip). */
+int lora_pool_read_row(lora_pool_t pool, const int32_t *page_table_dev, int num_slots, int slot,
+                       int m, int k, uint16_t *out_dev, lora_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Compute                                                                  */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of workspace the calls below need for T tokens and num_slots slots. */
+size_t lora_workspace_size(int T, int num_slots);
+
+/* Group tokens by adapter slot (page "Multi-LoRA Serving in Production",
+ * section SGMV: requests are grouped by their target adapter), stably, and
+ * store the plan of the batch in ws:
+ *   perm   [T]    tokens with a valid adapter, by slot ascending, then by
+ *                 token index; entries past the number of valid tokens are
+ *                 left untouched
+ *   seg_start [S+1]  tokens of slot i are perm[seg_start[i] .. seg_start[i+1])
+ * plus the work lists of the two compute paths.  When perm_out / seg_start_out
+ * (device) are not NULL the two arrays are also written there.
+ * Tokens with id -1 are dropped; invalid ids are dropped and flagged in err_dev.
+ * ranks: [num_slots] int32 (0 = empty slot).  The plan stays valid in ws for
+ * lora_apply_planned until ws is reused; it depends on ids, ranks, T,
+ * num_slots and the LORA_OPT_* values at the time of the call. */
+int lora_plan(const int32_t *ids, int T, const int32_t *ranks, int num_slots,
+              int32_t *perm_out, int32_t *seg_start_out,
+              void *ws, size_t ws_bytes, int32_t *err_dev, lora_stream_t stream);
+
+/* Shrink: V[t, k] = sum_j X[t, j] A_i[j, k] for k < r_i, fp32 accumulate.
+ *   X [T][d_in] bf16, V [T][LORA_MAX_RANK] fp32 (columns >= r_i and rows of
+ *   tokens without a valid adapter are left untouched).  pa's width must be d_in. */
+int lora_shrink(const uint16_t *X, int T, int d_in, const int32_t *ids, int num_slots,
+                const int32_t *ranks, const int32_t *page_table, lora_pool_t pa,
+                float *V, void *ws, size_t ws_bytes, int32_t *err_dev, lora_stream_t stream);
+
+/* Expand-add: Y[t, c] += s_i * sum_{k < r_i} V[t, k] B_i[k, c], fp32.
+ *   V [T][LORA_MAX_RANK] fp32, Y [T][d_out] fp32 in place, scales [num_slots]
+ *   fp32 (alpha_i / r_i).  pb's width must be d_out. */
+int lora_expand_add(const float *V, float *Y, int T, int d_out, const int32_t *ids, int num_slots,
+                    const int32_t *ranks, const float *scales, const int32_t *page_table,
+                    lora_pool_t pb, void *ws, size_t ws_bytes, int32_t *err_dev,
+                    lora_stream_t stream);
+
+/* Fused shrink + expand-add: Y[t] += s_i (X[t] A_i) B_i for every token.
+ *   X [T][d_in] bf16, Y [T][d_out] fp32 (holds Y_base = X W0 on entry, computed
+ *   by the caller; page "Multi-LoRA Serving Architecture ... (2026)", section
+ *   "Heterogeneous batching: the core compute trick": the base GEMM runs once
+ *   on the whole batch and the two branches are added).
+ * Segments shorter than the long-segment threshold take the gather
+ * (MBGMV-style) kernels; longer ones take the tensor-core (MBGMM-style)
+ * tiles.  The result does not depend on the token order. */
+int lora_apply(const uint16_t *X, float *Y, int T, int d_in, int d_out, const int32_t *ids,
+               int num_slots, const int32_t *ranks, const float *scales,
+               const int32_t *page_table, lora_pool_t pa, lora_pool_t pb,
+               void *ws, size_t ws_bytes, int32_t *err_dev, lora_stream_t stream);
+
+/* The compute half of lora_apply: Y[t] += s_i (X[t] A_i) B_i using the plan
+ * that lora_plan left in ws for this batch (same T, num_slots, ranks and
+ * options).  A model applies one plan to all of its adapted layers: a token's
+ * adapter slot is the same in every layer, only the pools, page tables and
+ * scales differ.  Launches only the compute kernels. */
+int lora_apply_planned(const uint16_t *X, float *Y, int T, int d_in, int d_out, int num_slots,
+                       const int32_t *ranks, const float *scales, const int32_t *page_table,
+                       lora_pool_t pa, lora_pool_t pb, void *ws, size_t ws_bytes,
+                       int32_t *err_dev, lora_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Options and diagnostics (process-wide)                                   */
+/* ------------------------------------------------------------------------ */
+
+#define LORA_OPT_LONG_SEGMENT   1   /* segments with >= this many tokens use the tensor-core path (default 16; 0 = never) */
+#define LORA_OPT_DECODE_JOB_TOKENS 2 /* max tokens per gather job (1..4, default 4) */
+
+int lora_set_option(int key, int value);
+int lora_get_option(int key);
+
+/* Message of the last CUDA error seen by this library (static string). */
+const char *lora_last_cuda_error(void);
+
+/* Number of kernels launched by the last lora_apply / lora_shrink /
+ * lora_expand_add / lora_plan call on the calling host thread. */
+int lora_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LORA_H_ */

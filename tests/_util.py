@@ -1,0 +1,65 @@
+"""Shared helpers of the GPU tests: upload a seeded workload through the C ABI
+and compare device results with the fp64 oracle."""
+from __future__ import annotations
+
+import numpy as np
+
+import workloads as W
+
+# Spec tolerance per element (fp32 accumulate): |err| <= 2e-3 + 1e-2 |ref|.
+ATOL, RTOL = 2e-3, 1e-2
+# A stricter bound on the adapter delta alone, relative to its largest magnitude.
+# It separates a wrong rank row / adapter / scale (O(1) relative) from rounding.
+DELTA_REL_GATHER = 1e-4     # fp32 v and fp32 accumulation throughout
+DELTA_REL_TENSOR = 8e-3     # v rounded to bf16 before the second product
+
+
+def make_layer(wl: W.Workload, max_tokens=None, shared_pool=False, extra_pages=0):
+    import torch
+    from heterogeneous_adapter_batching_b200 import AdapterLayer
+    layer = AdapterLayer(wl.d_in, wl.d_out, wl.S, wl.pages_a + extra_pages, wl.pages_b + extra_pages,
+                         max(1, max_tokens if max_tokens is not None else wl.T), shared_pool=shared_pool)
+    for i in range(wl.S):
+        a = wl.adapters[i]
+        if a is None:
+            continue
+        at = torch.from_numpy(W.bf16_bits(np.ascontiguousarray(a.A.T)).view(np.int16)).cuda()
+        b = torch.from_numpy(W.bf16_bits(a.B).view(np.int16)).cuda()
+        pid = None if shared_pool else torch.from_numpy(np.ascontiguousarray(wl.page_ids[i]))
+        layer.load(i, a.rank, a.alpha, at, b, page_ids=pid)
+    return layer
+
+
+def dev_inputs(wl: W.Workload):
+    import torch
+    X = torch.from_numpy(W.bf16_bits(wl.X).view(np.int16)).cuda().view(torch.bfloat16)
+    Y = torch.from_numpy(wl.Y_base.copy()).cuda()
+    ids = torch.from_numpy(wl.ids.copy()).cuda()
+    return X, Y, ids
+
+
+def oracle_full(wl: W.Workload, nthreads=0):
+    from oracle import build_oracle as OC
+    A = [None if a is None else a.A for a in wl.adapters]
+    B = [None if a is None else a.B for a in wl.adapters]
+    return OC.lora_apply_c(wl.X, wl.Y_base, wl.ids, A, B, wl.scales_f32(), nthreads=nthreads)
+
+
+def oracle_tokens(wl: W.Workload, tokens, nthreads=0):
+    from oracle import build_oracle as OC
+    X, Yb, ids, A, B, sc = W.subset_for_tokens(wl, tokens)
+    return OC.lora_apply_c(X, Yb, ids, A, B, sc, nthreads=nthreads)
+
+
+def assert_parity(Y_dev: np.ndarray, Y_ref: np.ndarray, Y_base: np.ndarray, delta_rel=DELTA_REL_GATHER):
+    Y_dev = np.asarray(Y_dev, np.float64)
+    err = np.abs(Y_dev - Y_ref)
+    bound = ATOL + RTOL * np.abs(Y_ref)
+    bad = err > bound
+    assert not bad.any(), f"{bad.sum()} elements outside 2e-3+1e-2|ref|; worst {err.max():.3e}"
+    d_ref = Y_ref - np.asarray(Y_base, np.float64)
+    d_dev = Y_dev - np.asarray(Y_base, np.float64)
+    scale = np.abs(d_ref).max()
+    if scale > 0:
+        worst = np.abs(d_dev - d_ref).max()
+        assert worst <= delta_rel * scale, f"delta error {worst:.3e} > {delta_rel:g} * {scale:.3e}"

@@ -1,0 +1,235 @@
+"""GPU parity: liblora (through the C ABI) against the fp64 oracle, element by element.
+
+Tolerance per element (fp32 accumulate): |err| <= 2e-3 + 1e-2 |ref|, plus a
+stricter bound on the adapter delta (see tests/_util.py).  All indexing
+(plan, pages, which rows change) is checked bit-exactly.
+"""
+import numpy as np
+import pytest
+
+import workloads as W
+from tests import _util as U
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def H():
+    import torch
+    import heterogeneous_adapter_batching_b200 as H
+    H.load_library()
+    torch.cuda.init()
+    return H
+
+
+@pytest.fixture(autouse=True)
+def _restore_options(H):
+    old = {k: H.lora_get_option(k) for k in (H.OPT_LONG_SEGMENT, H.OPT_DECODE_JOB_TOKENS)}
+    yield
+    for k, v in old.items():
+        H.lora_set_option(k, v)
+
+
+def _run_apply(H, wl, **kw):
+    import torch
+    layer = U.make_layer(wl, **kw)
+    X, Y, ids = U.dev_inputs(wl)
+    layer.err.zero_()
+    layer.apply(X, Y, ids)
+    torch.cuda.synchronize()
+    return Y.cpu().numpy(), int(layer.err.item()), layer
+
+
+def test_tiny_config(H):
+    wl = W.tiny()
+    Y, err, _ = _run_apply(H, wl)
+    ref, rerr = U.oracle_full(wl)
+    assert err == rerr == 0
+    U.assert_parity(Y, ref, wl.Y_base)
+
+
+@pytest.mark.parametrize("job_tokens", [1, 3, 4])
+@pytest.mark.parametrize("seed,T,d_in,d_out,S", [
+    (1, 1, 64, 64, 3), (2, 7, 24, 40, 5), (3, 33, 264, 136, 9), (4, 100, 512, 1032, 17),
+    (5, 257, 8, 8, 4), (6, 64, 1000, 2000, 40),
+])
+def test_random_small(H, seed, T, d_in, d_out, S, job_tokens):
+    H.lora_set_option(H.OPT_DECODE_JOB_TOKENS, job_tokens)
+    wl = W.random_small(seed=seed, T=T, d_in=d_in, d_out=d_out, S=S, ranks=(1, 4, 8, 15, 16, 17, 33, 64),
+                        p_none=0.15)
+    Y, err, _ = _run_apply(H, wl)
+    ref, rerr = U.oracle_full(wl)
+    assert err == rerr == 0
+    U.assert_parity(Y, ref, wl.Y_base)
+
+
+def test_decode_q_proj_7b_full(H):
+    wl = W.decode_q_proj_7b()
+    Y, err, _ = _run_apply(H, wl)
+    ref, rerr = U.oracle_full(wl)
+    assert err == rerr == 0
+    U.assert_parity(Y, ref, wl.Y_base)
+
+
+@pytest.mark.parametrize("which", ["up", "down"])
+def test_mixed_mlp_full(H, which):
+    wl = W.mixed_mlp(which=which)
+    Y, err, _ = _run_apply(H, wl)
+    ref, rerr = U.oracle_full(wl)
+    assert err == rerr == 0
+    U.assert_parity(Y, ref, wl.Y_base)
+
+
+def test_prefill_full(H):
+    wl = W.prefill()
+    Y, err, _ = _run_apply(H, wl)
+    ref, rerr = U.oracle_full(wl)
+    assert err == rerr == 0
+    U.assert_parity(Y, ref, wl.Y_base, delta_rel=U.DELTA_REL_TENSOR)
+
+
+@pytest.mark.parametrize("regime", ["one", "distinct"])
+@pytest.mark.parametrize("T", [1, 16, 64, 256, 1024])
+def test_sweep_8b(H, regime, T):
+    wl = W.sweep_8b(T=T, regime=regime)
+    Y, err, _ = _run_apply(H, wl)
+    assert err == 0
+    if T <= 64:
+        tokens = np.arange(T)
+    else:
+        tokens = np.sort(np.random.default_rng(T).choice(T, size=48, replace=False))
+    ref, rerr = U.oracle_tokens(wl, tokens)
+    assert rerr == 0
+    U.assert_parity(Y[tokens], ref, wl.Y_base[tokens], delta_rel=U.DELTA_REL_TENSOR)
+
+
+# ---------------------------------------------------------------------------
+# Invariants the pages fix
+# ---------------------------------------------------------------------------
+
+def test_zero_b_leaves_y_bit_exact(H):
+    import torch
+    wl = W.random_small(seed=11, T=50, d_in=256, d_out=320, S=6, ranks=(4, 16, 64))
+    layer = U.make_layer(wl)
+    # overwrite every B row with zeros through a reload into the same pages
+    for i in range(wl.S):
+        a = wl.adapters[i]
+        layer.evict(i)
+        at = torch.from_numpy(W.bf16_bits(np.ascontiguousarray(a.A.T)).view(np.int16)).cuda()
+        b0 = torch.zeros((a.rank, wl.d_out), dtype=torch.int16, device="cuda")
+        layer.load(i, a.rank, a.alpha, at, b0, page_ids=torch.from_numpy(wl.page_ids[i].copy()))
+    X, Y, ids = U.dev_inputs(wl)
+    layer.apply(X, Y, ids)
+    torch.cuda.synchronize()
+    assert np.array_equal(Y.cpu().numpy(), wl.Y_base)
+
+
+def test_permutation_equivariance_bit_exact(H):
+    import torch
+    wl = W.decode_q_proj_7b(T=64)
+    Y1, _, layer = _run_apply(H, wl)
+    P = np.random.default_rng(3).permutation(wl.T)
+    X, Y, ids = U.dev_inputs(wl)
+    Pt = torch.from_numpy(P).cuda()
+    X2, Y2, ids2 = X[Pt].contiguous(), Y[Pt].contiguous(), ids[Pt].contiguous()
+    layer.apply(X2, Y2, ids2)
+    torch.cuda.synchronize()
+    assert np.array_equal(Y2.cpu().numpy(), Y1[P])
+
+
+def test_none_and_invalid_ids(H):
+    import torch
+    wl = W.random_small(seed=12, T=40, d_in=128, d_out=96, S=5, ranks=(8, 16), p_none=0.0)
+    Yc, _, layer = _run_apply(H, wl)
+    X, Y, ids = U.dev_inputs(wl)
+    ids_h = wl.ids.copy()
+    ids_h[[1, 9]] = -1
+    ids_h[[3, 20]] = wl.S          # out of range
+    ids_h[[5]] = -7                # out of range
+    ids.copy_(torch.from_numpy(ids_h))
+    layer.err.zero_()
+    layer.apply(X, Y, ids)
+    torch.cuda.synchronize()
+    Yn = Y.cpu().numpy()
+    assert int(layer.err.item()) == H.DEV_ERR_BAD_ID
+    for t in (1, 9, 3, 20, 5):
+        assert np.array_equal(Yn[t], wl.Y_base[t])
+    others = [t for t in range(wl.T) if t not in (1, 9, 3, 20, 5)]
+    assert np.array_equal(Yn[others], Yc[others])
+
+
+def test_evicted_slot_sets_empty_bit_and_skips(H):
+    import torch
+    wl = W.random_small(seed=13, T=30, d_in=128, d_out=128, S=4, ranks=(16,), p_none=0.0)
+    Yc, _, layer = _run_apply(H, wl)
+    layer.evict(2)
+    X, Y, ids = U.dev_inputs(wl)
+    layer.err.zero_()
+    layer.apply(X, Y, ids)
+    torch.cuda.synchronize()
+    Yn = Y.cpu().numpy()
+    assert int(layer.err.item()) == H.DEV_ERR_EMPTY_SLOT
+    on2 = wl.ids == 2
+    assert on2.any()
+    assert np.array_equal(Yn[on2], wl.Y_base[on2])
+    assert np.array_equal(Yn[~on2], Yc[~on2])
+
+
+def test_all_tokens_one_adapter_matches_dense(H):
+    """One adapter for the whole batch equals one dense product (fp64 numpy matmul)."""
+    wl = W.sweep_8b(T=64, regime="one", pool=4, d_in=1024, d_out=2048)
+    Y, err, _ = _run_apply(H, wl)
+    i = int(wl.ids[0])
+    a = wl.adapters[i]
+    ref = wl.Y_base.astype(np.float64) + 2.0 * (wl.X.astype(np.float64) @ a.A.astype(np.float64)) @ a.B.astype(np.float64)
+    assert err == 0
+    U.assert_parity(Y, ref, wl.Y_base, delta_rel=U.DELTA_REL_TENSOR)
+
+
+def test_empty_batch_and_all_none(H):
+    import torch
+    wl = W.random_small(seed=14, T=16, d_in=64, d_out=64, S=3, ranks=(8,), p_none=1.0)
+    Y, err, _ = _run_apply(H, wl)
+    assert err == 0 and np.array_equal(Y, wl.Y_base)
+    layer = U.make_layer(wl)
+    X0 = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    Y0 = torch.empty((0, 64), dtype=torch.float32, device="cuda")
+    ids0 = torch.empty((0,), dtype=torch.int32, device="cuda")
+    layer.apply(X0, Y0, ids0)
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------------------
+# The two-step entry points
+# ---------------------------------------------------------------------------
+
+def test_shrink_matches_oracle(H):
+    import torch
+    from oracle import lora_oracle as O
+    wl = W.random_small(seed=15, T=70, d_in=520, d_out=64, S=7, ranks=(1, 8, 16, 40, 64), p_none=0.1)
+    layer = U.make_layer(wl)
+    X, _, ids = U.dev_inputs(wl)
+    V = torch.full((wl.T, 64), float("nan"), dtype=torch.float32, device="cuda")
+    layer.shrink(X, ids, V)
+    torch.cuda.synchronize()
+    Vd = V.cpu().numpy()
+    Vr, _ = O.lora_shrink(wl.X, wl.ids, [a.A for a in wl.adapters])
+    defined = ~np.isnan(Vr)
+    assert np.array_equal(np.isnan(Vd), ~defined)          # untouched entries stay NaN
+    err = np.abs(Vd[defined] - Vr[defined])
+    assert (err <= U.ATOL + U.RTOL * np.abs(Vr[defined])).all()
+    assert err.max() <= 1e-4 * np.abs(Vr[defined]).max()
+
+
+def test_expand_add_matches_oracle(H):
+    import torch
+    from oracle import lora_oracle as O
+    wl = W.random_small(seed=16, T=70, d_in=64, d_out=1000, S=7, ranks=(1, 8, 16, 40, 64), p_none=0.1)
+    layer = U.make_layer(wl)
+    _, Y, ids = U.dev_inputs(wl)
+    Vh = np.random.default_rng(16).standard_normal((wl.T, 64)).astype(np.float32)
+    V = torch.from_numpy(Vh).cuda()
+    layer.expand_add(V, Y, ids)
+    torch.cuda.synchronize()
+    ref, _ = O.lora_expand_add(Vh, wl.Y_base, wl.ids, [a.B for a in wl.adapters], wl.scales_f32())
+    U.assert_parity(Y.cpu().numpy(), ref, wl.Y_base)

@@ -56,6 +56,38 @@ class Adapter:
     B: np.ndarray  # [r, d_out] float32 holding bf16 values
 
 
+class Adapters:
+    """Per-slot adapters, each drawn from its own seed on first access, so a
+    large resident pool never has to be held in host memory at once."""
+
+    def __init__(self, seed: int, d_in: int, d_out: int, ranks: np.ndarray, cache: bool = True):
+        self.seed, self.d_in, self.d_out = seed, d_in, d_out
+        self.rank_of = np.asarray(ranks, dtype=np.int32)
+        self._cache = {} if cache else None
+
+    def __len__(self) -> int:
+        return len(self.rank_of)
+
+    def __getitem__(self, i: int) -> Optional[Adapter]:
+        i = int(i)
+        r = int(self.rank_of[i])
+        if r <= 0:
+            return None
+        if self._cache is not None and i in self._cache:
+            return self._cache[i]
+        rng = np.random.default_rng([self.seed, 100, i])
+        A = bf16_round(rng.standard_normal((self.d_in, r), dtype=np.float32) / np.float32(np.sqrt(self.d_in)))
+        B = bf16_round(rng.standard_normal((r, self.d_out), dtype=np.float32) / np.float32(np.sqrt(r)))
+        ad = Adapter(rank=r, alpha=2.0 * r, A=A, B=B)
+        if self._cache is not None:
+            self._cache[i] = ad
+        return ad
+
+    def __iter__(self):
+        for i in range(len(self)):
+            yield self[i]
+
+
 @dataclasses.dataclass
 class Workload:
     name: str
@@ -64,11 +96,10 @@ class Workload:
     X: np.ndarray          # [T, d_in] float32 (bf16 values)
     Y_base: np.ndarray     # [T, d_out] float32
     ids: np.ndarray        # [T] int32, -1 = base model only
-    adapters: List[Optional[Adapter]]  # one entry per slot; None = empty slot
-    # seeded physical page ids per slot: [S, 2, 4] (unused entries -1)
-    page_ids: np.ndarray
-    pages_a: int           # number of pages needed in the d_in-wide pool
-    pages_b: int           # number of pages needed in the d_out-wide pool
+    adapters: Adapters     # one entry per slot; None = empty slot
+    page_ids: np.ndarray   # seeded physical page ids per slot: [S, 2, 4] (unused -1)
+    pages_a: int           # pages in the d_in-wide pool
+    pages_b: int           # pages in the d_out-wide pool
 
     @property
     def T(self) -> int:
@@ -79,47 +110,50 @@ class Workload:
         return len(self.adapters)
 
     def ranks(self) -> np.ndarray:
-        return np.array([0 if a is None else a.rank for a in self.adapters], dtype=np.int32)
+        return self.adapters.rank_of.copy()
 
     def scales_f32(self) -> np.ndarray:
-        """alpha/r per slot, rounded once to fp32 (both sides widen this value)."""
-        out = np.zeros(self.S, dtype=np.float32)
-        for i, a in enumerate(self.adapters):
-            if a is not None:
-                out[i] = np.float32(a.alpha) / np.float32(a.rank)
+        """alpha/r per slot (alpha = 2r), rounded once to fp32; both sides widen this value."""
+        r = self.adapters.rank_of
+        out = np.zeros(len(r), dtype=np.float32)
+        nz = r > 0
+        out[nz] = np.float32(2.0) * r[nz].astype(np.float32) / r[nz].astype(np.float32)
         return out
 
-
-def _draw_adapter(rng: np.random.Generator, d_in: int, d_out: int, r: int) -> Adapter:
-    A = bf16_round(rng.standard_normal((d_in, r), dtype=np.float32) / np.sqrt(d_in))
-    B = bf16_round(rng.standard_normal((r, d_out), dtype=np.float32) / np.sqrt(r))
-    return Adapter(rank=r, alpha=2.0 * r, A=A, B=B)
+    def distinct(self) -> int:
+        v = self.ids[(self.ids >= 0) & (self.ids < self.S)]
+        return int(len(np.unique(v)))
 
 
-def _assign_pages(rng: np.random.Generator, ranks: np.ndarray, extra_pages: int = 3):
+def _assign_pages(seed: int, ranks: np.ndarray, extra_pages: int = 3):
     """Shuffled physical page ids for every (slot, matrix, page) of the resident adapters."""
+    rng = np.random.default_rng([seed, 5])
     S = len(ranks)
-    need = np.array([(int(r) + PAGE_ROWS - 1) // PAGE_ROWS for r in ranks], dtype=np.int64)
+    need = (np.maximum(ranks, 0).astype(np.int64) + PAGE_ROWS - 1) // PAGE_ROWS
     total = int(need.sum())
     pid = np.full((S, 2, 4), -1, dtype=np.int32)
     n_pool = total + extra_pages
     for m in range(2):
-        order = rng.permutation(n_pool)[:total]
+        order = rng.permutation(n_pool)[:total].astype(np.int32)
         k = 0
         for i in range(S):
-            for p in range(int(need[i])):
-                pid[i, m, p] = order[k]
-                k += 1
+            c = int(need[i])
+            pid[i, m, :c] = order[k:k + c]
+            k += c
     return pid, n_pool, n_pool
 
 
-def _finish(name, rng, d_in, d_out, T, ids, adapters) -> Workload:
-    X = bf16_round(rng.standard_normal((T, d_in), dtype=np.float32) / np.sqrt(d_in))
-    Y_base = rng.standard_normal((T, d_out), dtype=np.float32)
-    ranks = np.array([0 if a is None else a.rank for a in adapters], dtype=np.int32)
-    pid, na, nb = _assign_pages(rng, ranks)
+def _finish(name, seed, d_in, d_out, ids, ranks) -> Workload:
+    T = len(ids)
+    rx = np.random.default_rng([seed, 2])
+    X = bf16_round(rx.standard_normal((T, d_in), dtype=np.float32) / np.float32(np.sqrt(d_in)))
+    ry = np.random.default_rng([seed, 3])
+    Y_base = ry.standard_normal((T, d_out), dtype=np.float32)
+    ranks = np.asarray(ranks, dtype=np.int32)
+    pid, na, nb = _assign_pages(seed, ranks)
     return Workload(name=name, d_in=d_in, d_out=d_out, X=X, Y_base=Y_base,
-                    ids=np.ascontiguousarray(ids, dtype=np.int32), adapters=adapters,
+                    ids=np.ascontiguousarray(ids, dtype=np.int32),
+                    adapters=Adapters(seed, d_in, d_out, ranks, cache=len(ranks) <= 256),
                     page_ids=pid, pages_a=na, pages_b=nb)
 
 
@@ -129,53 +163,46 @@ def _finish(name, rng, d_in, d_out, T, ids, adapters) -> Workload:
 
 def tiny(seed: int = 0) -> Workload:
     """d_in = d_out = 256, 8 decode tokens, 3 adapters of rank 4, 8, 16, uniform ids."""
-    rng = np.random.default_rng(seed)
-    d = 256
-    adapters = [_draw_adapter(rng, d, d, r) for r in (4, 8, 16)]
+    rng = np.random.default_rng([seed, 1])
     ids = rng.integers(0, 3, size=8)
-    return _finish("tiny_d256_T8", rng, d, d, 8, ids, adapters)
+    return _finish("tiny_d256_T8", seed, 256, 256, ids, [4, 8, 16])
 
 
 def decode_q_proj_7b(seed: int = 1, T: int = 64) -> Workload:
     """d = 4096, one token per sequence, 32 resident rank-16 adapters drawn
     Zipf(1.0) without replacement from a 1000-adapter catalogue; each token draws
     a resident adapter with its renormalised Zipf weight."""
-    rng = np.random.default_rng(seed)
-    d = 4096
+    rng = np.random.default_rng([seed, 1])
     w = zipf_weights(1000, 1.0)
     cat = rng.choice(1000, size=32, replace=False, p=w)
     p = w[cat] / w[cat].sum()
-    adapters = [_draw_adapter(rng, d, d, 16) for _ in range(32)]
     ids = rng.choice(32, size=T, p=p)
-    return _finish(f"decode_q_proj_7b_T{T}", rng, d, d, T, ids, adapters)
+    return _finish(f"decode_q_proj_7b_T{T}", seed, 4096, 4096, ids, [16] * 32)
 
 
 def mixed_mlp(seed: int = 2, which: str = "up", T: int = 256) -> Workload:
     """256 decode tokens through the MLP up (4096 -> 11008) or down (11008 -> 4096)
     projection; 128 resident adapters with ranks uniform over {8,16,32,64};
     tokens assigned by Zipf(1.1) over the resident slots."""
-    rng = np.random.default_rng(seed)
+    rng = np.random.default_rng([seed, 1])
     d_in, d_out = (4096, 11008) if which == "up" else (11008, 4096)
     ranks = rng.choice(np.array([8, 16, 32, 64]), size=128)
-    adapters = [_draw_adapter(rng, d_in, d_out, int(r)) for r in ranks]
     slot_order = rng.permutation(128)
     ids = slot_order[rng.choice(128, size=T, p=zipf_weights(128, 1.1))]
-    return _finish(f"mixed_mlp_{which}_T{T}", rng, d_in, d_out, T, ids, adapters)
+    return _finish(f"mixed_mlp_{which}_T{T}", seed, d_in, d_out, ids, ranks)
 
 
 def prefill(seed: int = 3, n_seq: int = 16, len_lo: int = 128, len_hi: int = 2048,
             d: int = 4096) -> Workload:
     """16 sequences of length uniform in [128, 2048], each one adapter; 6 distinct
     adapters with ranks drawn from {8,16,32,64}; tokens of a sequence are contiguous."""
-    rng = np.random.default_rng(seed)
+    rng = np.random.default_rng([seed, 1])
     n_ad = 6
     ranks = rng.choice(np.array([8, 16, 32, 64]), size=n_ad)
-    adapters = [_draw_adapter(rng, d, d, int(r)) for r in ranks]
     lens = rng.integers(len_lo, len_hi + 1, size=n_seq)
     seq_ad = rng.permutation(np.arange(n_seq) % n_ad)
     ids = np.concatenate([np.full(int(L), int(a)) for L, a in zip(lens, seq_ad)])
-    T = int(lens.sum())
-    return _finish(f"prefill_{n_seq}seq_T{T}", rng, d, d, T, ids, adapters)
+    return _finish(f"prefill_{n_seq}seq_T{len(ids)}", seed, d, d, ids, ranks)
 
 
 def sweep_8b(seed: int = 4, T: int = 64, regime: str = "distinct", pool: int = 512,
@@ -183,29 +210,40 @@ def sweep_8b(seed: int = 4, T: int = 64, regime: str = "distinct", pool: int = 5
     """d_in = 4096, d_out = 14336, rank 64, a pool of 512 resident adapters;
     regime "one": every token on one adapter; "distinct": token t uses
     perm[t mod 512] so min(T, 512) distinct adapters."""
-    rng = np.random.default_rng(seed)
-    adapters = [_draw_adapter(rng, d_in, d_out, rank) for _ in range(pool)]
+    rng = np.random.default_rng([seed, 1])
     if regime == "one":
         ids = np.full(T, int(rng.integers(0, pool)))
     else:
         perm = rng.permutation(pool)
         ids = perm[np.arange(T) % pool]
-    return _finish(f"sweep_8b_{regime}_T{T}", rng, d_in, d_out, T, ids, adapters)
+    return _finish(f"sweep_8b_{regime}_T{T}", seed, d_in, d_out, ids, [rank] * pool)
 
 
 def random_small(seed: int, T: int, d_in: int, d_out: int, S: int,
                  ranks=(1, 4, 8, 16), p_none: float = 0.1, p_empty: float = 0.0) -> Workload:
     """Random small case: mixed ranks, some id = -1 tokens, optional empty slots."""
-    rng = np.random.default_rng(seed)
-    adapters: List[Optional[Adapter]] = []
-    for _ in range(S):
-        if rng.random() < p_empty:
-            adapters.append(None)
-        else:
-            adapters.append(_draw_adapter(rng, d_in, d_out, int(rng.choice(np.array(ranks)))))
+    rng = np.random.default_rng([seed, 1])
+    rk = rng.choice(np.array(ranks), size=S)
+    rk[rng.random(S) < p_empty] = 0
     ids = rng.integers(0, S, size=T)
     ids[rng.random(T) < p_none] = -1
-    return _finish(f"random_T{T}_{d_in}x{d_out}_S{S}", rng, d_in, d_out, T, ids, adapters)
+    return _finish(f"random_T{T}_{d_in}x{d_out}_S{S}", seed, d_in, d_out, ids, rk)
+
+
+def segments(seed: int, lens, d_in: int, d_out: int, S: int, ranks=(1, 4, 8, 16, 33, 64),
+             reuse: bool = False) -> Workload:
+    """Prefill-like batch: sequence i brings lens[i] consecutive tokens that all use
+    one adapter slot (distinct slots unless `reuse`, which lets sequences share a
+    slot so that its tokens are no longer contiguous)."""
+    rng = np.random.default_rng([seed, 1])
+    rk = rng.choice(np.array(ranks), size=S)
+    if reuse:
+        seg_slot = rng.integers(0, S, size=len(lens))
+    else:
+        assert len(lens) <= S
+        seg_slot = rng.permutation(S)[:len(lens)]
+    ids = np.concatenate([np.full(int(L), int(a)) for L, a in zip(lens, seg_slot)]) if len(lens) else np.zeros(0)
+    return _finish(f"segments_{len(lens)}_T{len(ids)}_{d_in}x{d_out}", seed, d_in, d_out, ids, rk)
 
 
 def by_name(name: str, **kw) -> Workload:
@@ -219,6 +257,20 @@ def by_name(name: str, **kw) -> Workload:
         "sweep_8b_distinct": lambda **k: sweep_8b(regime="distinct", **k),
     }
     return table[name](**kw)
+
+
+def subset_for_tokens(wl: Workload, tokens) -> tuple:
+    """(X, Y_base, ids, A list, B list, scales) restricted to `tokens`, with the
+    slots they use renumbered 0..k-1 (to run the oracle on sampled outputs)."""
+    tokens = np.asarray(tokens, dtype=np.int64)
+    ids = wl.ids[tokens]
+    used = sorted({int(i) for i in ids if 0 <= i < wl.S and wl.adapters.rank_of[i] > 0})
+    remap = {s: j for j, s in enumerate(used)}
+    new_ids = np.array([remap.get(int(i), -1 if i == -1 else len(used) + 7) for i in ids], dtype=np.int32)
+    A = [wl.adapters[s].A for s in used]
+    Bm = [wl.adapters[s].B for s in used]
+    sc = wl.scales_f32()[used] if used else np.zeros(0, np.float32)
+    return wl.X[tokens], wl.Y_base[tokens], new_ids, A, Bm, sc
 
 
 def shard_tokens(T: int, rank: int, world: int):
