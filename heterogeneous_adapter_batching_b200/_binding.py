@@ -20,6 +20,7 @@ LORA_OK = 0
 ERR_NAMES = {
     -1: "LORA_ERR_INVALID_ARG", -2: "LORA_ERR_BAD_RANK", -3: "LORA_ERR_WIDTH_MISMATCH",
     -4: "LORA_ERR_POOL_OOM", -5: "LORA_ERR_BAD_SLOT", -6: "LORA_ERR_CUDA", -7: "LORA_ERR_WORKSPACE",
+    -8: "LORA_ERR_TOO_LARGE",
 }
 DEV_ERR_BAD_ID = 1
 DEV_ERR_EMPTY_SLOT = 2
@@ -31,11 +32,13 @@ MAX_PAGES_PER_MATRIX = 4
 MAX_SLOTS = 4096
 OPT_LONG_SEGMENT = 1
 OPT_DECODE_JOB_TOKENS = 2
+NOALLOC_MAX_TOKENS = 32768
+NOALLOC_SCRATCH_BYTES = 1310720
 
 EXPORTS = [
     "lora_pool_create", "lora_pool_destroy", "lora_pool_free_pages", "lora_pool_num_pages",
     "lora_pool_load", "lora_pool_evict", "lora_pool_read_row", "lora_workspace_size",
-    "lora_plan", "lora_shrink", "lora_expand_add", "lora_apply", "lora_apply_planned",
+    "lora_plan", "lora_shrink", "lora_expand_add", "lora_apply", "lora_apply_planned", "lora_apply_noalloc",
     "lora_set_option", "lora_get_option", "lora_last_cuda_error", "lora_last_launch_count",
 ]
 
@@ -75,6 +78,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lora_expand_add": (I, [V, V, I, I, V, I, V, V, V, V, V, Z, V, V]),
         "lora_apply": (I, [V, V, I, I, I, V, I, V, V, V, V, V, V, Z, V, V]),
         "lora_apply_planned": (I, [V, V, I, I, I, I, V, V, V, V, V, V, Z, V, V]),
+        "lora_apply_noalloc": (I, [V, V, I, I, I, V, I, V, V, V, V, V, V, V]),
         "lora_set_option": (I, [I, I]),
         "lora_get_option": (I, [I]),
         "lora_last_cuda_error": (ctypes.c_char_p, []),
@@ -210,6 +214,15 @@ def lora_apply_planned(X, Y, T, d_in, d_out, num_slots, ranks, scales, page_tabl
     _check("lora_apply_planned", load_library().lora_apply_planned(
         _p(X), _p(Y), T, d_in, d_out, num_slots, _p(ranks), _p(scales), _p(page_table),
         pa._h, pb._h, _p(ws), ws.numel() * ws.element_size(), _p(err), _s(stream)))
+
+
+def lora_apply_noalloc(X, Y, T, d_in, d_out, ids, num_slots, ranks, scales, page_table, pa: Pool, pb: Pool,
+                       err=None, stream=None) -> None:
+    """lora_apply without a workspace: the plan lives in the library's fixed device
+    scratch, for callers that cannot allocate device memory (see include/lora.h)."""
+    _check("lora_apply_noalloc", load_library().lora_apply_noalloc(
+        _p(X), _p(Y), T, d_in, d_out, _p(ids), num_slots, _p(ranks), _p(scales), _p(page_table),
+        pa._h, pb._h, _p(err), _s(stream)))
 
 
 def lora_set_option(key: int, value: int) -> None:

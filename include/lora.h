@@ -53,6 +53,7 @@ typedef struct lora_pool_s *lora_pool_t;        /* opaque host handle of one pag
 #define LORA_ERR_BAD_SLOT       -5   /* slot outside [0, num_slots), or page id not free / out of range */
 #define LORA_ERR_CUDA           -6   /* a CUDA runtime call failed; see lora_last_cuda_error() */
 #define LORA_ERR_WORKSPACE      -7   /* ws is NULL or ws_bytes < lora_workspace_size(...) */
+#define LORA_ERR_TOO_LARGE      -8   /* lora_apply_noalloc: T or num_slots beyond its fixed scratch */
 
 /* Device error word bits. */
 #define LORA_DEV_ERR_BAD_ID      1   /* some id < -1 or id >= num_slots */
@@ -187,6 +188,34 @@ int lora_apply(const uint16_t *X, float *Y, int T, int d_in, int d_out, const in
 int lora_apply_planned(const uint16_t *X, float *Y, int T, int d_in, int d_out, int num_slots,
                        const int32_t *ranks, const float *scales, const int32_t *page_table,
                        lora_pool_t pa, lora_pool_t pb, void *ws, size_t ws_bytes,
+                       int32_t *err_dev, lora_stream_t stream);
+
+/* lora_apply without a workspace argument, for callers that cannot allocate
+ * device memory: e.g. a plug-in inside a host framework that owns all device
+ * memory through its own pool and forbids outside allocations, or a
+ * latency-critical serving loop that must not call cudaMalloc/cudaFree
+ * because they can synchronise the device.  The pages describe no such call;
+ * it has no counterpart there.
+ *
+ * Same arguments, result and error-word behaviour as lora_apply, minus
+ * (ws, ws_bytes).  The segment plan lives in one fixed scratch array of
+ * LORA_NOALLOC_SCRATCH_BYTES that is a static __device__ variable of the
+ * library: every GPU that loads the library holds it until the process exits,
+ * and the library itself never calls cudaMalloc, cudaFree or any allocating
+ * routine.  Limits: T <= LORA_NOALLOC_MAX_TOKENS and num_slots <=
+ * LORA_MAX_SLOTS; larger sizes return LORA_ERR_TOO_LARGE before any work is
+ * enqueued.  The first call on a device looks up the scratch's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.  All calls share the one array (it keeps the
+ * last call's contents; each call writes everything it reads, so nothing needs
+ * clearing), so calls whose kernels overlap on the GPU - on different streams
+ * or from different host threads without ordering - race and give undefined
+ * results: order them on one stream. */
+#define LORA_NOALLOC_MAX_TOKENS    32768
+#define LORA_NOALLOC_SCRATCH_BYTES 1310720   /* 1.25 MiB */
+int lora_apply_noalloc(const uint16_t *X, float *Y, int T, int d_in, int d_out, const int32_t *ids,
+                       int num_slots, const int32_t *ranks, const float *scales,
+                       const int32_t *page_table, lora_pool_t pa, lora_pool_t pb,
                        int32_t *err_dev, lora_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
