@@ -33,7 +33,7 @@ MAX_SLOTS = 4096
 OPT_LONG_SEGMENT = 1
 OPT_DECODE_JOB_TOKENS = 2
 NOALLOC_MAX_TOKENS = 32768
-NOALLOC_SCRATCH_BYTES = 1310720
+NOALLOC_SCRATCH_BYTES = 2097152
 
 EXPORTS = [
     "lora_pool_create", "lora_pool_destroy", "lora_pool_free_pages", "lora_pool_num_pages",

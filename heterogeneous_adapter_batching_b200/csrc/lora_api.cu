@@ -254,14 +254,7 @@ static int check_common(int T, int num_slots, const int32_t *ids, const int32_t 
 }
 
 static PlanOut plan_out(void *ws, int T, int S, int32_t *perm_out, int32_t *seg_out) {
-    const WsLayout l = ws_layout(T, S);
-    char *b = static_cast<char *>(ws);
-    PlanOut o;
-    o.header = reinterpret_cast<PlanHeader *>(b + l.header);
-    o.seg_start = reinterpret_cast<int32_t *>(b + l.seg_start);
-    o.perm = reinterpret_cast<int32_t *>(b + l.perm);
-    o.jobs = reinterpret_cast<int4 *>(b + l.jobs);
-    o.tiles = reinterpret_cast<int4 *>(b + l.tiles);
+    PlanOut o = plan_in_ws(ws, T, S);
     o.perm_copy = perm_out;
     o.seg_start_copy = seg_out;
     return o;
@@ -276,11 +269,11 @@ static int run_planned(const uint16_t *X, float *Y, int T, int d_in, int d_out, 
                        lora_pool_t pb, void *ws, int32_t *err_dev, cudaStream_t st) {
     const PlanOut o = plan_out(ws, T, num_slots, nullptr, nullptr);
     GatherArgs a = {};
-    a.X = X; a.Y = Y; a.T = T; a.d_in = d_in; a.d_out = d_out;
+    a.X = X; a.Y = Y; a.T = T; a.d_in = d_in; a.d_out = d_out; a.S = num_slots;
     a.ranks = ranks; a.scales = scales; a.pt = page_table; a.poolA = pa->base; a.poolB = pb->base;
-    a.perm = o.perm; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
+    a.perm = o.perm_short; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
     a.rowsA = (long long)pa->num_pages * LORA_PAGE_ROWS; a.rowsB = (long long)pb->num_pages * LORA_PAGE_ROWS;
-    if (int rc = launch_gather(kApply, a, st, true)) return rc;
+    if (int rc = launch_gather(kApply, a, pa, pb, st, true)) return rc;
     if (plan_uses_tiles(T)) {
         TileArgs ta = {};
         ta.X = X; ta.Y = Y; ta.T = T; ta.d_in = d_in; ta.d_out = d_out;
@@ -328,11 +321,11 @@ int lora_shrink(const uint16_t *X, int T, int d_in, const int32_t *ids, int num_
     const PlanOut o = plan_out(ws, T, num_slots, nullptr, nullptr);
     if (int rc = launch_plan(ids, T, ranks, num_slots, 0, opt_job_tokens(), o, err_dev, st)) return rc;
     GatherArgs a = {};
-    a.X = X; a.V = V; a.T = T; a.d_in = d_in; a.d_out = 8;
+    a.X = X; a.V = V; a.T = T; a.d_in = d_in; a.d_out = 8; a.S = num_slots;
     a.ranks = ranks; a.pt = page_table; a.poolA = pa->base;
-    a.perm = o.perm; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
+    a.perm = o.perm_short; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
     a.rowsA = (long long)pa->num_pages * LORA_PAGE_ROWS;
-    return launch_gather(kShrink, a, st, true);
+    return launch_gather(kShrink, a, pa, pa, st, true);
 }
 
 int lora_expand_add(const float *V, float *Y, int T, int d_out, const int32_t *ids, int num_slots,
@@ -348,11 +341,11 @@ int lora_expand_add(const float *V, float *Y, int T, int d_out, const int32_t *i
     const PlanOut o = plan_out(ws, T, num_slots, nullptr, nullptr);
     if (int rc = launch_plan(ids, T, ranks, num_slots, 0, opt_job_tokens(), o, err_dev, st)) return rc;
     GatherArgs a = {};
-    a.V = const_cast<float *>(V); a.Y = Y; a.T = T; a.d_in = 8; a.d_out = d_out;
+    a.V = const_cast<float *>(V); a.Y = Y; a.T = T; a.d_in = 8; a.d_out = d_out; a.S = num_slots;
     a.ranks = ranks; a.scales = scales; a.pt = page_table; a.poolB = pb->base;
-    a.perm = o.perm; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
+    a.perm = o.perm_short; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
     a.rowsB = (long long)pb->num_pages * LORA_PAGE_ROWS;
-    return launch_gather(kExpand, a, st, true);
+    return launch_gather(kExpand, a, pb, pb, st, true);
 }
 
 int lora_apply(const uint16_t *X, float *Y, int T, int d_in, int d_out, const int32_t *ids, int num_slots,

@@ -9,46 +9,57 @@
 // added to the base output.  Section "Unified Paging Architecture": the
 // weights are read straight out of the physical pages the page table names.
 //
-// Work unit = one gather job (an adapter slot and up to 8 of its tokens, from
+// Work unit = one gather job (an adapter slot and up to 4 of its tokens, from
 // the plan kernel) times one part e of an E-way split of d_out.  A cluster of
 // kCS CTAs runs one unit at a time and loops over the units (persistent grid
 // sized from the occupancy of the cluster shape).  Per CTA:
-//   * a producer warp streams the unit's rows into a ring of shared-memory
-//     stages with bulk asynchronous copies (cp.async.bulk, completion on an
-//     mbarrier): first the CTA's 1/kCS slice of d_in (rank rows of A^T from
-//     the pages, and the tokens' X rows), then its slice of d_out (rank rows
-//     of B, and the tokens' Y rows).  Only the r_i rows the adapter has are
-//     copied.  The producer runs ahead into the next unit while the
-//     consumers finish the current one, so B and Y are in flight during the
-//     shrink;
-//   * 8 consumer warps compute the shrink partial sums over the d_in slice
-//     (warps take rank rows, lanes take 8-column groups, warp shuffles reduce
-//     the lanes) and push them into every peer CTA's shared memory
-//     (distributed shared memory stores, then a release arrive on the peer's
-//     mbarrier);
+//   * a producer warp streams the adapter's pages into a ring of shared-memory
+//     stages with 2D TMA loads, one page (16 rank rows) by 256 columns per
+//     instruction: first the CTA's 1/kCS slice of d_in (rows of A^T), then its
+//     slice of d_out (rows of B).  It runs ahead into the next unit while the
+//     consumers finish the current one.  Only the pages the adapter has are
+//     read; a rank that is not a multiple of 16 reads the zeroed rows of its
+//     last page;
+//   * 8 consumer warps read the tokens' X and Y values straight from global
+//     memory (coalesced, issued before they wait for the weights), compute the
+//     shrink partial sums over the d_in slice (warps take rank rows, lanes take
+//     8-column groups, warp shuffles reduce the lanes) and push them into
+//     every peer CTA's shared memory (distributed shared memory stores, then a
+//     release arrive on the peer's mbarrier);
 //   * each CTA sums the kCS partials in rank order, so all CTAs hold the same
 //     fp32 v and the result is bit-reproducible, then expands its d_out slice:
-//     threads take columns, read B and the old Y from the stage and store the
-//     new Y row segments with coalesced stores.
-// Every wait is bounded; a wait that runs out sets LORA_DEV_ERR_TIMEOUT in the
-// error word and the kernel runs to completion without trapping.
+//     threads take columns, read B from the stage and store the new Y values
+//     with coalesced stores.
+// Small page tables (<= 256 slots) are staged in shared memory before the
+// kernel waits for the plan, so a unit's metadata costs one global read (the
+// job record).  Every wait is bounded; a wait that runs out sets
+// LORA_DEV_ERR_TIMEOUT in the error word and the kernel runs to completion
+// without trapping.  No cluster multicast is used.
 #include "lora_internal.cuh"
 
 namespace lora {
 namespace {
 
-constexpr int kCS = 8;                 // CTAs per cluster
+constexpr int kCS = 8;                       // CTAs per cluster
 constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kNT = 4;                 // max tokens per job
-constexpr int kStages = 4;
-constexpr int kStageBytes = 16384;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kThreads = kConsumers + 32;    // + one producer warp
+constexpr int kNT = 4;                       // max tokens per job
+constexpr int kStages = 2;
+constexpr int kBoxCols = 256;                // TMA box: 16 rows x 256 columns of bf16 = 8 KB
+constexpr int kBoxBytes = LORA_PAGE_ROWS * kBoxCols * 2;
+constexpr int kStageBoxes = 4;               // a stage holds 4 boxes = 32 KB
+constexpr int kTableSlots = 256;             // page tables up to this many slots live in shared memory
 constexpr long long kWaitLimit = 2000000000LL;   // cycles (~1 s)
 
-struct __align__(16) GatherSmem {
-    unsigned char stage[kStages][kStageBytes];
+struct __align__(128) GatherSmem {
+    unsigned char stage[kStages][kStageBoxes * kBoxBytes];   // box (page p, column block b) at (p * nb + b) * 8 KB
     float P[2][kCS][kNT * LORA_MAX_RANK];     // partial sums pushed by each peer, [t * r + k]
-    float4 v[LORA_MAX_RANK];                  // reduced v, [k] holds tokens 0..3
+    float4 v[LORA_MAX_RANK];                  // reduced v: v[k] holds tokens 0..3
+    uint4 xs[2][kNT][kStageBoxes * kBoxCols / 8];   // the chunk's X columns per token (double-buffered)
+    int4 pt[kTableSlots * 2];                 // staged page-table rows (A pages, B pages)
+    int ranks[kTableSlots];
+    float scales[kTableSlots];
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t xbar[2];
@@ -101,6 +112,15 @@ __device__ __forceinline__ void mbar_wait(uint64_t *bar, uint32_t parity, Gather
     }
 }
 
+// Bounded wait for this thread's own copies before it exits, not cut short
+// by the abort flag.
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
+    const uint32_t a = smem_u32(bar);
+    const long long t0 = clock64();
+    while (!mbar_try(a, parity) && clock64() - t0 < kWaitLimit / 8) {
+    }
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -109,10 +129,10 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+__device__ __forceinline__ void tma_load_box(void *dst, const CUtensorMap *m, int x, int y, uint64_t *bar) {
     asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ uint32_t map_peer(uint32_t addr, uint32_t rank) {
@@ -136,12 +156,8 @@ __device__ __forceinline__ uint32_t cluster_rank() {
     return r;
 }
 
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
 __device__ __forceinline__ void consumer_sync() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory");
 }
 
 __device__ __forceinline__ void bf16x8(const uint4 &v, float f[8]) {
@@ -151,64 +167,79 @@ __device__ __forceinline__ void bf16x8(const uint4 &v, float f[8]) {
     f[6] = __uint_as_float(v.w << 16); f[7] = __uint_as_float(v.w & 0xffff0000u);
 }
 
-// Column ranges, in units of 8 columns (16 bytes of bf16), of the CTA's
-// slices and the chunk widths that fit one stage.
+// Per-slot data of this call, from the shared-memory copy when staged.
+struct SlotMeta {
+    int r;           // rank, or 0 to skip the unit
+    int np;          // pages per matrix
+    int4 pga, pgb;   // page ids of A^T and B
+    float scale;
+    bool bad;
+};
+
+template <int MODE>
+__device__ __forceinline__ SlotMeta slot_meta(const GatherArgs &a, const GatherSmem &sm, bool staged, int slot) {
+    SlotMeta m;
+    int r;
+    if (staged) {
+        r = sm.ranks[slot];
+        m.pga = sm.pt[2 * slot];
+        m.pgb = sm.pt[2 * slot + 1];
+        m.scale = sm.scales[slot];
+    } else {
+        r = a.ranks[slot];
+        m.pga = reinterpret_cast<const int4 *>(a.pt)[2 * slot];
+        m.pgb = reinterpret_cast<const int4 *>(a.pt)[2 * slot + 1];
+        m.scale = (MODE == kShrink) ? 0.f : a.scales[slot];
+    }
+    m.bad = r > LORA_MAX_RANK;
+    if (r <= 0 || m.bad) r = 0;
+    const int np = (r + LORA_PAGE_ROWS - 1) / LORA_PAGE_ROWS;
+    const int pa[4] = {m.pga.x, m.pga.y, m.pga.z, m.pga.w};
+    const int pb[4] = {m.pgb.x, m.pgb.y, m.pgb.z, m.pgb.w};
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        if (p < np) {
+            if (MODE != kExpand && (pa[p] < 0 || (long long)(pa[p] + 1) * LORA_PAGE_ROWS > a.rowsA)) m.bad = true;
+            if (MODE != kShrink && (pb[p] < 0 || (long long)(pb[p] + 1) * LORA_PAGE_ROWS > a.rowsB)) m.bad = true;
+        }
+    }
+    m.r = m.bad ? 0 : r;
+    m.np = m.bad ? 0 : np;
+    return m;
+}
+
+// Column geometry of one unit for this CTA (columns, multiples of 8).
 struct UnitGeom {
-    int r, n;
-    int in_g0, in_g1, kw;    // d_in slice [in_g0, in_g1) groups; shrink chunk width in groups
-    int out_g0, out_g1, cw;  // d_out slice; expand chunk width in groups
+    int in0, in1;        // d_in slice
+    int out0, out1;      // d_out slice
+    int nb;              // 256-column boxes per chunk (chunk width nb * 256)
     int n_shrink, n_expand;
 };
 
-// The slot's rank for this call, or 0 when the rank or any page it needs is
-// out of range (the unit is then skipped: its Y rows stay untouched).  Every
-// thread of the CTA evaluates it on the same data, so all agree.
 template <int MODE>
-__device__ __forceinline__ int checked_rank(const GatherArgs &a, int slot, bool &bad) {
-    int r = a.ranks[slot];
-    bad = false;
-    if (r <= 0) return 0;
-    if (r > LORA_MAX_RANK) { bad = true; return 0; }
-    const int np = (r + LORA_PAGE_ROWS - 1) / LORA_PAGE_ROWS;
-    for (int p = 0; p < np; ++p) {
-        if (MODE != kExpand) {
-            const int pg = a.pt[slot * 8 + p];
-            if (pg < 0 || (long long)(pg + 1) * LORA_PAGE_ROWS > a.rowsA) bad = true;
-        }
-        if (MODE != kShrink) {
-            const int pg = a.pt[slot * 8 + 4 + p];
-            if (pg < 0 || (long long)(pg + 1) * LORA_PAGE_ROWS > a.rowsB) bad = true;
-        }
-    }
-    return bad ? 0 : r;
-}
-
-template <int MODE>
-__device__ __forceinline__ UnitGeom unit_geom(const GatherArgs &a, int r, int n, int e, int E, int crank) {
+__device__ __forceinline__ UnitGeom unit_geom(const GatherArgs &a, int np, int e, int E, int crank) {
     UnitGeom g;
-    g.r = r;
-    g.n = n;
     const int Gi = a.d_in >> 3, Go = a.d_out >> 3;
-    g.in_g0 = (int)((long long)Gi * crank / kCS);
-    g.in_g1 = (int)((long long)Gi * (crank + 1) / kCS);
+    g.in0 = 8 * (int)((long long)Gi * crank / kCS);
+    g.in1 = 8 * (int)((long long)Gi * (crank + 1) / kCS);
     const int ge0 = (int)((long long)Go * e / E), ge1 = (int)((long long)Go * (e + 1) / E);
-    g.out_g0 = ge0 + (int)((long long)(ge1 - ge0) * crank / kCS);
-    g.out_g1 = ge0 + (int)((long long)(ge1 - ge0) * (crank + 1) / kCS);
-    // Chunk widths (in 16-byte column groups) sized for the largest job, so that
-    // they depend on the rank only: a token's fp32 summation order is then the
-    // same whichever job it lands in, and results do not depend on batch order.
-    // Shrink: r + kNT rows of 16 B per group; expand: r rows of 16 B + kNT rows of 32 B.
-    g.kw = kStageBytes / ((r + kNT) * 16);
-    g.cw = kStageBytes / (r * 16 + kNT * 32);
-    const int win = g.in_g1 - g.in_g0, wout = g.out_g1 - g.out_g0;
-    g.n_shrink = (MODE == kExpand || win <= 0 || r == 0) ? 0 : (win + g.kw - 1) / g.kw;
-    g.n_expand = (MODE == kShrink || wout <= 0 || r == 0) ? 0 : (wout + g.cw - 1) / g.cw;
+    g.out0 = 8 * (ge0 + (int)((long long)(ge1 - ge0) * crank / kCS));
+    g.out1 = 8 * (ge0 + (int)((long long)(ge1 - ge0) * (crank + 1) / kCS));
+    // As many 256-column boxes per chunk as fit next to the rank's pages: the
+    // chunk width depends on the rank only, so a token's fp32 summation order
+    // does not depend on which job it lands in.
+    g.nb = np > 0 ? kStageBoxes / np : 1;
+    const int cw = g.nb * kBoxCols;
+    const int win = g.in1 - g.in0, wout = g.out1 - g.out0;
+    g.n_shrink = (MODE == kExpand || win <= 0 || np == 0) ? 0 : (win + cw - 1) / cw;
+    g.n_expand = (MODE == kShrink || wout <= 0 || np == 0) ? 0 : (wout + cw - 1) / cw;
     return g;
 }
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 2)
-gather_kernel(GatherArgs a, int e_max) {
+gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GatherArgs a,
+              int e_max) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     GatherSmem &sm = *reinterpret_cast<GatherSmem *>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -226,12 +257,35 @@ gather_kernel(GatherArgs a, int e_max) {
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    // Peers push into this CTA's barriers only after every CTA initialised them.
-    cluster_sync_all();
+    // Page tables, ranks and scales are never written by this library's kernels,
+    // and any caller write to them precedes this launch in stream order, so they
+    // are staged before waiting for the plan.
+    const bool staged = a.S <= kTableSlots;
+    if (staged) {
+        for (int i = threadIdx.x; i < a.S; i += kThreads) {
+            sm.pt[2 * i] = reinterpret_cast<const int4 *>(a.pt)[2 * i];
+            sm.pt[2 * i + 1] = reinterpret_cast<const int4 *>(a.pt)[2 * i + 1];
+            sm.ranks[i] = a.ranks[i];
+            sm.scales[i] = (MODE == kShrink) ? 0.f : a.scales[i];
+        }
+    }
+    __syncthreads();
+    // Announce this CTA's barriers to its peers; the matching wait comes just
+    // before the first push into a peer.
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 
-    // The plan kernel runs just before this one; wait for its output.
+    // The plan kernel runs before this one; wait for its output.  Then let the
+    // next kernel on the stream get its CTAs resident: it reads nothing the
+    // kernels write before its own wait, which returns only when this grid has
+    // completed.
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
 
+    // The first job record is read together with the job count (a guess that
+    // holds whenever there are at least half as many jobs as clusters).
+    const int spec = cluster_id < a.T ? cluster_id : a.T - 1;
+    const int4 spec_job = a.jobs[2 * spec];
+    const int4 spec_tok = a.jobs[2 * spec + 1];
     const int n_jobs = a.hdr->n_jobs;
     if (n_jobs <= 0) return;   // uniform over the grid; no peer traffic has happened
     int E = 1;
@@ -243,59 +297,35 @@ gather_kernel(GatherArgs a, int e_max) {
 
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------------------
-        // Producer warp: bulk copies of row segments into the stage ring.
+        // Producer warp (lane 0): TMA loads of the adapter's pages.
         // ------------------------------------------------------------------
-        int chunk = 0;
-        for (int u = cluster_id; u < n_units; u += n_clusters) {
-            const int4 job = a.jobs[u / E];
-            const int e = u - (u / E) * E;
-            const int slot = job.x, p0 = job.y, n = job.z;
-            bool bad;
-            const int r = checked_rank<MODE>(a, slot, bad);
-            const UnitGeom g = unit_geom<MODE>(a, r, n, e, E, crank);
-            // shrink chunks: rows of A^T (r) then X (n), each kw groups wide
-            for (int c = 0; c < g.n_shrink; ++c, ++chunk) {
-                const int s = chunk % kStages;
-                const uint32_t par = ((chunk / kStages) & 1) ^ 1;
-                const int c0 = g.in_g0 + c * g.kw;
-                const int w = min(g.kw, g.in_g1 - c0);
-                mbar_wait<false>(&sm.empty[s], par, sm, a.err);
-                if (lane == 0) mbar_expect_tx(&sm.full[s], (uint32_t)((r + n) * w * 16));
-                __syncwarp();
-                for (int i = lane; i < r + n; i += 32) {
-                    const uint16_t *src;
-                    if (i < r) {
-                        const int page = a.pt[slot * 8 + (i >> 4)];
-                        src = a.poolA + ((size_t)page * LORA_PAGE_ROWS + (i & 15)) * a.d_in + (size_t)c0 * 8;
-                    } else {
-                        const int t = i - r;
-                        src = a.X + (size_t)a.perm[p0 + t] * a.d_in + (size_t)c0 * 8;
-                    }
-                    bulk_g2s(sm.stage[s] + (size_t)i * w * 16, src, (uint32_t)(w * 16), &sm.full[s]);
+        if (lane == 0) {
+            int chunk = 0;
+            for (int u = cluster_id; u < n_units; u += n_clusters) {
+                const int ji = u / E;
+                const int4 job = (ji == spec) ? spec_job : a.jobs[2 * ji];
+                const int e = u - ji * E;
+                const SlotMeta m = slot_meta<MODE>(a, sm, staged, job.x);
+                const UnitGeom g = unit_geom<MODE>(a, m.np, e, E, crank);
+                const int pa[4] = {m.pga.x, m.pga.y, m.pga.z, m.pga.w};
+                const int pb[4] = {m.pgb.x, m.pgb.y, m.pgb.z, m.pgb.w};
+                for (int c = 0; c < g.n_shrink + g.n_expand; ++c, ++chunk) {
+                    const int s = chunk % kStages;
+                    mbar_wait<false>(&sm.empty[s], ((chunk / kStages) & 1) ^ 1, sm, a.err);
+                    const bool shrink = c < g.n_shrink;
+                    const int c0 = shrink ? g.in0 + c * g.nb * kBoxCols : g.out0 + (c - g.n_shrink) * g.nb * kBoxCols;
+                    const int c1 = shrink ? g.in1 : g.out1;
+                    const int boxes = min(g.nb, (c1 - c0 + kBoxCols - 1) / kBoxCols);
+                    mbar_expect_tx(&sm.full[s], (uint32_t)(m.np * boxes * kBoxBytes));
+                    for (int p = 0; p < m.np; ++p)
+                        for (int b = 0; b < boxes; ++b)
+                            tma_load_box(sm.stage[s] + (size_t)(p * g.nb + b) * kBoxBytes, shrink ? &tmA : &tmB,
+                                         c0 + b * kBoxCols, (shrink ? pa[p] : pb[p]) * LORA_PAGE_ROWS, &sm.full[s]);
                 }
             }
-            // expand chunks: rows of B (r, bf16) then Y (n, fp32)
-            for (int c = 0; c < g.n_expand; ++c, ++chunk) {
-                const int s = chunk % kStages;
-                const uint32_t par = ((chunk / kStages) & 1) ^ 1;
-                const int c0 = g.out_g0 + c * g.cw;
-                const int w = min(g.cw, g.out_g1 - c0);
-                mbar_wait<false>(&sm.empty[s], par, sm, a.err);
-                if (lane == 0) mbar_expect_tx(&sm.full[s], (uint32_t)((r * 16 + n * 32) * w));
-                __syncwarp();
-                for (int i = lane; i < r + n; i += 32) {
-                    if (i < r) {
-                        const int page = a.pt[slot * 8 + 4 + (i >> 4)];
-                        const uint16_t *src = a.poolB + ((size_t)page * LORA_PAGE_ROWS + (i & 15)) * a.d_out + (size_t)c0 * 8;
-                        bulk_g2s(sm.stage[s] + (size_t)i * w * 16, src, (uint32_t)(w * 16), &sm.full[s]);
-                    } else {
-                        const int t = i - r;
-                        const float *src = a.Y + (size_t)a.perm[p0 + t] * a.d_out + (size_t)c0 * 8;
-                        bulk_g2s(sm.stage[s] + (size_t)r * w * 16 + (size_t)t * w * 32, src, (uint32_t)(w * 32),
-                                 &sm.full[s]);
-                    }
-                }
-            }
+            // the loads armed last on each stage have landed before this thread exits
+            for (int i = (chunk > kStages ? chunk - kStages : 0); i < chunk; ++i)
+                drain_wait(&sm.full[i % kStages], (i / kStages) & 1);
         }
         return;
     }
@@ -305,15 +335,20 @@ gather_kernel(GatherArgs a, int e_max) {
     // ----------------------------------------------------------------------
     int chunk = 0;
     int iter = 0;
+    bool joined = false;   // waited on the start-up cluster barrier
     for (int u = cluster_id; u < n_units; u += n_clusters, ++iter) {
-        const int4 job = a.jobs[u / E];
-        const int e = u - (u / E) * E;
-        const int slot = job.x, p0 = job.y, n = job.z;
-        bool bad;
-        const int r = checked_rank<MODE>(a, slot, bad);
-        if (bad && threadIdx.x == 0 && crank == 0 && e == 0 && a.err) atomicOr(a.err, LORA_DEV_ERR_BAD_PAGE);
-        const UnitGeom g = unit_geom<MODE>(a, r, n, e, E, crank);
+        const int ji = u / E;
+        const int4 job = (ji == spec) ? spec_job : a.jobs[2 * ji];
+        const int4 tk = (ji == spec) ? spec_tok : a.jobs[2 * ji + 1];
+        const int e = u - ji * E;
+        const int slot = job.x, n = job.y;
+        const int tok[kNT] = {tk.x, tk.y, tk.z, tk.w};
+        const SlotMeta m = slot_meta<MODE>(a, sm, staged, slot);
+        if (m.bad && threadIdx.x == 0 && crank == 0 && e == 0 && a.err) atomicOr(a.err, LORA_DEV_ERR_BAD_PAGE);
+        const int r = m.r;
+        const UnitGeom g = unit_geom<MODE>(a, m.np, e, E, crank);
         const int buf = iter & 1;
+        const int cw = g.nb * kBoxCols;
 
         if (MODE != kExpand) {
             // ---- shrink: partial sums over this CTA's d_in slice ----
@@ -324,27 +359,36 @@ gather_kernel(GatherArgs a, int e_max) {
                 for (int t = 0; t < kNT; ++t) acc[j][t] = 0.f;
             for (int c = 0; c < g.n_shrink; ++c, ++chunk) {
                 const int s = chunk % kStages;
-                const uint32_t par = (chunk / kStages) & 1;
-                const int w = min(g.kw, g.in_g1 - (g.in_g0 + c * g.kw));
-                mbar_wait<false>(&sm.full[s], par, sm, a.err);
-                const uint4 *rows = reinterpret_cast<const uint4 *>(sm.stage[s]);
-                for (int q = lane; q < w; q += 32) {
-                    float xf[kNT][8];
+                const int c0 = g.in0 + c * cw;
+                const int wcols = min(cw, g.in1 - c0);
+                const int ng = wcols >> 3;   // 8-column groups in this chunk
+                uint4 (*xs)[kStageBoxes * kBoxCols / 8] = sm.xs[c & 1];
+                // stage the tokens' X columns of this chunk (coalesced, before the weights arrive)
+                for (int i = threadIdx.x; i < n * ng; i += kConsumers) {
+                    const int t = i / ng, q = i - t * ng;
+                    xs[t][q] = __ldg(reinterpret_cast<const uint4 *>(a.X + (size_t)tok[t] * a.d_in + c0 + q * 8));
+                }
+                mbar_wait<false>(&sm.full[s], (chunk / kStages) & 1, sm, a.err);
+                consumer_sync();
+                const unsigned char *st = sm.stage[s];
+                for (int q = lane; q < ng; q += 32) {
+                    const int b = (q * 8) / kBoxCols, cb = q * 8 - b * kBoxCols;
 #pragma unroll
-                    for (int t = 0; t < kNT; ++t)
-                        if (t < n) bf16x8(rows[(size_t)(r + t) * w + q], xf[t]);
+                    for (int t = 0; t < kNT; ++t) {
+                        if (t < n) {
+                            float xf[8];
+                            bf16x8(xs[t][q], xf);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int k = warp + j * kConsumerWarps;
-                        if (k < r) {
-                            float af[8];
-                            bf16x8(rows[(size_t)k * w + q], af);
-#pragma unroll
-                            for (int t = 0; t < kNT; ++t) {
-                                if (t < n) {
+                            for (int j = 0; j < 8; ++j) {
+                                const int k = warp + j * kConsumerWarps;
+                                if (k < r) {
+                                    float af[8];
+                                    bf16x8(*reinterpret_cast<const uint4 *>(st + (size_t)((k >> 4) * g.nb + b) * kBoxBytes +
+                                                                            (k & 15) * (kBoxCols * 2) + cb * 2),
+                                           af);
                                     float sum = acc[j][t];
 #pragma unroll
-                                    for (int i = 0; i < 8; ++i) sum = fmaf(af[i], xf[t][i], sum);
+                                    for (int i = 0; i < 8; ++i) sum = fmaf(af[i], xf[i], sum);
                                     acc[j][t] = sum;
                                 }
                             }
@@ -370,12 +414,17 @@ gather_kernel(GatherArgs a, int e_max) {
                     }
                 }
             }
+            if (!joined) {
+                asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+                joined = true;
+            }
             consumer_sync();
-            // push the partial vector [t * r + k] to every peer's slot `crank`
+            // push the partial vector [t * r + k] into every peer's slot `crank`
             const int nv = n * r;
-            for (int idx = threadIdx.x; idx < kCS * ((nv + 3) / 4); idx += kConsumerWarps * 32) {
-                const int q = idx / ((nv + 3) / 4);
-                const int v4 = idx - q * ((nv + 3) / 4);
+            const int nv4 = (nv + 3) / 4;
+            for (int idx = threadIdx.x; idx < kCS * nv4; idx += kConsumers) {
+                const int q = idx / nv4;
+                const int v4 = idx - q * nv4;
                 if (q == crank) continue;
                 const float *srcp = &sm.P[buf][crank][v4 * 4];
                 const float4 val = make_float4(srcp[0], v4 * 4 + 1 < nv ? srcp[1] : 0.f,
@@ -388,7 +437,7 @@ gather_kernel(GatherArgs a, int e_max) {
             }
             mbar_wait<true>(&sm.xbar[buf], (uint32_t)((iter >> 1) & 1), sm, a.err);
             // v[k][t] = sum over peers in rank order
-            for (int idx = threadIdx.x; idx < nv; idx += kConsumerWarps * 32) {
+            for (int idx = threadIdx.x; idx < nv; idx += kConsumers) {
                 const int t = idx / r, k = idx - t * r;
                 float sum = 0.f;
 #pragma unroll
@@ -398,53 +447,59 @@ gather_kernel(GatherArgs a, int e_max) {
             consumer_sync();
             if (MODE == kShrink) {
                 if (crank == 0) {
-                    for (int idx = threadIdx.x; idx < nv; idx += kConsumerWarps * 32) {
+                    for (int idx = threadIdx.x; idx < nv; idx += kConsumers) {
                         const int t = idx / r, k = idx - t * r;
-                        a.V[(size_t)a.perm[p0 + t] * LORA_MAX_RANK + k] = reinterpret_cast<const float *>(&sm.v[k])[t];
+                        a.V[(size_t)tok[t] * LORA_MAX_RANK + k] = reinterpret_cast<const float *>(&sm.v[k])[t];
                     }
                 }
                 consumer_sync();
                 continue;
             }
         } else {
-            for (int idx = threadIdx.x; idx < n * r; idx += kConsumerWarps * 32) {
+            for (int idx = threadIdx.x; idx < n * r; idx += kConsumers) {
                 const int t = idx / r, k = idx - t * r;
-                reinterpret_cast<float *>(&sm.v[k])[t] = a.V[(size_t)a.perm[p0 + t] * LORA_MAX_RANK + k];
+                reinterpret_cast<float *>(&sm.v[k])[t] = a.V[(size_t)tok[t] * LORA_MAX_RANK + k];
             }
             consumer_sync();
         }
 
         // ---- expand-add over this CTA's d_out slice ----
-        const float sc = a.scales[slot];
-        int tok[kNT];
-#pragma unroll
-        for (int t = 0; t < kNT; ++t) tok[t] = t < n ? a.perm[p0 + t] : 0;
+        const float sc = m.scale;
         for (int c = 0; c < g.n_expand; ++c, ++chunk) {
             const int s = chunk % kStages;
-            const uint32_t par = (chunk / kStages) & 1;
-            const int c0 = g.out_g0 + c * g.cw;
-            const int w = min(g.cw, g.out_g1 - c0);
-            mbar_wait<false>(&sm.full[s], par, sm, a.err);
-            const uint16_t *Bs = reinterpret_cast<const uint16_t *>(sm.stage[s]);
-            const float *Ys = reinterpret_cast<const float *>(sm.stage[s] + (size_t)r * w * 16);
-            const int ncol = w * 8;
-            for (int col = threadIdx.x; col < ncol; col += kConsumerWarps * 32) {
-                float accv[kNT];
+            const int c0 = g.out0 + c * cw;
+            const int wcols = min(cw, g.out1 - c0);
+            // old Y of this thread's columns, loaded before the weights arrive
+            float yv[kStageBoxes][kNT];
 #pragma unroll
-                for (int t = 0; t < kNT; ++t) accv[t] = 0.f;
+            for (int i = 0; i < kStageBoxes; ++i) {
+                const int col = threadIdx.x + i * kConsumers;
+#pragma unroll
+                for (int t = 0; t < kNT; ++t)
+                    yv[i][t] = (t < n && col < wcols) ? a.Y[(size_t)tok[t] * a.d_out + c0 + col] : 0.f;
+            }
+            mbar_wait<false>(&sm.full[s], (chunk / kStages) & 1, sm, a.err);
+            const unsigned char *st = sm.stage[s];
+#pragma unroll
+            for (int i = 0; i < kStageBoxes; ++i) {
+                const int col = threadIdx.x + i * kConsumers;
+                if (col < wcols) {
+                    const int b = col / kBoxCols, cb = col - b * kBoxCols;
+                    float accv[kNT];
+#pragma unroll
+                    for (int t = 0; t < kNT; ++t) accv[t] = 0.f;
 #pragma unroll 4
-                for (int k = 0; k < r; ++k) {
-                    const float b = __uint_as_float((uint32_t)Bs[(size_t)k * ncol + col] << 16);
-                    const float4 v0 = sm.v[k];
-                    accv[0] = fmaf(v0.x, b, accv[0]); accv[1] = fmaf(v0.y, b, accv[1]);
-                    accv[2] = fmaf(v0.z, b, accv[2]); accv[3] = fmaf(v0.w, b, accv[3]);
-                }
-#pragma unroll
-                for (int t = 0; t < kNT; ++t) {
-                    if (t < n) {
-                        const float y = fmaf(sc, accv[t], Ys[(size_t)t * ncol + col]);
-                        a.Y[(size_t)tok[t] * a.d_out + (size_t)c0 * 8 + col] = y;
+                    for (int k = 0; k < r; ++k) {
+                        const uint16_t braw = *reinterpret_cast<const uint16_t *>(
+                            st + (size_t)((k >> 4) * g.nb + b) * kBoxBytes + (k & 15) * (kBoxCols * 2) + cb * 2);
+                        const float bk = __uint_as_float((uint32_t)braw << 16);
+                        const float4 v0 = sm.v[k];
+                        accv[0] = fmaf(v0.x, bk, accv[0]); accv[1] = fmaf(v0.y, bk, accv[1]);
+                        accv[2] = fmaf(v0.z, bk, accv[2]); accv[3] = fmaf(v0.w, bk, accv[3]);
                     }
+#pragma unroll
+                    for (int t = 0; t < kNT; ++t)
+                        if (t < n) a.Y[(size_t)tok[t] * a.d_out + c0 + col] = fmaf(sc, accv[t], yv[i][t]);
                 }
             }
             __syncwarp();
@@ -452,15 +507,25 @@ gather_kernel(GatherArgs a, int e_max) {
         }
         consumer_sync();   // sm.v is rewritten by the next unit
     }
+    if (!joined) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 template <int MODE>
-int launch_mode(const GatherArgs &a, cudaStream_t st, bool pdl) {
+int launch_mode(const GatherArgs &a, lora_pool_s *pa, lora_pool_s *pb, cudaStream_t st, bool pdl) {
     static int max_clusters[64] = {};
     int dev = 0;
     if (int rc = cuda_check(cudaGetDevice(&dev))) return rc;
     if (dev < 0 || dev >= 64) return LORA_ERR_INVALID_ARG;
     const size_t smem = sizeof(GatherSmem);
+    CUtensorMap ma, mb;
+    if (MODE != kExpand) {
+        if (int rc = pool_tensor_map(pa, kPoolMapGather, &ma)) return rc;
+    }
+    if (MODE != kShrink) {
+        if (int rc = pool_tensor_map(pb, kPoolMapGather, &mb)) return rc;
+    }
+    if (MODE == kExpand) ma = mb;
+    if (MODE == kShrink) mb = ma;
 
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
@@ -492,18 +557,18 @@ int launch_mode(const GatherArgs &a, cudaStream_t st, bool pdl) {
     if (ncl < 1) ncl = 1;
     cfg.gridDim = dim3(kCS * ncl);
     cfg.numAttrs = pdl ? 2 : 1;
-    if (int rc = cuda_check(cudaLaunchKernelEx(&cfg, gather_kernel<MODE>, a, e_max))) return rc;
+    if (int rc = cuda_check(cudaLaunchKernelEx(&cfg, gather_kernel<MODE>, ma, mb, a, e_max))) return rc;
     count_launch();
     return LORA_OK;
 }
 
 }  // namespace
 
-int launch_gather(GatherMode mode, const GatherArgs &a, cudaStream_t st, bool pdl) {
+int launch_gather(GatherMode mode, const GatherArgs &a, lora_pool_s *pa, lora_pool_s *pb, cudaStream_t st, bool pdl) {
     switch (mode) {
-        case kApply: return launch_mode<kApply>(a, st, pdl);
-        case kShrink: return launch_mode<kShrink>(a, st, pdl);
-        case kExpand: return launch_mode<kExpand>(a, st, pdl);
+        case kApply: return launch_mode<kApply>(a, pa, pb, st, pdl);
+        case kShrink: return launch_mode<kShrink>(a, pa, pb, st, pdl);
+        case kExpand: return launch_mode<kExpand>(a, pa, pb, st, pdl);
     }
     return LORA_ERR_INVALID_ARG;
 }

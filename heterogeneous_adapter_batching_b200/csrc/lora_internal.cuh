@@ -1,6 +1,7 @@
 // Internal declarations shared by the liblora translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -28,19 +29,23 @@ struct PlanHeader {
 };
 
 struct WsLayout {
-    size_t header, seg_start, perm, jobs, tiles, total;
+    size_t header, seg_start, perm, perm_short, run_start, run_end, jobs, tiles, total;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 inline WsLayout ws_layout(int T, int S) {
     WsLayout l;
+    const size_t t = (size_t)(T > 0 ? T : 1);
     size_t o = 0;
-    l.header = o;    o = align_up(o + sizeof(PlanHeader), 256);
-    l.seg_start = o; o = align_up(o + sizeof(int32_t) * (size_t)(S + 1), 256);
-    l.perm = o;      o = align_up(o + sizeof(int32_t) * (size_t)(T > 0 ? T : 1), 256);
-    l.jobs = o;      o = align_up(o + sizeof(int4) * (size_t)(T > 0 ? T : 1), 256);
-    l.tiles = o;     o = align_up(o + sizeof(int4) * (size_t)(T > 0 ? T : 1), 256);
+    l.header = o;     o = align_up(o + sizeof(PlanHeader), 256);
+    l.seg_start = o;  o = align_up(o + sizeof(int32_t) * (size_t)(S + 1), 256);
+    l.perm = o;       o = align_up(o + sizeof(int32_t) * t, 256);
+    l.perm_short = o; o = align_up(o + sizeof(int32_t) * t, 256);
+    l.run_start = o;  o = align_up(o + sizeof(int32_t) * t, 256);
+    l.run_end = o;    o = align_up(o + sizeof(int32_t) * t, 256);
+    l.jobs = o;       o = align_up(o + 2 * sizeof(int4) * t, 256);   // two int4 per job
+    l.tiles = o;      o = align_up(o + sizeof(int4) * t, 256);
     l.total = o;
     return l;
 }
@@ -64,9 +69,21 @@ struct lora_pool_s {
     // (page table identity, slot, matrix) -> pages owned
     std::map<std::tuple<const void *, int, int>, std::vector<int>> owners;
     std::mutex mu;
+    // TMA descriptors of the pool, built on first use (see pool_tensor_map)
+    CUtensorMap tmap[2];
+    bool tmap_ok[2] = {false, false};
 };
 
 namespace lora {
+
+// TMA tensor maps (cuTensorMapEncodeTiled through the runtime's driver entry point).
+bool tma_supported();
+int make_tensor_map(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, uint64_t cols,
+                    uint64_t rows, uint32_t box_cols, uint32_t box_rows, bool swizzle128);
+// Pool maps: kPoolMapGather = box 256 columns x 16 rows (one page), no swizzle;
+// kPoolMapTile = box 64 columns x 16 rows, 128-byte swizzle.
+enum { kPoolMapGather = 0, kPoolMapTile = 1 };
+int pool_tensor_map(lora_pool_s *pool, int kind, CUtensorMap *out);
 
 // Process-wide options.
 int opt_long_segment();
@@ -84,11 +101,32 @@ struct PlanOut {
     PlanHeader *header;
     int32_t *seg_start;
     int32_t *perm;
-    int4 *jobs;
+    int32_t *perm_short;       // perm without the tokens of long runs (gather jobs index it)
+    int32_t *run_start;        // per token: first token of its run (scratch)
+    int32_t *run_end;          // per token: last token of its run if the run is long, else -1
+    int4 *jobs;                // per job: {slot, count, 0, 0}, {token 0..3 (-1 pad)}
     int4 *tiles;
     int32_t *perm_copy;        // optional second destination of perm (caller's buffer)
     int32_t *seg_start_copy;   // optional second destination of seg_start
 };
+
+// Pointers of the plan inside a workspace laid out by ws_layout(T, S).
+inline PlanOut plan_in_ws(void *ws, int T, int S) {
+    const WsLayout l = ws_layout(T, S);
+    char *b = static_cast<char *>(ws);
+    PlanOut o;
+    o.header = reinterpret_cast<PlanHeader *>(b + l.header);
+    o.seg_start = reinterpret_cast<int32_t *>(b + l.seg_start);
+    o.perm = reinterpret_cast<int32_t *>(b + l.perm);
+    o.perm_short = reinterpret_cast<int32_t *>(b + l.perm_short);
+    o.run_start = reinterpret_cast<int32_t *>(b + l.run_start);
+    o.run_end = reinterpret_cast<int32_t *>(b + l.run_end);
+    o.jobs = reinterpret_cast<int4 *>(b + l.jobs);
+    o.tiles = reinterpret_cast<int4 *>(b + l.tiles);
+    o.perm_copy = nullptr;
+    o.seg_start_copy = nullptr;
+    return o;
+}
 int launch_plan(const int32_t *ids, int T, const int32_t *ranks, int S, int long_thresh,
                 int job_tokens, const PlanOut &out, int32_t *err_dev, cudaStream_t st);
 
@@ -99,6 +137,7 @@ struct GatherArgs {
     float *Y;
     float *V;
     int T, d_in, d_out;
+    int S;              // slots in the page table
     const int32_t *ranks;
     const float *scales;
     const int32_t *pt;
@@ -111,7 +150,7 @@ struct GatherArgs {
     long long rowsA;   // rows in the A pool (pages * 16); 0 when unused
     long long rowsB;
 };
-int launch_gather(GatherMode mode, const GatherArgs &a, cudaStream_t st, bool pdl);
+int launch_gather(GatherMode mode, const GatherArgs &a, lora_pool_s *pa, lora_pool_s *pb, cudaStream_t st, bool pdl);
 
 struct TileArgs {
     const uint16_t *X;

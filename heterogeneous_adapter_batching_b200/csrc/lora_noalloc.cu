@@ -71,26 +71,18 @@ extern "C" int lora_apply_noalloc(const uint16_t *X, float *Y, int T, int d_in, 
     // Same launch sequence as lora_apply, with the plan kept in the scratch.
     // Every word the compute kernels read is written by the plan kernel of the
     // same call first, so nothing in the scratch has to start at zero.
-    char *b = static_cast<char *>(ws);
-    PlanOut o;
-    o.header = reinterpret_cast<PlanHeader *>(b + l.header);
-    o.seg_start = reinterpret_cast<int32_t *>(b + l.seg_start);
-    o.perm = reinterpret_cast<int32_t *>(b + l.perm);
-    o.jobs = reinterpret_cast<int4 *>(b + l.jobs);
-    o.tiles = reinterpret_cast<int4 *>(b + l.tiles);
-    o.perm_copy = nullptr;
-    o.seg_start_copy = nullptr;
+    const PlanOut o = plan_in_ws(ws, T, num_slots);
     const bool use_tiles = tiles_supported() && opt_long_segment() > 0 && T >= opt_long_segment();
     const int long_thresh = use_tiles ? opt_long_segment() : 0;
     if (int rc = launch_plan(ids, T, ranks, num_slots, long_thresh, opt_job_tokens(), o, err_dev, st)) return rc;
 
     GatherArgs a = {};
-    a.X = X; a.Y = Y; a.T = T; a.d_in = d_in; a.d_out = d_out;
+    a.X = X; a.Y = Y; a.T = T; a.d_in = d_in; a.d_out = d_out; a.S = num_slots;
     a.ranks = ranks; a.scales = scales; a.pt = page_table; a.poolA = pa->base; a.poolB = pb->base;
-    a.perm = o.perm; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
+    a.perm = o.perm_short; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
     a.rowsA = (long long)pa->num_pages * LORA_PAGE_ROWS;
     a.rowsB = (long long)pb->num_pages * LORA_PAGE_ROWS;
-    if (int rc = launch_gather(kApply, a, st, true)) return rc;
+    if (int rc = launch_gather(kApply, a, pa, pb, st, true)) return rc;
     if (use_tiles) {
         TileArgs ta = {};
         ta.X = X; ta.Y = Y; ta.T = T; ta.d_in = d_in; ta.d_out = d_out;

@@ -7,11 +7,11 @@
 // "Segmented Gather Matrix-Vector Multiplication (SGMV)": shrink v = x A on
 // the tensor cores, then expand v B scaled by alpha/r into the base output.
 //
-// Work unit = (tile, part): a tile is up to 128 consecutive tokens of one
-// segment (from the plan kernel) and a part is a slice of d_out in units of
-// 64 columns; the parts of one tile run on different CTAs when there are too
-// few tiles to fill the GPU (each recomputes the small shrink of its tile).
-// One CTA per SM, persistent over the units, warp-specialised:
+// Work: a tile is up to 128 consecutive tokens of one run (from the plan
+// kernel); an item is one tile times one 64-column n-tile of d_out.  Every CTA
+// (one per SM) takes an equal contiguous share of the items in tile-major
+// order and works through it as units of one tile each, recomputing the small
+// shrink of a tile whose items it shares with a neighbour.  Warp-specialised:
 //   warp 0     TMA producer of the shrink operands: X tile [128 x 64] and the
 //              adapter's A^T pages [16 x 64] per page, 128-byte swizzled;
 //   warp 1     TMA producer of the expand operands: B pages [16 x 64] of the
@@ -38,20 +38,21 @@ namespace {
 constexpr int kM = 128;              // tokens per tile (MMA M)
 constexpr int kKB = 64;              // shrink K block: one 128-byte swizzle row of bf16
 constexpr int kNB = 64;              // expand n-tile width (MMA N)
-constexpr int kStages = 4;           // shrink pipeline depth
+constexpr int kStages = 3;           // shrink pipeline depth
+constexpr int kBuf = 3;              // expand pipeline depth (B tile, Y tile, accumulator)
 constexpr int kThreads = 256;
-constexpr uint32_t kTmemCols = 256;  // D1 [0,64), D2[0] [64,128), D2[1] [128,192)
+constexpr uint32_t kTmemCols = 256;  // D1 [0,64), D2[b] [64 + 64b, 128 + 64b) for b < 3
 constexpr long long kWaitLimit = 2000000000LL;
 
 struct TileSmem {
     __nv_bfloat16 xs[kStages][kM * kKB];      // 16 KB each, K-major SW128
     __nv_bfloat16 as[kStages][64 * kKB];      //  8 KB each, up to 4 pages x 16 rows
     __nv_bfloat16 vs[kM * 64];                // 16 KB, V (expand A operand), K-major SW128
-    __nv_bfloat16 bs[2][64 * kNB];            //  8 KB each, B n-tile, rank rows x 64 cols (MN-major SW128)
-    float ys[2][kM * kNB];                    // 32 KB each, two SW128 boxes of [128 rows x 32 cols]
+    __nv_bfloat16 bs[kBuf][64 * kNB];         //  8 KB each, B n-tile, rank rows x 64 cols (MN-major SW128)
+    float ys[kBuf][kM * kNB];                 // 32 KB each, two SW128 boxes of [128 rows x 32 cols]
     uint64_t full[kStages], empty[kStages];
-    uint64_t bfull[2], bempty[2], yfull[2], yempty[2], accfull[2], accempty[2];
-    uint64_t shrink_done, d1_empty, v_ready, v_empty;
+    uint64_t bfull[kBuf], bempty[kBuf], yfull[kBuf], yempty[kBuf], accfull[kBuf], accempty[kBuf];
+    uint64_t shrink_done, d1_empty, v_ready, v_empty, mma_drain;
     uint32_t tmem_base;
     int abort;
 };
@@ -67,19 +68,32 @@ __device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t par) {
                  : "=r"(ok) : "r"(a), "r"(par) : "memory");
     return ok != 0;
 }
-__device__ __forceinline__ void mbar_wait(uint64_t *b, uint32_t par, TileSmem &sm, int32_t *err) {
+// Bounded wait: true when the phase completed.  On timeout it raises the
+// CTA's abort flag and records LORA_DEV_ERR_TIMEOUT; once the flag is up every
+// wait returns false at once and each role stops issuing work.
+__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t par, TileSmem &sm, int32_t *err) {
     const uint32_t a = su32(b);
-    if (mbar_try(a, par)) return;
+    if (mbar_try(a, par)) return true;
     const long long t0 = clock64();
     while (!mbar_try(a, par)) {
-        if (*(volatile int *)&sm.abort) return;
+        if (*(volatile int *)&sm.abort) return false;
         if (clock64() - t0 > kWaitLimit) {
             *(volatile int *)&sm.abort = 1;
             if (err) atomicOr(err, LORA_DEV_ERR_TIMEOUT);
-            return;
+            return false;
         }
     }
+    return true;
 }
+// Drain wait for this thread's own asynchronous operations before the CTA
+// exits: bounded, and not cut short by the abort flag.
+__device__ __forceinline__ void drain_wait(uint64_t *b, uint32_t par) {
+    const uint32_t a = su32(b);
+    const long long t0 = clock64();
+    while (!mbar_try(a, par) && clock64() - t0 < kWaitLimit / 8) {
+    }
+}
+__device__ __forceinline__ bool aborted(const TileSmem &sm) { return *(volatile const int *)&sm.abort != 0; }
 __device__ __forceinline__ void mbar_arrive(uint64_t *b) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
 }
@@ -135,21 +149,30 @@ __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// AND of `ok` over the 128 epilogue threads (a barrier too): every epilogue
+// thread takes the same branch after a wait that may have been cut short.
+__device__ __forceinline__ bool epi_all(bool ok) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, 2, 128, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r) : "r"((uint32_t)ok) : "memory");
+    return r != 0;
+}
 
 struct UnitInfo {
     int slot, row0, ntok, r, n1, np, j0, j1;
     bool skip;
 };
 
-__device__ __forceinline__ UnitInfo unit_info(const TileArgs &a, int u, int P, int nj) {
+__device__ __forceinline__ UnitInfo unit_info(const TileArgs &a, int tile, int j0, int j1) {
     UnitInfo ui;
-    const int tile = u / P, part = u - tile * P;
     const int4 t = a.tiles[tile];
     ui.slot = t.x;
     ui.row0 = t.y;
     ui.ntok = t.z;
-    ui.j0 = (int)((long long)nj * part / P);
-    ui.j1 = (int)((long long)nj * (part + 1) / P);
+    ui.j0 = j0;
+    ui.j1 = j1;
     int r = a.ranks[ui.slot];
     bool bad = r <= 0 || r > LORA_MAX_RANK;
     const int np = bad ? 0 : (r + 15) >> 4;
@@ -165,6 +188,32 @@ __device__ __forceinline__ UnitInfo unit_info(const TileArgs &a, int u, int P, i
     return ui;
 }
 
+// Every CTA takes an equal contiguous share of the (tile, n-tile) items in
+// tile-major order and walks it as units of one tile each; a CTA whose share
+// starts or ends inside a tile recomputes that tile's (small) shrink.
+struct UnitIter {
+    long long it, hi;
+    int nj;
+};
+
+__device__ __forceinline__ UnitIter unit_range(int n_tiles, int nj) {
+    UnitIter u;
+    const long long total = (long long)n_tiles * nj;
+    u.it = total * blockIdx.x / gridDim.x;
+    u.hi = total * (blockIdx.x + 1) / gridDim.x;
+    u.nj = nj;
+    return u;
+}
+
+__device__ __forceinline__ bool next_unit(const TileArgs &a, UnitIter &u, UnitInfo &ui) {
+    if (u.it >= u.hi) return false;
+    const int tile = (int)(u.it / u.nj), j0 = (int)(u.it % u.nj);
+    const int j1 = (int)min((long long)u.nj, j0 + (u.hi - u.it));
+    ui = unit_info(a, tile, j0, j1);
+    u.it += j1 - j0;
+    return true;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmA,
              const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmY, TileArgs a) {
@@ -172,9 +221,15 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
     TileSmem &sm = *reinterpret_cast<TileSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+    // The kernels before this one on the stream produce the plan.  A batch
+    // without long runs has no tiles: leave before touching tensor memory.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int n_tiles = a.hdr->n_tiles;
+    if (n_tiles <= 0) return;   // uniform over the grid
+
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], 1); }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kBuf; ++b) {
             mbar_init(&sm.bfull[b], 1); mbar_init(&sm.bempty[b], 1);
             mbar_init(&sm.yfull[b], 1); mbar_init(&sm.yempty[b], 1);
             mbar_init(&sm.accfull[b], 1); mbar_init(&sm.accempty[b], 128);
@@ -183,6 +238,7 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
         mbar_init(&sm.d1_empty, 128);
         mbar_init(&sm.v_ready, 128);
         mbar_init(&sm.v_empty, 1);
+        mbar_init(&sm.mma_drain, 1);
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -196,69 +252,73 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    // The kernels before this one on the stream produce the plan.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-
-    const int n_tiles = a.hdr->n_tiles;
     const int nj = (a.d_out + kNB - 1) / kNB;
     const int nkb = (a.d_in + kKB - 1) / kKB;
-    int P = n_tiles > 0 ? (int)((gridDim.x + n_tiles - 1) / n_tiles) : 1;
-    P = P < 1 ? 1 : (P > nj ? nj : P);
-    const int n_units = n_tiles * P;
 
     if (warp == 0 && lane == 0) {
         // ---------------- shrink operand producer ----------------
         int it = 0;
-        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-            const UnitInfo ui = unit_info(a, u, P, nj);
+        UnitIter ur = unit_range(n_tiles, nj);
+        UnitInfo ui;
+        while (next_unit(a, ur, ui) && !aborted(sm)) {
             if (ui.skip) continue;
             int pg[4];
             for (int p = 0; p < 4; ++p) pg[p] = p < ui.np ? a.pt[ui.slot * 8 + p] : 0;
             for (int kb = 0; kb < nkb; ++kb, ++it) {
                 const int s = it % kStages;
-                mbar_wait(&sm.empty[s], ((it / kStages) & 1) ^ 1, sm, a.err);
+                if (!mbar_wait(&sm.empty[s], ((it / kStages) & 1) ^ 1, sm, a.err)) break;
                 mbar_expect_tx(&sm.full[s], (uint32_t)(kM * kKB * 2 + ui.np * 16 * kKB * 2));
                 tma_load(sm.xs[s], &tmX, kb * kKB, ui.row0, &sm.full[s]);
                 for (int p = 0; p < ui.np; ++p)
                     tma_load(&sm.as[s][p * 16 * kKB], &tmA, kb * kKB, pg[p] * LORA_PAGE_ROWS, &sm.full[s]);
             }
         }
+        // the loads this thread armed last on each stage have landed before exit
+        for (int i = (it > kStages ? it - kStages : 0); i < it; ++i) drain_wait(&sm.full[i % kStages], (i / kStages) & 1);
     } else if (warp == 1 && lane == 0) {
         // ---------------- expand operand producer ----------------
         int it = 0;
-        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-            const UnitInfo ui = unit_info(a, u, P, nj);
+        UnitIter ur = unit_range(n_tiles, nj);
+        UnitInfo ui;
+        while (next_unit(a, ur, ui) && !aborted(sm)) {
             if (ui.skip) continue;
             int pg[4];
             for (int p = 0; p < 4; ++p) pg[p] = p < ui.np ? a.pt[ui.slot * 8 + 4 + p] : 0;
             for (int j = ui.j0; j < ui.j1; ++j, ++it) {
-                const int b = it & 1;
-                const uint32_t par = ((it >> 1) & 1) ^ 1;
-                mbar_wait(&sm.bempty[b], par, sm, a.err);
+                const int b = it % kBuf;
+                const uint32_t par = ((it / kBuf) & 1) ^ 1;
+                if (!mbar_wait(&sm.bempty[b], par, sm, a.err)) break;
+                if (!mbar_wait(&sm.yempty[b], par, sm, a.err)) break;
                 mbar_expect_tx(&sm.bfull[b], (uint32_t)(ui.np * 16 * kNB * 2));
                 for (int p = 0; p < ui.np; ++p)
                     tma_load(&sm.bs[b][p * 16 * kNB], &tmB, j * kNB, pg[p] * LORA_PAGE_ROWS, &sm.bfull[b]);
-                mbar_wait(&sm.yempty[b], par, sm, a.err);
                 mbar_expect_tx(&sm.yfull[b], (uint32_t)(kM * kNB * 4));
                 tma_load(&sm.ys[b][0], &tmY, j * kNB, ui.row0, &sm.yfull[b]);
                 tma_load(&sm.ys[b][kM * 32], &tmY, j * kNB + 32, ui.row0, &sm.yfull[b]);
             }
         }
+        for (int i = (it > kBuf ? it - kBuf : 0); i < it; ++i) {
+            drain_wait(&sm.bfull[i % kBuf], (i / kBuf) & 1);
+            drain_wait(&sm.yfull[i % kBuf], (i / kBuf) & 1);
+        }
     } else if (warp == 2 && lane == 0) {
         // ---------------- MMA issuer ----------------
         int it = 0, ite = 0, itt = 0;
+        bool issued = false;
         const uint32_t idesc2 = idesc_bf16(kM, kNB, 0, 1);
-        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-            const UnitInfo ui = unit_info(a, u, P, nj);
+        UnitIter ur = unit_range(n_tiles, nj);
+        UnitInfo ui;
+        while (next_unit(a, ur, ui) && !aborted(sm)) {
             if (ui.skip) continue;
             const uint32_t idesc1 = idesc_bf16(kM, ui.n1, 0, 0);
             // shrink: D1 = X A over all K blocks
-            mbar_wait(&sm.d1_empty, (itt & 1) ^ 1, sm, a.err);
+            if (!mbar_wait(&sm.d1_empty, (itt & 1) ^ 1, sm, a.err)) break;
             tc_fence_after();
             for (int kb = 0; kb < nkb; ++kb, ++it) {
                 const int s = it % kStages;
-                mbar_wait(&sm.full[s], (it / kStages) & 1, sm, a.err);
+                if (!mbar_wait(&sm.full[s], (it / kStages) & 1, sm, a.err)) break;
                 tc_fence_after();
+                issued = true;
                 const uint64_t da = sdesc(sm.xs[s], 16, 1024);
                 const uint64_t db = sdesc(sm.as[s], 16, 1024);
 #pragma unroll
@@ -266,16 +326,17 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
                     mma_bf16(tmem, da + (uint64_t)(k * 2), db + (uint64_t)(k * 2), idesc1, (kb | k) != 0);
                 mma_commit(&sm.empty[s]);
             }
+            if (aborted(sm)) break;
             mma_commit(&sm.shrink_done);
-            // expand: one 64-column n-tile at a time into a double-buffered accumulator
-            mbar_wait(&sm.v_ready, itt & 1, sm, a.err);
+            // expand: one 64-column n-tile at a time into a buffered accumulator
+            if (!mbar_wait(&sm.v_ready, itt & 1, sm, a.err)) break;
             tc_fence_after();
             const uint64_t dv = sdesc(sm.vs, 16, 1024);
             for (int j = ui.j0; j < ui.j1; ++j, ++ite) {
-                const int b = ite & 1;
-                const uint32_t par = (ite >> 1) & 1;
-                mbar_wait(&sm.accempty[b], par ^ 1, sm, a.err);
-                mbar_wait(&sm.bfull[b], par, sm, a.err);
+                const int b = ite % kBuf;
+                const uint32_t par = (ite / kBuf) & 1;
+                if (!mbar_wait(&sm.accempty[b], par ^ 1, sm, a.err)) break;
+                if (!mbar_wait(&sm.bfull[b], par, sm, a.err)) break;
                 tc_fence_after();
                 const uint64_t dbb = sdesc(sm.bs[b], (uint32_t)(ui.n1 * 128), 1024);
                 for (int k = 0; k < ui.np; ++k)
@@ -284,8 +345,14 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
                 mma_commit(&sm.bempty[b]);
                 mma_commit(&sm.accfull[b]);
             }
+            if (aborted(sm)) break;
             mma_commit(&sm.v_empty);
             ++itt;
+        }
+        // every MMA this thread issued has completed before tensor memory is freed
+        if (issued) {
+            mma_commit(&sm.mma_drain);
+            drain_wait(&sm.mma_drain, 0);
         }
     } else if (warp >= 4) {
         // ---------------- epilogue ----------------
@@ -293,13 +360,16 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
         const int m = q * 32 + lane;         // tile row = accumulator lane
         const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
         const bool leader = (warp == 4 && lane == 0);
+        int pending = -1;   // buffer whose TMA store may still be reading it
         int ite = 0, itt = 0;
-        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-            const UnitInfo ui = unit_info(a, u, P, nj);
+        UnitIter ur = unit_range(n_tiles, nj);
+        UnitInfo ui;
+        while (next_unit(a, ur, ui)) {
+            if (!epi_all(!aborted(sm))) break;   // same decision in all 128 epilogue threads
             if (ui.skip) continue;
             const float sc = a.scales[ui.slot];
             // v = D1 row m, rounded to bf16 into the swizzled V tile
-            mbar_wait(&sm.shrink_done, itt & 1, sm, a.err);
+            if (!epi_all(mbar_wait(&sm.shrink_done, itt & 1, sm, a.err))) break;
             tc_fence_after();
             float d1[64];
 #pragma unroll
@@ -308,7 +378,7 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&sm.d1_empty);
-            mbar_wait(&sm.v_empty, (itt & 1) ^ 1, sm, a.err);
+            if (!epi_all(mbar_wait(&sm.v_empty, (itt & 1) ^ 1, sm, a.err))) break;
             unsigned char *vrow = reinterpret_cast<unsigned char *>(sm.vs) + m * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -329,10 +399,11 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
             mbar_arrive(&sm.v_ready);
             // n-tiles
             for (int j = ui.j0; j < ui.j1; ++j, ++ite) {
-                const int b = ite & 1;
-                const uint32_t par = (ite >> 1) & 1;
-                mbar_wait(&sm.accfull[b], par, sm, a.err);
-                mbar_wait(&sm.yfull[b], par, sm, a.err);
+                const int b = ite % kBuf;
+                const uint32_t par = (ite / kBuf) & 1;
+                bool ok = mbar_wait(&sm.accfull[b], par, sm, a.err);
+                ok = mbar_wait(&sm.yfull[b], par, sm, a.err) && ok;
+                if (!epi_all(ok)) break;
                 tc_fence_after();
                 float acc[64];
 #pragma unroll
@@ -366,14 +437,29 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
                         tma_store(&tmY, j * kNB, ui.row0, &sm.ys[b][0]);
                         tma_store(&tmY, j * kNB + 32, ui.row0, &sm.ys[b][kM * 32]);
                         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-                        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                        // the previous store has finished reading its buffer once at
+                        // most one group (this one) is still reading
+                        asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                        if (pending >= 0) mbar_arrive(&sm.yempty[pending]);
+                        pending = b;
+                    } else {
+                        // a buffer whose store is still pending would otherwise wait for
+                        // the next full tile, which may never come on this CTA
+                        if (pending >= 0) {
+                            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                            mbar_arrive(&sm.yempty[pending]);
+                            pending = -1;
+                        }
+                        mbar_arrive(&sm.yempty[b]);
                     }
-                    mbar_arrive(&sm.yempty[b]);
                 }
             }
             ++itt;
         }
-        if (leader) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        if (leader) {
+            asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+            if (pending >= 0) mbar_arrive(&sm.yempty[pending]);
+        }
     }
 
     tc_fence_before();
@@ -385,40 +471,9 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-int make_map(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, uint64_t cols, uint64_t rows,
-             uint32_t box_cols, uint32_t box_rows) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return LORA_ERR_CUDA;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * (uint64_t)esize};
-    cuuint32_t box[2] = {box_cols, box_rows};
-    cuuint32_t es[2] = {1, 1};
-    CUresult r = enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? LORA_OK : LORA_ERR_CUDA;
-}
-
 }  // namespace
 
-bool tiles_supported() { return encode_fn() != nullptr; }
+bool tiles_supported() { return tma_supported(); }
 
 int launch_tiles(const TileArgs &a, cudaStream_t st, bool pdl) {
     static int num_sms[64] = {};
@@ -433,22 +488,23 @@ int launch_tiles(const TileArgs &a, cudaStream_t st, bool pdl) {
         if (int rc = cuda_check(cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev))) return rc;
         num_sms[dev] = n > 0 ? n : 1;
     }
-    CUtensorMap mx, ma, mb, my;
-    if (make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.X, (uint64_t)a.d_in, (uint64_t)a.T, kKB, kM) ||
-        make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.pa->base, (uint64_t)a.d_in, (uint64_t)a.rowsA, kKB, 16) ||
-        make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.pb->base, (uint64_t)a.d_out, (uint64_t)a.rowsB, kNB, 16) ||
-        make_map(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.Y, (uint64_t)a.d_out, (uint64_t)a.T, 32, kM))
-        return LORA_ERR_CUDA;
-    // upper bound of units: every tile of every long segment times the d_out split
-    const int max_tiles = (a.T + kM - 1) / kM + (a.long_thresh > 0 ? a.T / a.long_thresh : 0);
-    int grid = num_sms[dev];
+    CUtensorMap mx, my, ma, mb;
+    if (int rc = make_tensor_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.X, (uint64_t)a.d_in, (uint64_t)a.T, kKB, kM, true))
+        return rc;
+    if (int rc = make_tensor_map(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.Y, (uint64_t)a.d_out, (uint64_t)a.T, 32, kM, true))
+        return rc;
+    if (int rc = pool_tensor_map(const_cast<lora_pool_s *>(a.pa), kPoolMapTile, &ma)) return rc;
+    if (int rc = pool_tensor_map(const_cast<lora_pool_s *>(a.pb), kPoolMapTile, &mb)) return rc;
+    // one CTA per SM (never more than there can be (tile, n-tile) items)
+    const long long max_tiles = (a.T + kM - 1) / kM + (a.long_thresh > 0 ? a.T / a.long_thresh : 0);
+    long long grid = num_sms[dev];
     if (grid > max_tiles * ((a.d_out + kNB - 1) / kNB)) grid = max_tiles * ((a.d_out + kNB - 1) / kNB);
     if (grid < 1) grid = 1;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.gridDim = dim3(grid);
+    cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;

@@ -212,7 +212,7 @@ int lora_apply_planned(const uint16_t *X, float *Y, int T, int d_in, int d_out, 
  * or from different host threads without ordering - race and give undefined
  * results: order them on one stream. */
 #define LORA_NOALLOC_MAX_TOKENS    32768
-#define LORA_NOALLOC_SCRATCH_BYTES 1310720   /* 1.25 MiB */
+#define LORA_NOALLOC_SCRATCH_BYTES 2097152   /* 2 MiB */
 int lora_apply_noalloc(const uint16_t *X, float *Y, int T, int d_in, int d_out, const int32_t *ids,
                        int num_slots, const int32_t *ranks, const float *scales,
                        const int32_t *page_table, lora_pool_t pa, lora_pool_t pb,

@@ -63,3 +63,41 @@ def assert_parity(Y_dev: np.ndarray, Y_ref: np.ndarray, Y_base: np.ndarray, delt
     if scale > 0:
         worst = np.abs(d_dev - d_ref).max()
         assert worst <= delta_rel * scale, f"delta error {worst:.3e} > {delta_rel:g} * {scale:.3e}"
+
+
+def expected_work(ids, ranks, long_thresh: int, job_tokens: int):
+    """(n_jobs, n_tiles) the plan should produce: maximal runs of one valid slot with at
+    least long_thresh tokens become ceil(len/128) tiles; the other valid tokens of
+    each slot are split into ceil(count/job_tokens) gather jobs."""
+    ids = np.asarray(ids)
+    S = len(ranks)
+    valid = np.array([(0 <= i < S) and ranks[i] > 0 for i in ids], dtype=bool)
+    T = len(ids)
+    in_long = np.zeros(T, dtype=bool)
+    n_tiles = 0
+    if long_thresh > 0 and T >= long_thresh:
+        t = 0
+        while t < T:
+            if not valid[t]:
+                t += 1
+                continue
+            e = t
+            while e + 1 < T and valid[e + 1] and ids[e + 1] == ids[t]:
+                e += 1
+            L = e - t + 1
+            if L >= long_thresh:
+                in_long[t:e + 1] = True
+                n_tiles += (L + 127) // 128
+            t = e + 1
+    n_jobs = 0
+    short = ids[valid & ~in_long]
+    for k, c in zip(*np.unique(short, return_counts=True)):
+        n_jobs += (int(c) + job_tokens - 1) // job_tokens
+    return n_jobs, n_tiles
+
+
+def plan_counts(ws):
+    """(n_valid, n_seg, n_jobs, n_tiles) from the head of a workspace the library
+    filled (the plan header is the workspace's first 16 bytes)."""
+    h = ws[:16].cpu().numpy().view(np.int32)
+    return tuple(int(x) for x in h[:4])

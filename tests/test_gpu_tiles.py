@@ -31,13 +31,19 @@ def _restore_options(H):
         H.lora_set_option(k, v)
 
 
-def _apply(wl):
+def _apply(wl, H=None):
+    """Run lora_apply; when H is given also check the plan's job / tile counts."""
     import torch
     layer = U.make_layer(wl)
     X, Y, ids = U.dev_inputs(wl)
     layer.err.zero_()
     layer.apply(X, Y, ids)
     torch.cuda.synchronize()
+    if H is not None:
+        lt = H.lora_get_option(H.OPT_LONG_SEGMENT)
+        jt = H.lora_get_option(H.OPT_DECODE_JOB_TOKENS)
+        n_valid, n_seg, n_jobs, n_tiles = U.plan_counts(layer.ws)
+        assert (n_jobs, n_tiles) == U.expected_work(wl.ids, wl.ranks(), lt, jt)
     return Y.cpu().numpy(), int(layer.err.item())
 
 
@@ -48,11 +54,12 @@ def _apply(wl):
     (3, [17, 250, 5, 64, 400], 200, 328),
     (4, [513, 7, 1000], 1032, 520),
     (5, [90, 33, 256, 256, 12], 4096, 4096),
+    (6, [5000], 256, 512),
 ])
 def test_tile_path_segments(H, thresh, seed, lens, d_in, d_out):
     H.lora_set_option(H.OPT_LONG_SEGMENT, thresh)
     wl = W.segments(seed, lens, d_in, d_out, S=max(8, len(lens)), ranks=(1, 4, 8, 15, 16, 17, 33, 48, 64))
-    Y, err = _apply(wl)
+    Y, err = _apply(wl, H)
     ref, rerr = U.oracle_full(wl)
     assert err == rerr == 0
     U.assert_parity(Y, ref, wl.Y_base, delta_rel=U.DELTA_REL_TENSOR)
@@ -67,7 +74,7 @@ def test_tile_path_with_shared_slots_and_none(H):
     ids = wl.ids.copy()
     ids[[0, 45, 250, 600]] = -1
     wl.ids[:] = ids
-    Y, err = _apply(wl)
+    Y, err = _apply(wl, H)
     ref, rerr = U.oracle_full(wl)
     assert err == rerr == 0
     U.assert_parity(Y, ref, wl.Y_base, delta_rel=U.DELTA_REL_TENSOR)
@@ -79,9 +86,9 @@ def test_tile_and_gather_paths_agree_with_oracle(H):
     wl = W.segments(7, [300, 200, 100], 1024, 1024, S=4)
     ref, _ = U.oracle_full(wl)
     H.lora_set_option(H.OPT_LONG_SEGMENT, 16)
-    Yt, e1 = _apply(wl)
+    Yt, e1 = _apply(wl, H)
     H.lora_set_option(H.OPT_LONG_SEGMENT, 0)
-    Yg, e2 = _apply(wl)
+    Yg, e2 = _apply(wl, H)
     assert e1 == e2 == 0
     U.assert_parity(Yt, ref, wl.Y_base, delta_rel=U.DELTA_REL_TENSOR)
     U.assert_parity(Yg, ref, wl.Y_base)
@@ -91,7 +98,8 @@ def test_prefill_config_tile_path(H):
     """The prefill workload (16 sequences of 128-2048 tokens, 6 adapters) through the
     default threshold, i.e. on the tensor-core tiles."""
     wl = W.prefill()
-    Y, err = _apply(wl)
+    Y, err = _apply(wl, H)
+    assert U.expected_work(wl.ids, wl.ranks(), 16, 4)[1] >= 130   # the tiles really run
     ref, rerr = U.oracle_full(wl)
     assert err == rerr == 0
     U.assert_parity(Y, ref, wl.Y_base, delta_rel=U.DELTA_REL_TENSOR)
