@@ -11,8 +11,8 @@
 //
 // Work unit = one gather job (an adapter slot and up to 4 of its tokens, from
 // the plan kernel) times one part e of an E-way split of d_out.  A cluster of
-// kCS CTAs runs one unit at a time and loops over the units (persistent grid
-// sized from the occupancy of the cluster shape).  Per CTA:
+// kCS CTAs (one per SM) runs one unit at a time and loops over the units
+// (persistent grid sized from the occupancy of the cluster shape).  Per CTA:
 //   * a producer warp streams the adapter's pages into a ring of shared-memory
 //     stages with 2D TMA loads, one page (16 rank rows) by 256 columns per
 //     instruction: first the CTA's 1/kCS slice of d_in (rows of A^T), then its
@@ -40,12 +40,12 @@
 namespace lora {
 namespace {
 
-constexpr int kCS = 8;                       // CTAs per cluster
+constexpr int kCS = 4;                       // CTAs per cluster
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;    // + one producer warp
 constexpr int kNT = 4;                       // max tokens per job
-constexpr int kStages = 2;
+constexpr int kStages = 4;
 constexpr int kBoxCols = 256;                // TMA box: 16 rows x 256 columns of bf16 = 8 KB
 constexpr int kBoxBytes = LORA_PAGE_ROWS * kBoxCols * 2;
 constexpr int kStageBoxes = 4;               // a stage holds 4 boxes = 32 KB
@@ -236,8 +236,66 @@ __device__ __forceinline__ UnitGeom unit_geom(const GatherArgs &a, int np, int e
     return g;
 }
 
+__device__ __forceinline__ int4 ld_v4_now(const int4 *p) {
+    int4 v;
+    asm volatile("ld.global.v4.s32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ int ld_s32_now(const int *p) {
+    int v;
+    asm volatile("ld.global.s32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+// 8-term dot product summed as a tree (a fixed order, shorter dependency chains).
+__device__ __forceinline__ float dot8(const float a[8], const float x[8]) {
+    const float p0 = fmaf(a[1], x[1], a[0] * x[0]);
+    const float p1 = fmaf(a[3], x[3], a[2] * x[2]);
+    const float p2 = fmaf(a[5], x[5], a[4] * x[4]);
+    const float p3 = fmaf(a[7], x[7], a[6] * x[6]);
+    return (p0 + p1) + (p2 + p3);
+}
+
+// One staged chunk of the shrink: this warp's rank rows k = warp + 8 j for
+// j < RPW, lanes over the chunk's 8-column groups.
+template <int RPW>
+__device__ __forceinline__ void shrink_chunk(const unsigned char *st, const uint4 (*xs)[kStageBoxes * kBoxCols / 8],
+                                             int ng, int nb, int warp, int lane, int r, int n, float (&acc)[8][kNT]) {
+    // tokens in groups of TG: all four at once for few rank rows per warp, two
+    // at a time for 8 rows (the rows' values are re-read from shared memory)
+    constexpr int TG = RPW >= 8 ? 2 : kNT;
+    for (int q = lane; q < ng; q += 32) {
+        const int b = (q * 8) / kBoxCols, cb = q * 8 - b * kBoxCols;
+#pragma unroll
+        for (int t0 = 0; t0 < kNT; t0 += TG) {
+            if (t0 >= n) break;
+            float xf[TG][8];
+#pragma unroll
+            for (int t = 0; t < TG; ++t) {
+                if (t0 + t < n) bf16x8(xs[t0 + t][q], xf[t]);
+                else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) xf[t][i] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < RPW; ++j) {
+                const int k = warp + j * kConsumerWarps;
+                if (k < r) {
+                    float af[8];
+                    bf16x8(*reinterpret_cast<const uint4 *>(st + (size_t)((k >> 4) * nb + b) * kBoxBytes +
+                                                            (k & 15) * (kBoxCols * 2) + cb * 2),
+                           af);
+#pragma unroll
+                    for (int t = 0; t < TG; ++t) acc[j][t0 + t] += dot8(af, xf[t]);
+                }
+            }
+        }
+    }
+}
+
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
 gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GatherArgs a,
               int e_max) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -252,24 +310,12 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], kConsumerWarps);
         }
-        mbar_init(&sm.xbar[0], kCS);
-        mbar_init(&sm.xbar[1], kCS);
+        // every consumer warp of every CTA of the cluster arrives once per unit
+        mbar_init(&sm.xbar[0], kCS * kConsumerWarps);
+        mbar_init(&sm.xbar[1], kCS * kConsumerWarps);
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    // Page tables, ranks and scales are never written by this library's kernels,
-    // and any caller write to them precedes this launch in stream order, so they
-    // are staged before waiting for the plan.
-    const bool staged = a.S <= kTableSlots;
-    if (staged) {
-        for (int i = threadIdx.x; i < a.S; i += kThreads) {
-            sm.pt[2 * i] = reinterpret_cast<const int4 *>(a.pt)[2 * i];
-            sm.pt[2 * i + 1] = reinterpret_cast<const int4 *>(a.pt)[2 * i + 1];
-            sm.ranks[i] = a.ranks[i];
-            sm.scales[i] = (MODE == kShrink) ? 0.f : a.scales[i];
-        }
-    }
-    __syncthreads();
     // Announce this CTA's barriers to its peers; the matching wait comes just
     // before the first push into a peer.
     asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
@@ -281,12 +327,24 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
 
-    // The first job record is read together with the job count (a guess that
-    // holds whenever there are at least half as many jobs as clusters).
+    // Issue the first job record (a guess that holds whenever there are at
+    // least half as many jobs as clusters), the job count and the slot tables
+    // together, so their latencies overlap.
     const int spec = cluster_id < a.T ? cluster_id : a.T - 1;
-    const int4 spec_job = a.jobs[2 * spec];
-    const int4 spec_tok = a.jobs[2 * spec + 1];
-    const int n_jobs = a.hdr->n_jobs;
+    const int4 spec_job = ld_v4_now(a.jobs + 2 * spec);
+    const int4 spec_tok = ld_v4_now(a.jobs + 2 * spec + 1);
+    const int n_jobs = ld_s32_now(&a.hdr->n_jobs);
+    // Small page tables, ranks and scales are staged in shared memory.
+    const bool staged = a.S <= kTableSlots;
+    if (staged) {
+        for (int i = threadIdx.x; i < a.S; i += kThreads) {
+            sm.pt[2 * i] = reinterpret_cast<const int4 *>(a.pt)[2 * i];
+            sm.pt[2 * i + 1] = reinterpret_cast<const int4 *>(a.pt)[2 * i + 1];
+            sm.ranks[i] = a.ranks[i];
+            sm.scales[i] = (MODE == kShrink) ? 0.f : a.scales[i];
+        }
+    }
+    __syncthreads();
     if (n_jobs <= 0) return;   // uniform over the grid; no peer traffic has happened
     int E = 1;
     if (MODE != kShrink) {
@@ -349,6 +407,17 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         const UnitGeom g = unit_geom<MODE>(a, m.np, e, E, crank);
         const int buf = iter & 1;
         const int cw = g.nb * kBoxCols;
+        // old Y of this thread's columns of the first expand chunk, fetched early
+        float yv[kStageBoxes][kNT];
+        auto load_y = [&](int c0, int wcols) {
+#pragma unroll
+            for (int i = 0; i < kStageBoxes; ++i) {
+                const int col = threadIdx.x + i * kConsumers;
+#pragma unroll
+                for (int t = 0; t < kNT; ++t)
+                    yv[i][t] = (t < n && col < wcols) ? a.Y[(size_t)tok[t] * a.d_out + c0 + col] : 0.f;
+            }
+        };
 
         if (MODE != kExpand) {
             // ---- shrink: partial sums over this CTA's d_in slice ----
@@ -357,6 +426,7 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             for (int j = 0; j < 8; ++j)
 #pragma unroll
                 for (int t = 0; t < kNT; ++t) acc[j][t] = 0.f;
+            const int rpw = (r + kConsumerWarps - 1) / kConsumerWarps;
             for (int c = 0; c < g.n_shrink; ++c, ++chunk) {
                 const int s = chunk % kStages;
                 const int c0 = g.in0 + c * cw;
@@ -371,34 +441,20 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 mbar_wait<false>(&sm.full[s], (chunk / kStages) & 1, sm, a.err);
                 consumer_sync();
                 const unsigned char *st = sm.stage[s];
-                for (int q = lane; q < ng; q += 32) {
-                    const int b = (q * 8) / kBoxCols, cb = q * 8 - b * kBoxCols;
-#pragma unroll
-                    for (int t = 0; t < kNT; ++t) {
-                        if (t < n) {
-                            float xf[8];
-                            bf16x8(xs[t][q], xf);
-#pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                const int k = warp + j * kConsumerWarps;
-                                if (k < r) {
-                                    float af[8];
-                                    bf16x8(*reinterpret_cast<const uint4 *>(st + (size_t)((k >> 4) * g.nb + b) * kBoxBytes +
-                                                                            (k & 15) * (kBoxCols * 2) + cb * 2),
-                                           af);
-                                    float sum = acc[j][t];
-#pragma unroll
-                                    for (int i = 0; i < 8; ++i) sum = fmaf(af[i], xf[i], sum);
-                                    acc[j][t] = sum;
-                                }
-                            }
-                        }
-                    }
-                }
+                if (rpw <= 1) shrink_chunk<1>(st, xs, ng, g.nb, warp, lane, r, n, acc);
+                else if (rpw <= 2) shrink_chunk<2>(st, xs, ng, g.nb, warp, lane, r, n, acc);
+                else if (rpw <= 4) shrink_chunk<4>(st, xs, ng, g.nb, warp, lane, r, n, acc);
+                else shrink_chunk<8>(st, xs, ng, g.nb, warp, lane, r, n, acc);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.empty[s]);
             }
-            // reduce over lanes; lane 0 keeps the warp's sums
+            if (MODE == kApply && g.n_expand > 0) load_y(g.out0, min(cw, g.out1 - g.out0));
+            if (!joined) {
+                asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+                joined = true;
+            }
+            // reduce over lanes (every lane gets the sum), then lane q stores the
+            // value into peer q's slot `crank` and arrives on peer q's barrier
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int k = warp + j * kConsumerWarps;
@@ -409,34 +465,19 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                             float x = acc[j][t];
 #pragma unroll
                             for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-                            if (lane == 0) sm.P[buf][crank][t * r + k] = x;   // own slot, local copy
+                            if (lane < kCS)
+                                asm volatile("st.shared::cluster.f32 [%0], %1;"
+                                             ::"r"(map_peer(smem_u32(&sm.P[buf][crank][t * r + k]), (uint32_t)lane)),
+                                             "f"(x) : "memory");
                         }
                     }
                 }
             }
-            if (!joined) {
-                asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-                joined = true;
-            }
-            consumer_sync();
-            // push the partial vector [t * r + k] into every peer's slot `crank`
-            const int nv = n * r;
-            const int nv4 = (nv + 3) / 4;
-            for (int idx = threadIdx.x; idx < kCS * nv4; idx += kConsumers) {
-                const int q = idx / nv4;
-                const int v4 = idx - q * nv4;
-                if (q == crank) continue;
-                const float *srcp = &sm.P[buf][crank][v4 * 4];
-                const float4 val = make_float4(srcp[0], v4 * 4 + 1 < nv ? srcp[1] : 0.f,
-                                               v4 * 4 + 2 < nv ? srcp[2] : 0.f, v4 * 4 + 3 < nv ? srcp[3] : 0.f);
-                st_peer_v4(map_peer(smem_u32(&sm.P[buf][crank][v4 * 4]), (uint32_t)q), val);
-            }
-            consumer_sync();
-            if (threadIdx.x == 0) {
-                for (int q = 0; q < kCS; ++q) arrive_peer_release(map_peer(smem_u32(&sm.xbar[buf]), (uint32_t)q));
-            }
+            __syncwarp();
+            if (lane < kCS) arrive_peer_release(map_peer(smem_u32(&sm.xbar[buf]), (uint32_t)lane));
             mbar_wait<true>(&sm.xbar[buf], (uint32_t)((iter >> 1) & 1), sm, a.err);
             // v[k][t] = sum over peers in rank order
+            const int nv = n * r;
             for (int idx = threadIdx.x; idx < nv; idx += kConsumers) {
                 const int t = idx / r, k = idx - t * r;
                 float sum = 0.f;
@@ -460,6 +501,7 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 const int t = idx / r, k = idx - t * r;
                 reinterpret_cast<float *>(&sm.v[k])[t] = a.V[(size_t)tok[t] * LORA_MAX_RANK + k];
             }
+            if (g.n_expand > 0) load_y(g.out0, min(cw, g.out1 - g.out0));
             consumer_sync();
         }
 
@@ -469,15 +511,7 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             const int s = chunk % kStages;
             const int c0 = g.out0 + c * cw;
             const int wcols = min(cw, g.out1 - c0);
-            // old Y of this thread's columns, loaded before the weights arrive
-            float yv[kStageBoxes][kNT];
-#pragma unroll
-            for (int i = 0; i < kStageBoxes; ++i) {
-                const int col = threadIdx.x + i * kConsumers;
-#pragma unroll
-                for (int t = 0; t < kNT; ++t)
-                    yv[i][t] = (t < n && col < wcols) ? a.Y[(size_t)tok[t] * a.d_out + c0 + col] : 0.f;
-            }
+            if (c > 0) load_y(c0, wcols);   // the first chunk's Y was fetched before the exchange
             mbar_wait<false>(&sm.full[s], (chunk / kStages) & 1, sm, a.err);
             const unsigned char *st = sm.stage[s];
 #pragma unroll
