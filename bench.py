@@ -262,6 +262,35 @@ class Ring:
         return n
 
 
+PROFILE_FOR = {
+    # workload -> (profile summary, kernel source it was captured from)
+    "decode_q_proj_7b": ("profiles/gather_kernel_decode_q_proj_7b.md",
+                         "heterogeneous_adapter_batching_b200/csrc/lora_gather.cu"),
+    "prefill": ("profiles/tiles_kernel_prefill.md", "heterogeneous_adapter_batching_b200/csrc/lora_tiles.cu"),
+}
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary,
+    or None when there is none or the kernel source changed since the capture."""
+    import hashlib
+    if workload not in PROFILE_FOR:
+        return None
+    prof, src = (os.path.join(ROOT, x) for x in PROFILE_FOR[workload])
+    try:
+        fields = {}
+        for line in open(prof):
+            if ":" in line and not line.startswith(("#", "|", " ")):
+                k, v = line.split(":", 1)
+                fields[k.strip()] = v.strip()
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        if fields.get("source_sha256") != sha:
+            return None
+        return int(fields["traffic_bytes_per_launch"])
+    except Exception:
+        return None
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -369,7 +398,7 @@ def run_gpu(args):
     peak, peak_kind = measured_peaks()
     kname = "gather_kernel<apply>" if n_tiles == 0 else "gather_kernel<apply> + tiles_kernel"
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-            "traffic": None, "peak_source": peak_kind, "kernel": kname,
+            "traffic": profiled_traffic(args.workload), "peak_source": peak_kind, "kernel": kname,
             "kernel_us": per_launch_ms * 1000.0, "algorithmic_bytes_per_launch": alg,
             "launches_per_layer": apply_launches // n_layers}
 

@@ -9,7 +9,7 @@
 namespace lora {
 
 namespace {
-std::atomic<int> g_long_segment{16};
+std::atomic<int> g_long_segment{128};
 std::atomic<int> g_job_tokens{4};
 thread_local int t_launches = 0;
 thread_local const char *t_last_cuda_error = "no error";

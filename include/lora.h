@@ -222,7 +222,8 @@ int lora_apply_noalloc(const uint16_t *X, float *Y, int T, int d_in, int d_out, 
 /* Options and diagnostics (process-wide)                                   */
 /* ------------------------------------------------------------------------ */
 
-#define LORA_OPT_LONG_SEGMENT   1   /* segments with >= this many tokens use the tensor-core path (default 16; 0 = never) */
+#define LORA_OPT_LONG_SEGMENT   1   /* runs of >= this many consecutive tokens of one slot use the tensor-core path
+                                        (default 128, one full tile; 0 = never) */
 #define LORA_OPT_DECODE_JOB_TOKENS 2 /* max tokens per gather job (1..4, default 4) */
 
 int lora_set_option(int key, int value);

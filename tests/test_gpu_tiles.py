@@ -99,7 +99,7 @@ def test_prefill_config_tile_path(H):
     default threshold, i.e. on the tensor-core tiles."""
     wl = W.prefill()
     Y, err = _apply(wl, H)
-    assert U.expected_work(wl.ids, wl.ranks(), 16, 4)[1] >= 130   # the tiles really run
+    assert U.expected_work(wl.ids, wl.ranks(), H.lora_get_option(H.OPT_LONG_SEGMENT), 4)[1] >= 130  # tiles run
     ref, rerr = U.oracle_full(wl)
     assert err == rerr == 0
     U.assert_parity(Y, ref, wl.Y_base, delta_rel=U.DELTA_REL_TENSOR)
