@@ -10,7 +10,7 @@ namespace lora {
 
 namespace {
 std::atomic<int> g_long_segment{128};
-std::atomic<int> g_job_tokens{4};
+std::atomic<int> g_job_tokens{LORA_MAX_JOB_TOKENS};
 thread_local int t_launches = 0;
 thread_local const char *t_last_cuda_error = "no error";
 
@@ -96,7 +96,8 @@ using namespace lora;
 extern "C" {
 
 int lora_pool_create(void *dev_buf, size_t bytes, int width, int page_rows, lora_pool_t *out) {
-    if (!out || !dev_buf || width <= 0 || (width % 8) != 0 || page_rows != LORA_PAGE_ROWS) return LORA_ERR_INVALID_ARG;
+    if (!out || !dev_buf || width <= 0 || (width % 8) != 0 || width > (1 << 24) || page_rows != LORA_PAGE_ROWS)
+        return LORA_ERR_INVALID_ARG;
     if (!aligned(dev_buf, 256)) return LORA_ERR_INVALID_ARG;
     const size_t page_bytes = (size_t)page_rows * width * 2;
     const size_t np = bytes / page_bytes;
@@ -371,7 +372,7 @@ int lora_set_option(int key, int value) {
             g_long_segment.store(value);
             return LORA_OK;
         case LORA_OPT_DECODE_JOB_TOKENS:
-            if (value < 1 || value > 4) return LORA_ERR_INVALID_ARG;
+            if (value < 1 || value > LORA_MAX_JOB_TOKENS) return LORA_ERR_INVALID_ARG;
             g_job_tokens.store(value);
             return LORA_OK;
     }

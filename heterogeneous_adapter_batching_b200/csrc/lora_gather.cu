@@ -9,27 +9,31 @@
 // added to the base output.  Section "Unified Paging Architecture": the
 // weights are read straight out of the physical pages the page table names.
 //
-// Work unit = one gather job (an adapter slot and up to 4 of its tokens, from
+// Work unit = one gather job (an adapter slot and up to 16 of its tokens, from
 // the plan kernel) times one part e of an E-way split of d_out.  A cluster of
 // kCS CTAs (one per SM) runs one unit at a time and loops over the units
 // (persistent grid sized from the occupancy of the cluster shape).  Per CTA:
 //   * a producer warp streams the adapter's pages into a ring of shared-memory
-//     stages with 2D TMA loads, one page (16 rank rows) by 256 columns per
-//     instruction: first the CTA's 1/kCS slice of d_in (rows of A^T), then its
+//     stages with 2D TMA loads of 16 rank rows x 64 columns (128-byte
+//     swizzled): first the CTA's 1/kCS slice of d_in (rows of A^T), then its
 //     slice of d_out (rows of B).  It runs ahead into the next unit while the
 //     consumers finish the current one.  Only the pages the adapter has are
 //     read; a rank that is not a multiple of 16 reads the zeroed rows of its
 //     last page;
-//   * 8 consumer warps read the tokens' X and Y values straight from global
-//     memory (coalesced, issued before they wait for the weights), compute the
-//     shrink partial sums over the d_in slice (warps take rank rows, lanes take
-//     8-column groups, warp shuffles reduce the lanes) and push them into
-//     every peer CTA's shared memory (distributed shared memory stores, then a
-//     release arrive on the peer's mbarrier);
-//   * each CTA sums the kCS partials in rank order, so all CTAs hold the same
-//     fp32 v and the result is bit-reproducible, then expands its d_out slice:
-//     threads take columns, read B from the stage and store the new Y values
-//     with coalesced stores.
+//   * 15 consumer warps copy the tokens' X columns of each chunk into shared
+//     memory (cp.async, issued one chunk ahead) and run the shrink on the
+//     tensor cores with warp-level bf16 MMAs (m16n8k16, fp32 accumulate): a
+//     page's 16 rank rows are the M side, up to 8 tokens the N side, and each
+//     warp owns every 15th 16-column step of the slice.  The warps' partial
+//     sums are added in warp order, the CTAs exchange theirs through
+//     distributed shared memory after one hardware cluster barrier, and each
+//     CTA adds the kCS partials in rank order, so all CTAs hold the same fp32
+//     v and a token's result does not depend on the job it landed in;
+//   * v is split into a bf16 high part and a bf16 low part (v - high), and the
+//     expand runs as two MMAs per page (output columns on the M side, read
+//     with transposing ldmatrix), which keeps v to about 16 significant bits;
+//     each warp owns every 15th 16-column tile of the d_out slice and adds
+//     scale * (v B) to Y in place.
 // Small page tables (<= 256 slots) are staged in shared memory before the
 // kernel waits for the plan, so a unit's metadata costs one global read (the
 // job record).  Every wait is bounded; a wait that runs out sets
@@ -41,28 +45,51 @@ namespace lora {
 namespace {
 
 constexpr int kCS = 4;                       // CTAs per cluster
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 15;           // + 1 producer = 16 warps: 4 per SM sub-partition
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;    // + one producer warp
-constexpr int kNT = 4;                       // max tokens per job
+constexpr int kNTok = 8;                     // tokens per MMA (the N side)
+constexpr int kMaxNTiles = LORA_MAX_JOB_TOKENS / kNTok;
+constexpr int kMaxJobTokens = kMaxNTiles * kNTok;
+constexpr int kMaxPages = LORA_MAX_RANK / LORA_PAGE_ROWS;
 constexpr int kStages = 4;
-constexpr int kBoxCols = 256;                // TMA box: 16 rows x 256 columns of bf16 = 8 KB
+constexpr int kBoxCols = 64;                 // TMA box: 16 rows x 64 columns of bf16 = 2 KB, 128B swizzle
 constexpr int kBoxBytes = LORA_PAGE_ROWS * kBoxCols * 2;
-constexpr int kStageBoxes = 4;               // a stage holds 4 boxes = 32 KB
-constexpr int kTableSlots = 256;             // page tables up to this many slots live in shared memory
+constexpr int kStageBoxes = 16;              // a stage holds 16 boxes = 32 KB
+constexpr int kMaxChunkCols = kStageBoxes * kBoxCols;   // chunk width with a single page
+constexpr int kTableSlots = 128;             // page tables up to this many slots live in shared memory
 constexpr long long kWaitLimit = 2000000000LL;   // cycles (~1 s)
+constexpr int kMTW = (kMaxChunkCols / 16 + kConsumerWarps - 1) / kConsumerWarps;   // a warp's 16-column tiles per chunk
 
-struct __align__(128) GatherSmem {
-    unsigned char stage[kStages][kStageBoxes * kBoxBytes];   // box (page p, column block b) at (p * nb + b) * 8 KB
-    float P[2][kCS][kNT * LORA_MAX_RANK];     // partial sums pushed by each peer, [t * r + k]
-    float4 v[LORA_MAX_RANK];                  // reduced v: v[k] holds tokens 0..3
-    uint4 xs[2][kNT][kStageBoxes * kBoxCols / 8];   // the chunk's X columns per token (double-buffered)
-    int4 pt[kTableSlots * 2];                 // staged page-table rows (A pages, B pages)
+static_assert(kMaxJobTokens == LORA_MAX_JOB_TOKENS, "job size must be a whole number of MMA tiles");
+// After the shrink the X buffers hold the warps' partial sums (kRedBytes),
+// then this CTA's partial; after the exchange, v in bf16 (high and low parts).
+constexpr int kRedBytes = kConsumerWarps * kMaxPages * kMaxNTiles * 128 * 4;
+constexpr int kPartFloats = kMaxJobTokens * LORA_MAX_RANK;
+constexpr int kVBytes = kMaxJobTokens * LORA_MAX_RANK * 2;   // one bf16 part of v
+static_assert(kRedBytes + kPartFloats * 4 <= 2 * kMaxJobTokens * kMaxChunkCols * 2,
+              "the partial sums must fit in the X buffers");
+
+struct __align__(1024) GatherSmem {
+    // stage s, box (page p, column block b) at (p * nb + b) * 2 KB, each box
+    // 1024-byte aligned in the TMA's 128-byte swizzle
+    unsigned char stage[kStages][kStageBoxes * kBoxBytes];
+    // X of a chunk: one row of the chunk's columns per token (bf16, the
+    // 16-byte groups XOR-swizzled by token row), double-buffered.  After the
+    // shrink: the warps' partial sums at 0, this CTA's partial [t][k] at
+    // kRedBytes; after the exchange: v's bf16 high part [t][k] (groups
+    // swizzled) at 0 and its low part at kVBytes.
+    unsigned char xs[2][kMaxJobTokens * kMaxChunkCols * 2];
+    // the peers' partial sums [t][k] of the current unit, written by their
+    // asynchronous DSMEM stores that complete on rbar; double-buffered over
+    // units (slot (q - this rank - 1) mod kCS holds rank q's)
+    float R[2][kCS - 1][kPartFloats];
+    int4 pt[kTableSlots * 2];                         // staged page-table rows (A pages, B pages)
     int ranks[kTableSlots];
     float scales[kTableSlots];
     uint64_t full[kStages];
     uint64_t empty[kStages];
-    uint64_t xbar[2];
+    uint64_t rbar[2];
     int abort;
 };
 
@@ -84,25 +111,14 @@ __device__ __forceinline__ bool mbar_try(uint32_t addr, uint32_t parity) {
     return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_try_cluster(uint32_t addr, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok) : "r"(addr), "r"(parity) : "memory");
-    return ok != 0;
-}
-
 // Bounded wait.  On timeout the CTA-wide abort flag is raised (later waits
 // return at once) and the error word records it; execution continues so
 // that no peer is left waiting for this CTA.
-template <bool kCluster>
 __device__ __forceinline__ void mbar_wait(uint64_t *bar, uint32_t parity, GatherSmem &sm, int32_t *err) {
     const uint32_t a = smem_u32(bar);
-    if (kCluster ? mbar_try_cluster(a, parity) : mbar_try(a, parity)) return;
+    if (mbar_try(a, parity)) return;
     const long long t0 = clock64();
-    while (!(kCluster ? mbar_try_cluster(a, parity) : mbar_try(a, parity))) {
+    while (!mbar_try(a, parity)) {
         if (*(volatile int *)&sm.abort) return;
         if (clock64() - t0 > kWaitLimit) {
             *(volatile int *)&sm.abort = 1;
@@ -121,8 +137,12 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
     }
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+// A consumer warp frees a stage: its reads of the stage have completed (the
+// MMAs that use them issued earlier), and nothing else this arrival would
+// order must reach the producer, so the arrive is relaxed: a release here
+// would wait for the warp's outstanding global stores of Y.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
@@ -141,13 +161,11 @@ __device__ __forceinline__ uint32_t map_peer(uint32_t addr, uint32_t rank) {
     return r;
 }
 
-__device__ __forceinline__ void st_peer_v4(uint32_t addr, float4 v) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
-                 ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
-}
-
-__device__ __forceinline__ void arrive_peer_release(uint32_t addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+// Asynchronous 4-byte store into a peer CTA's shared memory that completes
+// its transaction count on the peer's mbarrier (no fence needed).
+__device__ __forceinline__ void st_async_peer(uint32_t addr, float v, uint32_t bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+                 ::"r"(addr), "r"(__float_as_uint(v)), "r"(bar) : "memory");
 }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -156,16 +174,52 @@ __device__ __forceinline__ uint32_t cluster_rank() {
     return r;
 }
 
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory");
 }
 
-__device__ __forceinline__ void bf16x8(const uint4 &v, float f[8]) {
-    f[0] = __uint_as_float(v.x << 16); f[1] = __uint_as_float(v.x & 0xffff0000u);
-    f[2] = __uint_as_float(v.y << 16); f[3] = __uint_as_float(v.y & 0xffff0000u);
-    f[4] = __uint_as_float(v.z << 16); f[5] = __uint_as_float(v.z & 0xffff0000u);
-    f[6] = __uint_as_float(v.w << 16); f[7] = __uint_as_float(v.w & 0xffff0000u);
+// 16-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t &r0, uint32_t &r1) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr) : "memory");
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr) : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr) : "memory");
+}
+
+// d += a (16 x 16, row) * b (16 x 8, col); bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+                 "{%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint16_t bf16_rn(float f) {
+    uint16_t h;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(f));
+    return h;
+}
+
+// Byte offset of 16-byte group j of row t in a row-major shared array whose
+// rows are a multiple of 128 bytes: groups are XOR-swizzled by row so that
+// the eight rows an ldmatrix reads sit in different banks.
+__device__ __forceinline__ uint32_t swz(int t, int pitch, int j) { return (uint32_t)(t * pitch + ((j ^ (t & 7)) << 4)); }
 
 // Per-slot data of this call, from the shared-memory copy when staged.
 struct SlotMeta {
@@ -212,22 +266,26 @@ __device__ __forceinline__ SlotMeta slot_meta(const GatherArgs &a, const GatherS
 struct UnitGeom {
     int in0, in1;        // d_in slice
     int out0, out1;      // d_out slice
-    int nb;              // 256-column boxes per chunk (chunk width nb * 256)
+    int nb;              // 64-column boxes per page in a chunk (chunk width nb * 64)
     int n_shrink, n_expand;
 };
 
 template <int MODE>
 __device__ __forceinline__ UnitGeom unit_geom(const GatherArgs &a, int np, int e, int E, int crank) {
     UnitGeom g;
-    const int Gi = a.d_in >> 3, Go = a.d_out >> 3;
-    g.in0 = 8 * (int)((long long)Gi * crank / kCS);
-    g.in1 = 8 * (int)((long long)Gi * (crank + 1) / kCS);
-    const int ge0 = (int)((long long)Go * e / E), ge1 = (int)((long long)Go * (e + 1) / E);
-    g.out0 = 8 * (ge0 + (int)((long long)(ge1 - ge0) * crank / kCS));
-    g.out1 = 8 * (ge0 + (int)((long long)(ge1 - ge0) * (crank + 1) / kCS));
-    // As many 256-column boxes per chunk as fit next to the rank's pages: the
-    // chunk width depends on the rank only, so a token's fp32 summation order
-    // does not depend on which job it lands in.
+    // 32-bit arithmetic: column groups fit easily (d <= 2^24 checked on the
+    // host); floor(Go * e / E) is split so that no product leaves 32 bits
+    const unsigned Gi = (unsigned)a.d_in >> 3, Go = (unsigned)a.d_out >> 3;
+    g.in0 = 8 * (int)(Gi * crank / kCS);
+    g.in1 = 8 * (int)(Gi * (crank + 1) / kCS);
+    const unsigned q = Go / (unsigned)E, rm = Go % (unsigned)E;
+    const unsigned ge0 = (unsigned)e * q + ((unsigned)e * rm) / (unsigned)E;
+    const unsigned ge1 = (unsigned)(e + 1) * q + ((unsigned)(e + 1) * rm) / (unsigned)E;
+    g.out0 = 8 * (int)(ge0 + (ge1 - ge0) * crank / kCS);
+    g.out1 = 8 * (int)(ge0 + (ge1 - ge0) * (crank + 1) / kCS);
+    // As many boxes per page as fit in a stage: the chunk width depends on the
+    // rank only, so a token's fp32 summation order does not depend on which
+    // job it lands in.
     g.nb = np > 0 ? kStageBoxes / np : 1;
     const int cw = g.nb * kBoxCols;
     const int win = g.in1 - g.in0, wout = g.out1 - g.out0;
@@ -247,59 +305,20 @@ __device__ __forceinline__ int ld_s32_now(const int *p) {
     return v;
 }
 
-// 8-term dot product summed as a tree (a fixed order, shorter dependency chains).
-__device__ __forceinline__ float dot8(const float a[8], const float x[8]) {
-    const float p0 = fmaf(a[1], x[1], a[0] * x[0]);
-    const float p1 = fmaf(a[3], x[3], a[2] * x[2]);
-    const float p2 = fmaf(a[5], x[5], a[4] * x[4]);
-    const float p3 = fmaf(a[7], x[7], a[6] * x[6]);
-    return (p0 + p1) + (p2 + p3);
-}
-
-// One staged chunk of the shrink: this warp's rank rows k = warp + 8 j for
-// j < RPW, lanes over the chunk's 8-column groups.
-template <int RPW>
-__device__ __forceinline__ void shrink_chunk(const unsigned char *st, const uint4 (*xs)[kStageBoxes * kBoxCols / 8],
-                                             int ng, int nb, int warp, int lane, int r, int n, float (&acc)[8][kNT]) {
-    // tokens in groups of TG: all four at once for few rank rows per warp, two
-    // at a time for 8 rows (the rows' values are re-read from shared memory)
-    constexpr int TG = RPW >= 8 ? 2 : kNT;
-    for (int q = lane; q < ng; q += 32) {
-        const int b = (q * 8) / kBoxCols, cb = q * 8 - b * kBoxCols;
-#pragma unroll
-        for (int t0 = 0; t0 < kNT; t0 += TG) {
-            if (t0 >= n) break;
-            float xf[TG][8];
-#pragma unroll
-            for (int t = 0; t < TG; ++t) {
-                if (t0 + t < n) bf16x8(xs[t0 + t][q], xf[t]);
-                else {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) xf[t][i] = 0.f;
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < RPW; ++j) {
-                const int k = warp + j * kConsumerWarps;
-                if (k < r) {
-                    float af[8];
-                    bf16x8(*reinterpret_cast<const uint4 *>(st + (size_t)((k >> 4) * nb + b) * kBoxBytes +
-                                                            (k & 15) * (kBoxCols * 2) + cb * 2),
-                           af);
-#pragma unroll
-                    for (int t = 0; t < TG; ++t) acc[j][t0 + t] += dot8(af, xf[t]);
-                }
-            }
-        }
-    }
+// Token index t of a job: the first four are in the job record, the rest
+// in the plan's slot-ordered token list.  -1 past the job's end.
+__device__ __forceinline__ int job_token(const GatherArgs &a, const int4 &tk, int q0, int n, int t) {
+    if (t >= n) return -1;
+    if (t < 4) return t == 0 ? tk.x : t == 1 ? tk.y : t == 2 ? tk.z : tk.w;
+    return __ldg(a.perm + q0 + t);
 }
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GatherArgs a,
               int e_max) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    GatherSmem &sm = *reinterpret_cast<GatherSmem *>(smem_raw);
+    extern __shared__ unsigned char smem_raw[];
+    GatherSmem &sm = *reinterpret_cast<GatherSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int crank = (int)cluster_rank();
     const int cluster_id = blockIdx.x / kCS;
@@ -310,16 +329,28 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], kConsumerWarps);
         }
-        // every consumer warp of every CTA of the cluster arrives once per unit
-        mbar_init(&sm.xbar[0], kCS * kConsumerWarps);
-        mbar_init(&sm.xbar[1], kCS * kConsumerWarps);
+        // one arrival per unit (this CTA's expect_tx) plus the peers' bytes
+        mbar_init(&sm.rbar[0], 1);
+        mbar_init(&sm.rbar[1], 1);
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    // Announce this CTA's barriers to its peers; the matching wait comes just
-    // before the first push into a peer.
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-
+    // The cluster barrier is used once: every thread arrives here (thread 0
+    // after initialising the barriers above and fencing that for the
+    // cluster), and waits before its CTA first stores into a peer (or before
+    // it exits).  Peers store into this CTA only for units this CTA also runs
+    // and waits on, so no CTA exits while a store into it is pending.
+    cluster_arrive_relaxed();
+    // Every launch's parameters sit in memory this SM has not read yet: fetch
+    // them and both tensor maps now, while the previous kernel drains, rather
+    // than on first use.
+    if (threadIdx.x == kConsumers) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+    }
+    asm volatile("" ::"l"(a.X), "l"(a.Y), "l"(a.V), "r"(a.T), "r"(a.d_in), "r"(a.d_out), "r"(a.S), "l"(a.ranks),
+                 "l"(a.scales), "l"(a.pt), "l"(a.perm), "l"(a.jobs), "l"(a.hdr), "l"(a.err), "l"(a.rowsA),
+                 "l"(a.rowsB), "r"(e_max));
     // The plan kernel runs before this one; wait for its output.  Then let the
     // next kernel on the stream get its CTAs resident: it reads nothing the
     // kernels write before its own wait, which returns only when this grid has
@@ -345,7 +376,10 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         }
     }
     __syncthreads();
-    if (n_jobs <= 0) return;   // uniform over the grid; no peer traffic has happened
+    if (n_jobs <= 0) {   // uniform over the grid; no peer traffic has happened
+        cluster_wait();
+        return;
+    }
     int E = 1;
     if (MODE != kShrink) {
         E = n_clusters / n_jobs;
@@ -353,210 +387,395 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     }
     const int n_units = n_jobs * E;
 
+    // Cluster exchange of the shrink partials (apply and shrink modes).
+    constexpr bool kXchg = MODE != kExpand;
+
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------------------
-        // Producer warp (lane 0): TMA loads of the adapter's pages.
+        // Producer warp: lane 0 issues the TMA loads of the adapter's pages;
+        // the whole warp takes part in the cluster barriers.
         // ------------------------------------------------------------------
+        int chunk = 0;
+        for (int u = cluster_id; u < n_units; u += n_clusters) {
+            const int ji = u / E;
+            const int4 job = (ji == spec) ? spec_job : a.jobs[2 * ji];
+            const int e = u - ji * E;
+            const SlotMeta m = slot_meta<MODE>(a, sm, staged, job.x);
+            const UnitGeom g = unit_geom<MODE>(a, m.np, e, E, crank);
+            // Shrink chunks, then expand chunks, in the order the consumers use
+            // them; the ring lets the loads run up to kStages chunks ahead,
+            // into the next unit.
+            const int pa[4] = {m.pga.x, m.pga.y, m.pga.z, m.pga.w};
+            const int pb[4] = {m.pgb.x, m.pgb.y, m.pgb.z, m.pgb.w};
+            const int cw = g.nb * kBoxCols;
+            auto issue = [&](int c) {
+                const int s = chunk % kStages;
+                mbar_wait(&sm.empty[s], ((chunk / kStages) & 1) ^ 1, sm, a.err);
+                const bool shrink = c < g.n_shrink;
+                const int c0 = shrink ? g.in0 + c * cw : g.out0 + (c - g.n_shrink) * cw;
+                const int c1 = shrink ? g.in1 : g.out1;
+                const int boxes = min(g.nb, (c1 - c0 + kBoxCols - 1) / kBoxCols);
+                mbar_expect_tx(&sm.full[s], (uint32_t)(m.np * boxes * kBoxBytes));
+                for (int p = 0; p < m.np; ++p)
+                    for (int b = 0; b < boxes; ++b)
+                        tma_load_box(sm.stage[s] + (size_t)(p * g.nb + b) * kBoxBytes, shrink ? &tmA : &tmB,
+                                     c0 + b * kBoxCols, (shrink ? pa[p] : pb[p]) * LORA_PAGE_ROWS, &sm.full[s]);
+                ++chunk;
+            };
+            if (lane == 0)
+                for (int c = 0; c < g.n_shrink + g.n_expand; ++c) issue(c);
+            __syncwarp();
+        }
         if (lane == 0) {
-            int chunk = 0;
-            for (int u = cluster_id; u < n_units; u += n_clusters) {
-                const int ji = u / E;
-                const int4 job = (ji == spec) ? spec_job : a.jobs[2 * ji];
-                const int e = u - ji * E;
-                const SlotMeta m = slot_meta<MODE>(a, sm, staged, job.x);
-                const UnitGeom g = unit_geom<MODE>(a, m.np, e, E, crank);
-                const int pa[4] = {m.pga.x, m.pga.y, m.pga.z, m.pga.w};
-                const int pb[4] = {m.pgb.x, m.pgb.y, m.pgb.z, m.pgb.w};
-                for (int c = 0; c < g.n_shrink + g.n_expand; ++c, ++chunk) {
-                    const int s = chunk % kStages;
-                    mbar_wait<false>(&sm.empty[s], ((chunk / kStages) & 1) ^ 1, sm, a.err);
-                    const bool shrink = c < g.n_shrink;
-                    const int c0 = shrink ? g.in0 + c * g.nb * kBoxCols : g.out0 + (c - g.n_shrink) * g.nb * kBoxCols;
-                    const int c1 = shrink ? g.in1 : g.out1;
-                    const int boxes = min(g.nb, (c1 - c0 + kBoxCols - 1) / kBoxCols);
-                    mbar_expect_tx(&sm.full[s], (uint32_t)(m.np * boxes * kBoxBytes));
-                    for (int p = 0; p < m.np; ++p)
-                        for (int b = 0; b < boxes; ++b)
-                            tma_load_box(sm.stage[s] + (size_t)(p * g.nb + b) * kBoxBytes, shrink ? &tmA : &tmB,
-                                         c0 + b * kBoxCols, (shrink ? pa[p] : pb[p]) * LORA_PAGE_ROWS, &sm.full[s]);
-                }
-            }
             // the loads armed last on each stage have landed before this thread exits
             for (int i = (chunk > kStages ? chunk - kStages : 0); i < chunk; ++i)
                 drain_wait(&sm.full[i % kStages], (i / kStages) & 1);
         }
+        __syncwarp();
+        cluster_wait();
         return;
     }
 
     // ----------------------------------------------------------------------
     // Consumer warps.
     // ----------------------------------------------------------------------
+    const int g8 = lane >> 2, tig = lane & 3;    // MMA fragment coordinates
+    const int li = lane & 7, lj = lane >> 3;     // ldmatrix: row within a matrix, matrix index
     int chunk = 0;
     int iter = 0;
-    bool joined = false;   // waited on the start-up cluster barrier
+    bool joined = false;   // passed the start-up cluster barrier
     for (int u = cluster_id; u < n_units; u += n_clusters, ++iter) {
         const int ji = u / E;
         const int4 job = (ji == spec) ? spec_job : a.jobs[2 * ji];
         const int4 tk = (ji == spec) ? spec_tok : a.jobs[2 * ji + 1];
         const int e = u - ji * E;
-        const int slot = job.x, n = job.y;
-        const int tok[kNT] = {tk.x, tk.y, tk.z, tk.w};
+        const int slot = job.x, n = min(job.y, kMaxJobTokens), q0 = job.z;
         const SlotMeta m = slot_meta<MODE>(a, sm, staged, slot);
         if (m.bad && threadIdx.x == 0 && crank == 0 && e == 0 && a.err) atomicOr(a.err, LORA_DEV_ERR_BAD_PAGE);
-        const int r = m.r;
-        const UnitGeom g = unit_geom<MODE>(a, m.np, e, E, crank);
+        const int r = m.r, np = m.np;
+        const UnitGeom g = unit_geom<MODE>(a, np, e, E, crank);
         const int buf = iter & 1;
         const int cw = g.nb * kBoxCols;
-        // old Y of this thread's columns of the first expand chunk, fetched early
-        float yv[kStageBoxes][kNT];
-        auto load_y = [&](int c0, int wcols) {
+        const int nt = (n + kNTok - 1) / kNTok;   // token tiles of 8
+        const int rows = nt * kNTok;
+        const int pitch = cw * 2;                   // bytes per token row of a staged X chunk
+        if (kXchg && threadIdx.x == 0)   // the peers' partials of this unit: (kCS - 1) * n * r floats
+            mbar_expect_tx(&sm.rbar[buf], (uint32_t)((kCS - 1) * n * r * 4));
+        // this thread's tokens in the expand's output fragments (columns 2 tig,
+        // 2 tig + 1 of each 8-token tile)
+        int otok[kMaxNTiles][2];
 #pragma unroll
-            for (int i = 0; i < kStageBoxes; ++i) {
-                const int col = threadIdx.x + i * kConsumers;
+        for (int j = 0; j < kMaxNTiles; ++j)
 #pragma unroll
-                for (int t = 0; t < kNT; ++t)
-                    yv[i][t] = (t < n && col < wcols) ? a.Y[(size_t)tok[t] * a.d_out + c0 + col] : 0.f;
+            for (int h = 0; h < 2; ++h) otok[j][h] = job_token(a, tk, q0, n, j * kNTok + 2 * tig + h);
+        // Old Y of token tile 0 for this warp's 16-column tiles of an expand
+        // chunk, loaded ahead of use: chunk 0's before the exchange, chunk
+        // c + 1's while chunk c is computed.  Each (token, column) belongs to
+        // exactly one unit.
+        float ypf[kMTW][4];
+        auto load_y = [&](int c, int i) {
+            const int c0 = g.out0 + c * cw;
+            const int nmt = (min(cw, g.out1 - c0) + 15) >> 4;
+            int mt = warp - (c * (cw >> 4)) % kConsumerWarps;
+            if (mt < 0) mt += kConsumerWarps;
+            mt += i * kConsumerWarps;
+            const int colA = c0 + mt * 16 + g8, colB = colA + 8;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int tok = otok[0][h];
+                ypf[i][h] = (mt < nmt && tok >= 0 && colA < g.out1) ? a.Y[(size_t)tok * a.d_out + colA] : 0.f;
+                ypf[i][2 + h] = (mt < nmt && tok >= 0 && colB < g.out1) ? a.Y[(size_t)tok * a.d_out + colB] : 0.f;
+            }
+        };
+        auto load_y0 = [&]() {
+            if (g.n_expand > 0) {
+#pragma unroll
+                for (int i = 0; i < kMTW; ++i) load_y(0, i);
             }
         };
 
         if (MODE != kExpand) {
             // ---- shrink: partial sums over this CTA's d_in slice ----
-            float acc[8][kNT];
+            float acc[kMaxPages][kMaxNTiles][4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
+            for (int p = 0; p < kMaxPages; ++p)
 #pragma unroll
-                for (int t = 0; t < kNT; ++t) acc[j][t] = 0.f;
-            const int rpw = (r + kConsumerWarps - 1) / kConsumerWarps;
+                for (int j = 0; j < kMaxNTiles; ++j)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) acc[p][j][i] = 0.f;
+            const int gq = cw >> 3;   // 16-byte groups per token row
+            auto stage_x = [&](int c) {
+                const int c0 = g.in0 + c * cw;
+                const uint32_t base = smem_u32(sm.xs[c & 1]);
+                for (int i = threadIdx.x; i < rows * gq; i += kConsumers) {
+                    const int t = i / gq, q = i - t * gq;
+                    const int col = c0 + q * 8;
+                    const int tok = (col < g.in1) ? job_token(a, tk, q0, n, t) : -1;
+                    const uint16_t *src = tok >= 0 ? a.X + (size_t)tok * a.d_in + col : a.X;
+                    cp_async16(base + swz(t, pitch, q), src, tok >= 0 ? 16 : 0);
+                }
+                cp_async_commit();
+            };
+            if (g.n_shrink > 0) stage_x(0);
+            int kbase = 0;   // 16-column steps of the slice before this chunk
             for (int c = 0; c < g.n_shrink; ++c, ++chunk) {
                 const int s = chunk % kStages;
                 const int c0 = g.in0 + c * cw;
-                const int wcols = min(cw, g.in1 - c0);
-                const int ng = wcols >> 3;   // 8-column groups in this chunk
-                uint4 (*xs)[kStageBoxes * kBoxCols / 8] = sm.xs[c & 1];
-                // stage the tokens' X columns of this chunk (coalesced, before the weights arrive)
-                for (int i = threadIdx.x; i < n * ng; i += kConsumers) {
-                    const int t = i / ng, q = i - t * ng;
-                    xs[t][q] = __ldg(reinterpret_cast<const uint4 *>(a.X + (size_t)tok[t] * a.d_in + c0 + q * 8));
-                }
-                mbar_wait<false>(&sm.full[s], (chunk / kStages) & 1, sm, a.err);
-                consumer_sync();
-                const unsigned char *st = sm.stage[s];
-                if (rpw <= 1) shrink_chunk<1>(st, xs, ng, g.nb, warp, lane, r, n, acc);
-                else if (rpw <= 2) shrink_chunk<2>(st, xs, ng, g.nb, warp, lane, r, n, acc);
-                else if (rpw <= 4) shrink_chunk<4>(st, xs, ng, g.nb, warp, lane, r, n, acc);
-                else shrink_chunk<8>(st, xs, ng, g.nb, warp, lane, r, n, acc);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.empty[s]);
-            }
-            if (MODE == kApply && g.n_expand > 0) load_y(g.out0, min(cw, g.out1 - g.out0));
-            if (!joined) {
-                asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-                joined = true;
-            }
-            // reduce over lanes (every lane gets the sum), then lane q stores the
-            // value into peer q's slot `crank` and arrives on peer q's barrier
+                const int nks = (min(cw, g.in1 - c0) + 15) >> 4;
+                cp_async_wait_all();
+                mbar_wait(&sm.full[s], (chunk / kStages) & 1, sm, a.err);
+                consumer_sync();   // every thread's X copies of chunk c are in; chunk c-1 is done
+                if (c + 1 < g.n_shrink) stage_x(c + 1);
+                const uint32_t xb = smem_u32(sm.xs[c & 1]);
+                const uint32_t sb = smem_u32(sm.stage[s]);
+                int kk = warp - kbase % kConsumerWarps;
+                if (kk < 0) kk += kConsumerWarps;
+                for (; kk < nks; kk += kConsumerWarps) {
+                    // X fragments (B side) of this step for both token tiles
+                    uint32_t bx[kMaxNTiles][2];
+                    {
+                        const int t = (lj >> 1) * kNTok + li;
+                        const uint32_t ad = xb + swz(t, pitch, 2 * kk + (lj & 1));
+                        if (nt > 1) {
+                            uint32_t r4[4];
+                            ldsm_x4(ad, r4);
+                            bx[0][0] = r4[0]; bx[0][1] = r4[1];
+                            bx[kMaxNTiles - 1][0] = r4[2]; bx[kMaxNTiles - 1][1] = r4[3];
+                        } else {
+                            ldsm_x2(ad, bx[0][0], bx[0][1]);
+                        }
+                    }
+                    const int b = kk >> 2, ks = kk & 3;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int k = warp + j * kConsumerWarps;
-                if (k < r) {
-#pragma unroll
-                    for (int t = 0; t < kNT; ++t) {
-                        if (t < n) {
-                            float x = acc[j][t];
-#pragma unroll
-                            for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-                            if (lane < kCS)
-                                asm volatile("st.shared::cluster.f32 [%0], %1;"
-                                             ::"r"(map_peer(smem_u32(&sm.P[buf][crank][t * r + k]), (uint32_t)lane)),
-                                             "f"(x) : "memory");
+                    for (int p = 0; p < kMaxPages; ++p) {
+                        if (p < np) {
+                            uint32_t af[4];
+                            const int row = li + 8 * (lj & 1);
+                            ldsm_x4(sb + (uint32_t)((p * g.nb + b) * kBoxBytes + row * 128 +
+                                                    (((2 * ks + (lj >> 1)) ^ li) << 4)),
+                                    af);
+                            mma_bf16(acc[p][0], af, bx[0][0], bx[0][1]);
+                            if (kMaxNTiles > 1 && nt > 1)
+                                mma_bf16(acc[p][kMaxNTiles - 1], af, bx[kMaxNTiles - 1][0], bx[kMaxNTiles - 1][1]);
                         }
                     }
                 }
+                kbase += nks;
+                __syncwarp();
+                if (lane == 0) mbar_arrive_relaxed(&sm.empty[s]);
             }
-            __syncwarp();
-            if (lane < kCS) arrive_peer_release(map_peer(smem_u32(&sm.xbar[buf]), (uint32_t)lane));
-            mbar_wait<true>(&sm.xbar[buf], (uint32_t)((iter >> 1) & 1), sm, a.err);
-            // v[k][t] = sum over peers in rank order
+            // the warps' partial sums, added in warp order, become this CTA's
+            // partial; it goes to its own slot and into every peer's
+            consumer_sync();   // every warp is done with the X buffers
+            float *red = reinterpret_cast<float *>(sm.xs);
+#pragma unroll
+            for (int p = 0; p < kMaxPages; ++p)
+#pragma unroll
+                for (int j = 0; j < kMaxNTiles; ++j)
+                    if (p < np && j < nt)
+                        *reinterpret_cast<float4 *>(red + ((warp * kMaxPages + p) * kMaxNTiles + j) * 128 + lane * 4) =
+                            make_float4(acc[p][j][0], acc[p][j][1], acc[p][j][2], acc[p][j][3]);
+            consumer_sync();
+            if (MODE == kApply) load_y0();
+            if (!joined) {   // the peers' barriers are initialised
+                cluster_wait();
+                joined = true;
+            }
+            float *own = reinterpret_cast<float *>(reinterpret_cast<unsigned char *>(&sm.xs) + kRedBytes);
+            const uint32_t own_bar = smem_u32(&sm.rbar[buf]);
+            for (int idx = threadIdx.x; idx < np * nt * 128; idx += kConsumers) {
+                const int p = idx / (nt * 128), rest = idx - p * nt * 128;
+                const int j = rest >> 7, el = rest & 127;
+                // element el of a fragment: lane el / 4, register el % 4
+                const int fl = el >> 2, fr = el & 3;
+                const int k = p * LORA_PAGE_ROWS + (fl >> 2) + 8 * (fr >> 1);
+                const int t = j * kNTok + 2 * (fl & 3) + (fr & 1);
+                if (t < n && k < r) {
+                    float sum = 0.f;
+#pragma unroll 5
+                    for (int w = 0; w < kConsumerWarps; ++w)
+                        sum += red[((w * kMaxPages + p) * kMaxNTiles + j) * 128 + el];
+                    const int o = t * LORA_MAX_RANK + k;
+                    own[o] = sum;
+#pragma unroll
+                    for (int d = 1; d < kCS; ++d) {   // into slot (crank - peer - 1) mod kCS = kCS - 1 - d of peer
+                        const uint32_t peer = (uint32_t)((crank + d) % kCS);
+                        st_async_peer(map_peer(smem_u32(&sm.R[buf][kCS - 1 - d][o]), peer), sum, map_peer(own_bar, peer));
+                    }
+                }
+            }
+            mbar_wait(&sm.rbar[buf], (uint32_t)((iter >> 1) & 1), sm, a.err);
+            consumer_sync();   // this CTA's own partial is complete too; the warps' sums are read
+            // v[t][k] = sum of the CTAs' partials in rank order
             const int nv = n * r;
             for (int idx = threadIdx.x; idx < nv; idx += kConsumers) {
                 const int t = idx / r, k = idx - t * r;
-                float sum = 0.f;
+                const int o = t * LORA_MAX_RANK + k;
+                float v = 0.f;
 #pragma unroll
-                for (int q = 0; q < kCS; ++q) sum += sm.P[buf][q][idx];
-                reinterpret_cast<float *>(&sm.v[k])[t] = sum;
-            }
-            consumer_sync();
-            if (MODE == kShrink) {
-                if (crank == 0) {
-                    for (int idx = threadIdx.x; idx < nv; idx += kConsumers) {
-                        const int t = idx / r, k = idx - t * r;
-                        a.V[(size_t)tok[t] * LORA_MAX_RANK + k] = reinterpret_cast<const float *>(&sm.v[k])[t];
-                    }
+                for (int q = 0; q < kCS; ++q) v += (q == crank) ? own[o] : sm.R[buf][(q - crank - 1 + kCS) % kCS][o];
+                if (MODE == kShrink) {
+                    if (crank == 0) a.V[(size_t)job_token(a, tk, q0, n, t) * LORA_MAX_RANK + k] = v;
+                } else {
+                    const uint16_t h = bf16_rn(v);
+                    const uint16_t l = bf16_rn(v - __uint_as_float((uint32_t)h << 16));
+                    const uint32_t so = swz(t, LORA_MAX_RANK * 2, k >> 3) + (k & 7) * 2;
+                    *reinterpret_cast<uint16_t *>(reinterpret_cast<unsigned char *>(&sm.xs) + so) = h;
+                    *reinterpret_cast<uint16_t *>(reinterpret_cast<unsigned char *>(&sm.xs) + kVBytes + so) = l;
                 }
+            }
+            if (MODE == kShrink) {
                 consumer_sync();
                 continue;
             }
         } else {
+            load_y0();
             for (int idx = threadIdx.x; idx < n * r; idx += kConsumers) {
                 const int t = idx / r, k = idx - t * r;
-                reinterpret_cast<float *>(&sm.v[k])[t] = a.V[(size_t)tok[t] * LORA_MAX_RANK + k];
+                const float v = a.V[(size_t)job_token(a, tk, q0, n, t) * LORA_MAX_RANK + k];
+                const uint16_t h = bf16_rn(v);
+                const uint16_t l = bf16_rn(v - __uint_as_float((uint32_t)h << 16));
+                const uint32_t so = swz(t, LORA_MAX_RANK * 2, k >> 3) + (k & 7) * 2;
+                *reinterpret_cast<uint16_t *>(reinterpret_cast<unsigned char *>(&sm.xs) + so) = h;
+                *reinterpret_cast<uint16_t *>(reinterpret_cast<unsigned char *>(&sm.xs) + kVBytes + so) = l;
             }
-            if (g.n_expand > 0) load_y(g.out0, min(cw, g.out1 - g.out0));
-            consumer_sync();
         }
+        // rank rows past r (up to the page end) and token rows past n of the
+        // tiles hold zeros: the weights' padding rows are zero in the pool,
+        // and 0 * v must not meet a stale non-finite value
+        for (int idx = threadIdx.x; idx < rows * np * LORA_PAGE_ROWS; idx += kConsumers) {
+            const int t = idx / (np * LORA_PAGE_ROWS), k = idx - t * (np * LORA_PAGE_ROWS);
+            if (t >= n || k >= r) {
+                const uint32_t so = swz(t, LORA_MAX_RANK * 2, k >> 3) + (k & 7) * 2;
+                *reinterpret_cast<uint16_t *>(reinterpret_cast<unsigned char *>(&sm.xs) + so) = 0;
+                *reinterpret_cast<uint16_t *>(reinterpret_cast<unsigned char *>(&sm.xs) + kVBytes + so) = 0;
+            }
+        }
+        consumer_sync();
 
         // ---- expand-add over this CTA's d_out slice ----
+        // v fragments (B side) are read from shared memory per page and token
+        // tile: high part (matrices 0, 1) and low part (matrices 2, 3)
+        const uint32_t vbase = smem_u32(&sm.xs) + ((lj >> 1) ? kVBytes : 0);
         const float sc = m.scale;
         for (int c = 0; c < g.n_expand; ++c, ++chunk) {
             const int s = chunk % kStages;
             const int c0 = g.out0 + c * cw;
-            const int wcols = min(cw, g.out1 - c0);
-            if (c > 0) load_y(c0, wcols);   // the first chunk's Y was fetched before the exchange
-            mbar_wait<false>(&sm.full[s], (chunk / kStages) & 1, sm, a.err);
-            const unsigned char *st = sm.stage[s];
+            const int nmt = (min(cw, g.out1 - c0) + 15) >> 4;
+            mbar_wait(&sm.full[s], (chunk / kStages) & 1, sm, a.err);
+            const uint32_t sb = smem_u32(sm.stage[s]);
+            int mt0 = warp - (c * (cw >> 4)) % kConsumerWarps;
+            if (mt0 < 0) mt0 += kConsumerWarps;
 #pragma unroll
-            for (int i = 0; i < kStageBoxes; ++i) {
-                const int col = threadIdx.x + i * kConsumers;
-                if (col < wcols) {
-                    const int b = col / kBoxCols, cb = col - b * kBoxCols;
-                    float accv[kNT];
+            for (int i = 0; i < kMTW; ++i) {
+                const int mt = mt0 + i * kConsumerWarps;
+                if (mt < nmt) {
+                    const int colA = c0 + mt * 16 + g8, colB = colA + 8;
+                    const bool okA = colA < g.out1, okB = colB < g.out1;
+                    // old Y of token tile 1 (tile 0's was loaded ahead)
+                    float y1[4] = {0.f, 0.f, 0.f, 0.f};
+                    if (kMaxNTiles > 1 && nt > 1) {
 #pragma unroll
-                    for (int t = 0; t < kNT; ++t) accv[t] = 0.f;
-#pragma unroll 4
-                    for (int k = 0; k < r; ++k) {
-                        const uint16_t braw = *reinterpret_cast<const uint16_t *>(
-                            st + (size_t)((k >> 4) * g.nb + b) * kBoxBytes + (k & 15) * (kBoxCols * 2) + cb * 2);
-                        const float bk = __uint_as_float((uint32_t)braw << 16);
-                        const float4 v0 = sm.v[k];
-                        accv[0] = fmaf(v0.x, bk, accv[0]); accv[1] = fmaf(v0.y, bk, accv[1]);
-                        accv[2] = fmaf(v0.z, bk, accv[2]); accv[3] = fmaf(v0.w, bk, accv[3]);
+                        for (int h = 0; h < 2; ++h) {
+                            const int tok = otok[kMaxNTiles - 1][h];
+                            if (tok >= 0 && okA) y1[h] = a.Y[(size_t)tok * a.d_out + colA];
+                            if (tok >= 0 && okB) y1[2 + h] = a.Y[(size_t)tok * a.d_out + colB];
+                        }
+                    }
+                    float d[kMaxNTiles][4];
+#pragma unroll
+                    for (int j = 0; j < kMaxNTiles; ++j)
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) d[j][e2] = 0.f;
+                    const int b = mt >> 2, ms = mt & 3;
+#pragma unroll
+                    for (int p = 0; p < kMaxPages; ++p) {
+                        if (p < np) {
+                            uint32_t af[4];
+                            const int krow = li + 8 * (lj >> 1);
+                            ldsm_x4_t(sb + (uint32_t)((p * g.nb + b) * kBoxBytes + krow * 128 +
+                                                      (((2 * ms + (lj & 1)) ^ li) << 4)),
+                                      af);
+#pragma unroll
+                            for (int j = 0; j < kMaxNTiles; ++j) {
+                                if (j < nt) {
+                                    uint32_t bv[4];
+                                    ldsm_x4(vbase + swz(j * kNTok + li, LORA_MAX_RANK * 2, 2 * p + (lj & 1)), bv);
+                                    mma_bf16(d[j], af, bv[0], bv[1]);
+                                    mma_bf16(d[j], af, bv[2], bv[3]);
+                                }
+                            }
+                        }
                     }
 #pragma unroll
-                    for (int t = 0; t < kNT; ++t)
-                        if (t < n) a.Y[(size_t)tok[t] * a.d_out + c0 + col] = fmaf(sc, accv[t], yv[i][t]);
+                    for (int h = 0; h < 2; ++h) {
+                        const int tok0 = otok[0][h];
+                        if (tok0 >= 0 && okA) a.Y[(size_t)tok0 * a.d_out + colA] = fmaf(sc, d[0][h], ypf[i][h]);
+                        if (tok0 >= 0 && okB) a.Y[(size_t)tok0 * a.d_out + colB] = fmaf(sc, d[0][2 + h], ypf[i][2 + h]);
+                        if (kMaxNTiles > 1) {
+                            const int tok1 = otok[kMaxNTiles - 1][h];
+                            if (tok1 >= 0 && okA)
+                                a.Y[(size_t)tok1 * a.d_out + colA] = fmaf(sc, d[kMaxNTiles - 1][h], y1[h]);
+                            if (tok1 >= 0 && okB)
+                                a.Y[(size_t)tok1 * a.d_out + colB] = fmaf(sc, d[kMaxNTiles - 1][2 + h], y1[2 + h]);
+                        }
+                    }
                 }
+                if (c + 1 < g.n_expand) load_y(c + 1, i);   // this slot's tile of the next chunk
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.empty[s]);
+            if (lane == 0) mbar_arrive_relaxed(&sm.empty[s]);
         }
-        consumer_sync();   // sm.v is rewritten by the next unit
+        consumer_sync();   // v is rewritten by the next unit
     }
-    if (!joined) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    if (!joined) cluster_wait();
+}
+
+constexpr size_t kGatherSmemBytes = sizeof(GatherSmem) + 1024;   // + room to align the base to 1 KB
+int g_max_clusters[64] = {};
+
+// Occupancy in clusters of the gather kernel (every mode has the same shape).
+int max_clusters(int *out) {
+    int dev = 0;
+    if (int rc = cuda_check(cudaGetDevice(&dev))) return rc;
+    if (dev < 0 || dev >= 64) return LORA_ERR_INVALID_ARG;
+    if (g_max_clusters[dev] == 0) {
+        const void *fns[3] = {(const void *)gather_kernel<kApply>, (const void *)gather_kernel<kShrink>,
+                              (const void *)gather_kernel<kExpand>};
+        for (const void *f : fns)
+            if (int rc = cuda_check(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                         (int)kGatherSmemBytes)))
+                return rc;
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = kCS;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = kGatherSmemBytes;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cfg.gridDim = dim3(kCS * 256);
+        int ncl = 0;
+        if (int rc = cuda_check(cudaOccupancyMaxActiveClusters(&ncl, gather_kernel<kApply>, &cfg))) return rc;
+        g_max_clusters[dev] = ncl > 0 ? ncl : 1;
+    }
+    *out = g_max_clusters[dev];
+    return LORA_OK;
 }
 
 template <int MODE>
 int launch_mode(const GatherArgs &a, lora_pool_s *pa, lora_pool_s *pb, cudaStream_t st, bool pdl) {
-    static int max_clusters[64] = {};
-    int dev = 0;
-    if (int rc = cuda_check(cudaGetDevice(&dev))) return rc;
-    if (dev < 0 || dev >= 64) return LORA_ERR_INVALID_ARG;
-    const size_t smem = sizeof(GatherSmem);
+    int mcl = 1;
+    if (int rc = max_clusters(&mcl)) return rc;
+    const size_t smem = kGatherSmemBytes;
     CUtensorMap ma, mb;
     if (MODE != kExpand) {
-        if (int rc = pool_tensor_map(pa, kPoolMapGather, &ma)) return rc;
+        if (int rc = pool_tensor_map(pa, &ma)) return rc;
     }
     if (MODE != kShrink) {
-        if (int rc = pool_tensor_map(pb, kPoolMapGather, &mb)) return rc;
+        if (int rc = pool_tensor_map(pb, &mb)) return rc;
     }
     if (MODE == kExpand) ma = mb;
     if (MODE == kShrink) mb = ma;
@@ -574,20 +793,11 @@ int launch_mode(const GatherArgs &a, lora_pool_s *pa, lora_pool_s *pb, cudaStrea
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (max_clusters[dev] == 0) {
-        if (int rc = cuda_check(cudaFuncSetAttribute(gather_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                     (int)smem)))
-            return rc;
-        int ncl = 0;
-        cfg.gridDim = dim3(kCS * 256);
-        if (int rc = cuda_check(cudaOccupancyMaxActiveClusters(&ncl, gather_kernel<MODE>, &cfg))) return rc;
-        max_clusters[dev] = ncl > 0 ? ncl : 1;
-    }
     const int G = a.d_out >> 3;
     int e_max = G / (kCS * 8);
     if (e_max < 1) e_max = 1;
     long long want = (long long)(a.T > 0 ? a.T : 1) * (MODE == kShrink ? 1 : e_max);
-    int ncl = (int)(want < max_clusters[dev] ? want : max_clusters[dev]);
+    int ncl = (int)(want < mcl ? want : mcl);
     if (ncl < 1) ncl = 1;
     cfg.gridDim = dim3(kCS * ncl);
     cfg.numAttrs = pdl ? 2 : 1;
@@ -597,6 +807,8 @@ int launch_mode(const GatherArgs &a, lora_pool_s *pa, lora_pool_s *pb, cudaStrea
 }
 
 }  // namespace
+
+int gather_clusters(int *out) { return max_clusters(out); }
 
 int launch_gather(GatherMode mode, const GatherArgs &a, lora_pool_s *pa, lora_pool_s *pb, cudaStream_t st, bool pdl) {
     switch (mode) {

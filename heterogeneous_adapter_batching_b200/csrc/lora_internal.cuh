@@ -70,8 +70,8 @@ struct lora_pool_s {
     std::map<std::tuple<const void *, int, int>, std::vector<int>> owners;
     std::mutex mu;
     // TMA descriptors of the pool, built on first use (see pool_tensor_map)
-    CUtensorMap tmap[2];
-    bool tmap_ok[2] = {false, false};
+    CUtensorMap tmap;
+    bool tmap_ok = false;
 };
 
 namespace lora {
@@ -80,10 +80,8 @@ namespace lora {
 bool tma_supported();
 int make_tensor_map(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, uint64_t cols,
                     uint64_t rows, uint32_t box_cols, uint32_t box_rows, bool swizzle128);
-// Pool maps: kPoolMapGather = box 256 columns x 16 rows (one page), no swizzle;
-// kPoolMapTile = box 64 columns x 16 rows, 128-byte swizzle.
-enum { kPoolMapGather = 0, kPoolMapTile = 1 };
-int pool_tensor_map(lora_pool_s *pool, int kind, CUtensorMap *out);
+// The pool's map: a box is 64 columns x 16 rows (one page high), 128-byte swizzle.
+int pool_tensor_map(lora_pool_s *pool, CUtensorMap *out);
 
 // Process-wide options.
 int opt_long_segment();
@@ -151,6 +149,9 @@ struct GatherArgs {
     long long rowsB;
 };
 int launch_gather(GatherMode mode, const GatherArgs &a, lora_pool_s *pa, lora_pool_s *pb, cudaStream_t st, bool pdl);
+// Clusters the gather kernel keeps resident on the current device (its grid
+// size in clusters when there is enough work).
+int gather_clusters(int *out);
 
 struct TileArgs {
     const uint16_t *X;

@@ -18,10 +18,12 @@
 //   perm_short          perm without the tokens of such runs (a stable
 //                       compaction, so still grouped by slot);
 //   jobs                the short tokens of every slot, split into gather
-//                       jobs of at most job_tokens (<= 4): two int4 per job,
-//                       {slot, count, first index into perm_short, 0} and the
-//                       job's token indices (-1 padded), so a consumer needs
-//                       a single read to know its work.
+//                       jobs of at most job_tokens (<= LORA_MAX_JOB_TOKENS),
+//                       balanced in size: two int4 per job, {slot, count,
+//                       first index into perm_short, 0} and the job's first
+//                       four token indices (-1 padded), so a decode consumer
+//                       needs a single read to know its work (a larger job's
+//                       further tokens follow in perm_short).
 // Invalid ids (outside [-1, S) or an empty slot) are dropped and flagged.
 //
 // One CTA of 1024 threads.  W warps (W * S <= 16384) own contiguous token
@@ -81,7 +83,7 @@ __device__ __forceinline__ bool is_break(const int32_t *ids, int t, int id, bool
 
 __global__ void __launch_bounds__(kPlanThreads, 1)
 plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ ranks, int S, int W,
-            int long_thresh, int job_tokens, PlanOut out, int32_t *err_dev) {
+            int long_thresh, int job_tokens, int clusters, PlanOut out, int32_t *err_dev) {
     // Let the dependent kernel's CTAs get resident while the plan runs; they
     // wait for this grid's completion before reading its output.
     asm volatile("griddepcontrol.launch_dependents;");
@@ -90,7 +92,7 @@ plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ 
     int *cnt = smem;                       // [S][W] per-warp counts, then scan offsets
     int *scnt = cnt + (size_t)S * W;       // [S] short tokens per slot
     __shared__ int warp_tot[32];
-    __shared__ int s_total[8];
+    __shared__ int s_total[12];
     __shared__ int wfirst[32], wlast[32], carry_l[32], carry_r[32];
 
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -270,6 +272,29 @@ plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ 
     {
         const int per = (S + blockDim.x - 1) / blockDim.x;   // <= 4 for S <= 4096
         const int k0 = tid * per, k1 = min(S, k0 + per);
+        // Job size: the candidates are 4, 8 and the cap job_tokens (each at
+        // most the cap).  The largest is taken that still gives min(jobs at
+        // the smallest size, clusters) jobs: a batch with fewer jobs than the
+        // gather kernel has clusters keeps its parallelism, a larger one gets
+        // fewer reads of each adapter.
+        const int cand[3] = {min(4, job_tokens), min(8, job_tokens), job_tokens};
+        int njc[3] = {0, 0, 0};
+        for (int k = k0; k < k1; ++k) {
+            const int c = scnt[k];
+#pragma unroll
+            for (int i = 0; i < 3; ++i)
+                if (c > 0) njc[i] += (c + cand[i] - 1) / cand[i];
+        }
+#pragma unroll
+        for (int i = 0; i < 3; ++i) (void)block_exclusive_scan(njc[i], warp_tot, &s_total[6 + i]);
+        {
+            const int want = min(s_total[6], clusters);
+            int jt = cand[0];
+#pragma unroll
+            for (int i = 1; i < 3; ++i)
+                if (cand[i] <= job_tokens && s_total[6 + i] >= want) jt = cand[i];
+            job_tokens = jt;
+        }
         int sh_local = 0, nj_local = 0, ns_local = 0;
         for (int k = k0; k < k1; ++k) {
             const int c = scnt[k];
@@ -347,7 +372,9 @@ int launch_plan(const int32_t *ids, int T, const int32_t *ranks, int S, int long
         if (rc) return rc;
         attr_set[dev] = true;
     }
-    plan_kernel<<<1, kPlanThreads, smem, st>>>(ids, T, ranks, S, W, long_thresh, job_tokens, out, err_dev);
+    int clusters = 1;
+    if (int rc = gather_clusters(&clusters)) return rc;
+    plan_kernel<<<1, kPlanThreads, smem, st>>>(ids, T, ranks, S, W, long_thresh, job_tokens, clusters, out, err_dev);
     count_launch();
     return cuda_check(cudaGetLastError());
 }

@@ -221,6 +221,16 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
     TileSmem &sm = *reinterpret_cast<TileSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+    // Fetch this launch's parameters and tensor maps while the previous
+    // kernel drains.
+    if (threadIdx.x == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmX)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmY)) : "memory");
+    }
+    asm volatile("" ::"l"(a.X), "l"(a.Y), "r"(a.T), "r"(a.d_in), "r"(a.d_out), "l"(a.ranks), "l"(a.scales),
+                 "l"(a.pt), "l"(a.tiles), "l"(a.hdr), "l"(a.err), "l"(a.rowsA), "l"(a.rowsB), "r"(a.long_thresh));
     // The kernels before this one on the stream produce the plan.  A batch
     // without long runs has no tiles: leave before touching tensor memory.
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -493,8 +503,8 @@ int launch_tiles(const TileArgs &a, cudaStream_t st, bool pdl) {
         return rc;
     if (int rc = make_tensor_map(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.Y, (uint64_t)a.d_out, (uint64_t)a.T, 32, kM, true))
         return rc;
-    if (int rc = pool_tensor_map(const_cast<lora_pool_s *>(a.pa), kPoolMapTile, &ma)) return rc;
-    if (int rc = pool_tensor_map(const_cast<lora_pool_s *>(a.pb), kPoolMapTile, &mb)) return rc;
+    if (int rc = pool_tensor_map(const_cast<lora_pool_s *>(a.pa), &ma)) return rc;
+    if (int rc = pool_tensor_map(const_cast<lora_pool_s *>(a.pb), &mb)) return rc;
     // one CTA per SM (never more than there can be (tile, n-tile) items)
     const long long max_tiles = (a.T + kM - 1) / kM + (a.long_thresh > 0 ? a.T / a.long_thresh : 0);
     long long grid = num_sms[dev];

@@ -45,20 +45,17 @@ int make_tensor_map(CUtensorMap *m, CUtensorMapDataType dt, int esize, const voi
     return r == CUDA_SUCCESS ? LORA_OK : LORA_ERR_CUDA;
 }
 
-int pool_tensor_map(lora_pool_s *pool, int kind, CUtensorMap *out) {
-    if (!pool || kind < 0 || kind > 1) return LORA_ERR_INVALID_ARG;
+int pool_tensor_map(lora_pool_s *pool, CUtensorMap *out) {
+    if (!pool) return LORA_ERR_INVALID_ARG;
     std::lock_guard<std::mutex> g(pool->mu);
-    if (!pool->tmap_ok[kind]) {
+    if (!pool->tmap_ok) {
         const uint64_t rows = (uint64_t)pool->num_pages * LORA_PAGE_ROWS;
-        const int rc = kind == kPoolMapGather
-                           ? make_tensor_map(&pool->tmap[kind], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pool->base,
-                                             (uint64_t)pool->width, rows, 256, LORA_PAGE_ROWS, false)
-                           : make_tensor_map(&pool->tmap[kind], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pool->base,
-                                             (uint64_t)pool->width, rows, 64, LORA_PAGE_ROWS, true);
-        if (rc) return rc;
-        pool->tmap_ok[kind] = true;
+        if (int rc = make_tensor_map(&pool->tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pool->base,
+                                     (uint64_t)pool->width, rows, 64, LORA_PAGE_ROWS, true))
+            return rc;
+        pool->tmap_ok = true;
     }
-    *out = pool->tmap[kind];
+    *out = pool->tmap;
     return LORA_OK;
 }
 

@@ -66,6 +66,7 @@ typedef struct lora_pool_s *lora_pool_t;        /* opaque host handle of one pag
 #define LORA_PAGE_ROWS            16   /* rank-rows per page */
 #define LORA_MAX_RANK             64
 #define LORA_MAX_PAGES_PER_MATRIX 4    /* LORA_MAX_RANK / LORA_PAGE_ROWS */
+#define LORA_MAX_JOB_TOKENS       16   /* most tokens one gather job serves (one weight read) */
 #define LORA_MAX_SLOTS            4096
 
 /* ------------------------------------------------------------------------ */
@@ -77,7 +78,7 @@ typedef struct lora_pool_s *lora_pool_t;        /* opaque host handle of one pag
 /* Wrap caller-owned device memory dev_buf[bytes] as a pool of pages of
  * page_rows (must be LORA_PAGE_ROWS) rows of `width` bf16 values each.
  * num_pages = bytes / (page_rows * width * 2).  dev_buf must be 256-byte
- * aligned and width a positive multiple of 8.  The caller keeps ownership of
+ * aligned and width a positive multiple of 8, at most 2^24.  The caller keeps ownership of
  * dev_buf and must keep it alive until lora_pool_destroy; the library owns
  * the host-side free list.  Physical row p*page_rows + j of the pool is the
  * bf16 row at dev_buf + (p*page_rows + j) * width * 2 bytes. */
@@ -224,7 +225,9 @@ int lora_apply_noalloc(const uint16_t *X, float *Y, int T, int d_in, int d_out, 
 
 #define LORA_OPT_LONG_SEGMENT   1   /* runs of >= this many consecutive tokens of one slot use the tensor-core path
                                         (default 128, one full tile; 0 = never) */
-#define LORA_OPT_DECODE_JOB_TOKENS 2 /* max tokens per gather job (1..4, default 4) */
+#define LORA_OPT_DECODE_JOB_TOKENS 2 /* max tokens per gather job: the short tokens of a slot are split into
+                                        jobs of at most this many, each reading the weights once
+                                        (1..LORA_MAX_JOB_TOKENS, default LORA_MAX_JOB_TOKENS) */
 
 int lora_set_option(int key, int value);
 int lora_get_option(int key);

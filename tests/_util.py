@@ -96,6 +96,16 @@ def expected_work(ids, ranks, long_thresh: int, job_tokens: int):
     return n_jobs, n_tiles
 
 
+def job_size_candidates(jmax: int):
+    """Job sizes the plan chooses from under the cap jmax."""
+    return sorted({min(4, jmax), min(8, jmax), jmax})
+
+
+def plan_job_tokens(ws):
+    """Job size the plan chose (PlanHeader field 6 at the head of the workspace)."""
+    return int(ws[:32].cpu().numpy().view(np.int32)[6])
+
+
 def plan_counts(ws):
     """(n_valid, n_seg, n_jobs, n_tiles) from the head of a workspace the library
     filled (the plan header is the workspace's first 16 bytes)."""

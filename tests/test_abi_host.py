@@ -123,7 +123,8 @@ def test_options(lib):
     try:
         assert lib.lora_set_option(1, 0) == 0 and lib.lora_get_option(1) == 0
         assert lib.lora_set_option(1, -1) == -1
-        assert lib.lora_set_option(2, 5) == -1 and lib.lora_set_option(2, 0) == -1
+        assert lib.lora_set_option(2, 17) == -1 and lib.lora_set_option(2, 0) == -1
+        assert lib.lora_set_option(2, 16) == 0 and lib.lora_get_option(2) == 16
         assert lib.lora_set_option(2, 3) == 0 and lib.lora_get_option(2) == 3
         assert lib.lora_set_option(99, 1) == -1 and lib.lora_get_option(99) == -1
     finally:

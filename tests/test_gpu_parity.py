@@ -48,7 +48,7 @@ def test_tiny_config(H):
     U.assert_parity(Y, ref, wl.Y_base)
 
 
-@pytest.mark.parametrize("job_tokens", [1, 3, 4])
+@pytest.mark.parametrize("job_tokens", [1, 3, 4, 9, 16])
 @pytest.mark.parametrize("seed,T,d_in,d_out,S", [
     (1, 1, 64, 64, 3), (2, 7, 24, 40, 5), (3, 33, 264, 136, 9), (4, 100, 512, 1032, 17),
     (5, 257, 8, 8, 4), (6, 64, 1000, 2000, 40),
@@ -63,21 +63,34 @@ def test_random_small(H, seed, T, d_in, d_out, S, job_tokens):
     U.assert_parity(Y, ref, wl.Y_base)
 
 
+def _check_job_size(layer, wl, expect):
+    """The plan's job size and job count.  On a B200 the gather kernel keeps
+    about 33 clusters: 64 Zipf decode tokens give 25 jobs of 4 (fewer than
+    the clusters, so the size stays 4); 256 MLP tokens give about 100 (so the
+    size grows to 16, still leaving more jobs than clusters)."""
+    jt = U.plan_job_tokens(layer.ws)
+    assert jt == expect
+    n_jobs = U.plan_counts(layer.ws)[2]
+    assert n_jobs == U.expected_work(wl.ids, wl.ranks(), 0, jt)[0]
+
+
 def test_decode_q_proj_7b_full(H):
     wl = W.decode_q_proj_7b()
-    Y, err, _ = _run_apply(H, wl)
+    Y, err, layer = _run_apply(H, wl)
     ref, rerr = U.oracle_full(wl)
     assert err == rerr == 0
     U.assert_parity(Y, ref, wl.Y_base)
+    _check_job_size(layer, wl, 4)
 
 
 @pytest.mark.parametrize("which", ["up", "down"])
 def test_mixed_mlp_full(H, which):
     wl = W.mixed_mlp(which=which)
-    Y, err, _ = _run_apply(H, wl)
+    Y, err, layer = _run_apply(H, wl)
     ref, rerr = U.oracle_full(wl)
     assert err == rerr == 0
     U.assert_parity(Y, ref, wl.Y_base)
+    _check_job_size(layer, wl, 16)
 
 
 def test_prefill_full(H):

@@ -41,7 +41,9 @@ def _apply(wl, H=None):
     torch.cuda.synchronize()
     if H is not None:
         lt = H.lora_get_option(H.OPT_LONG_SEGMENT)
-        jt = H.lora_get_option(H.OPT_DECODE_JOB_TOKENS)
+        jmax = H.lora_get_option(H.OPT_DECODE_JOB_TOKENS)
+        jt = U.plan_job_tokens(layer.ws)
+        assert jt in U.job_size_candidates(jmax)
         n_valid, n_seg, n_jobs, n_tiles = U.plan_counts(layer.ws)
         assert (n_jobs, n_tiles) == U.expected_work(wl.ids, wl.ranks(), lt, jt)
     return Y.cpu().numpy(), int(layer.err.item())
