@@ -59,6 +59,7 @@ constexpr int kStageBoxes = 16;              // a stage holds 16 boxes = 32 KB
 constexpr int kMaxChunkCols = kStageBoxes * kBoxCols;   // chunk width with a single page
 constexpr int kTableSlots = 128;             // page tables up to this many slots live in shared memory
 constexpr long long kWaitLimit = 2000000000LL;   // cycles (~1 s)
+constexpr int kMaxSplit = 64;                // most parts d_out is split into
 constexpr int kMTW = (kMaxChunkCols / 16 + kConsumerWarps - 1) / kConsumerWarps;   // a warp's 16-column tiles per chunk
 
 static_assert(kMaxJobTokens == LORA_MAX_JOB_TOKENS, "job size must be a whole number of MMA tiles");
@@ -87,6 +88,7 @@ struct __align__(1024) GatherSmem {
     int4 pt[kTableSlots * 2];                         // staged page-table rows (A pages, B pages)
     int ranks[kTableSlots];
     float scales[kTableSlots];
+    int ebound[kMaxSplit + 1];                        // d_out split: first 8-column group of part e
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t rbar[2];
@@ -271,16 +273,13 @@ struct UnitGeom {
 };
 
 template <int MODE>
-__device__ __forceinline__ UnitGeom unit_geom(const GatherArgs &a, int np, int e, int E, int crank) {
+__device__ __forceinline__ UnitGeom unit_geom(const GatherArgs &a, const GatherSmem &sm, int np, int e, int crank) {
     UnitGeom g;
-    // 32-bit arithmetic: column groups fit easily (d <= 2^24 checked on the
-    // host); floor(Go * e / E) is split so that no product leaves 32 bits
-    const unsigned Gi = (unsigned)a.d_in >> 3, Go = (unsigned)a.d_out >> 3;
+    // 32-bit arithmetic: column groups fit easily (d <= 2^24 checked on the host)
+    const unsigned Gi = (unsigned)a.d_in >> 3;
     g.in0 = 8 * (int)(Gi * crank / kCS);
     g.in1 = 8 * (int)(Gi * (crank + 1) / kCS);
-    const unsigned q = Go / (unsigned)E, rm = Go % (unsigned)E;
-    const unsigned ge0 = (unsigned)e * q + ((unsigned)e * rm) / (unsigned)E;
-    const unsigned ge1 = (unsigned)(e + 1) * q + ((unsigned)(e + 1) * rm) / (unsigned)E;
+    const unsigned ge0 = (unsigned)sm.ebound[e], ge1 = (unsigned)sm.ebound[e + 1];
     g.out0 = 8 * (int)(ge0 + (ge1 - ge0) * crank / kCS);
     g.out1 = 8 * (int)(ge0 + (ge1 - ge0) * (crank + 1) / kCS);
     // As many boxes per page as fit in a stage: the chunk width depends on the
@@ -351,21 +350,11 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     asm volatile("" ::"l"(a.X), "l"(a.Y), "l"(a.V), "r"(a.T), "r"(a.d_in), "r"(a.d_out), "r"(a.S), "l"(a.ranks),
                  "l"(a.scales), "l"(a.pt), "l"(a.perm), "l"(a.jobs), "l"(a.hdr), "l"(a.err), "l"(a.rowsA),
                  "l"(a.rowsB), "r"(e_max));
-    // The plan kernel runs before this one; wait for its output.  Then let the
-    // next kernel on the stream get its CTAs resident: it reads nothing the
-    // kernels write before its own wait, which returns only when this grid has
-    // completed.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;");
-
-    // Issue the first job record (a guess that holds whenever there are at
-    // least half as many jobs as clusters), the job count and the slot tables
-    // together, so their latencies overlap.
-    const int spec = cluster_id < a.T ? cluster_id : a.T - 1;
-    const int4 spec_job = ld_v4_now(a.jobs + 2 * spec);
-    const int4 spec_tok = ld_v4_now(a.jobs + 2 * spec + 1);
-    const int n_jobs = ld_s32_now(&a.hdr->n_jobs);
-    // Small page tables, ranks and scales are staged in shared memory.
+    // Small page tables, ranks and scales are staged in shared memory.  They
+    // are the caller's slot state, not the plan's output, so they are read
+    // before this kernel waits for the kernels ahead of it (the library's own
+    // kernels, the only ones here that let a dependent start early, never
+    // write them).
     const bool staged = a.S <= kTableSlots;
     if (staged) {
         for (int i = threadIdx.x; i < a.S; i += kThreads) {
@@ -375,15 +364,32 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             sm.scales[i] = (MODE == kShrink) ? 0.f : a.scales[i];
         }
     }
+    // The plan kernel runs before this one; wait for its output.  Then let the
+    // next kernel on the stream get its CTAs resident: it reads nothing the
+    // kernels write before its own wait, which returns only when this grid has
+    // completed.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+
+    // Issue the first job record (a guess that holds whenever there are at
+    // least half as many jobs as clusters) and the job count together, so
+    // their latencies overlap.
+    const int spec = cluster_id < a.T ? cluster_id : a.T - 1;
+    const int4 spec_job = ld_v4_now(a.jobs + 2 * spec);
+    const int4 spec_tok = ld_v4_now(a.jobs + 2 * spec + 1);
+    const int n_jobs = ld_s32_now(&a.hdr->n_jobs);
+    int E = 1;
+    if (MODE != kShrink && n_jobs > 0) {
+        E = n_clusters / n_jobs;
+        E = E < 1 ? 1 : (E > e_max ? e_max : E);
+        E = E > kMaxSplit ? kMaxSplit : E;
+    }
+    // part e of the d_out split starts at 8-column group floor(Go * e / E)
+    if (threadIdx.x <= E) sm.ebound[threadIdx.x] = (int)((long long)(a.d_out >> 3) * threadIdx.x / E);
     __syncthreads();
     if (n_jobs <= 0) {   // uniform over the grid; no peer traffic has happened
         cluster_wait();
         return;
-    }
-    int E = 1;
-    if (MODE != kShrink) {
-        E = n_clusters / n_jobs;
-        E = E < 1 ? 1 : (E > e_max ? e_max : E);
     }
     const int n_units = n_jobs * E;
 
@@ -401,7 +407,7 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             const int4 job = (ji == spec) ? spec_job : a.jobs[2 * ji];
             const int e = u - ji * E;
             const SlotMeta m = slot_meta<MODE>(a, sm, staged, job.x);
-            const UnitGeom g = unit_geom<MODE>(a, m.np, e, E, crank);
+            const UnitGeom g = unit_geom<MODE>(a, sm, m.np, e, crank);
             // Shrink chunks, then expand chunks, in the order the consumers use
             // them; the ring lets the loads run up to kStages chunks ahead,
             // into the next unit.
@@ -453,7 +459,7 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         const SlotMeta m = slot_meta<MODE>(a, sm, staged, slot);
         if (m.bad && threadIdx.x == 0 && crank == 0 && e == 0 && a.err) atomicOr(a.err, LORA_DEV_ERR_BAD_PAGE);
         const int r = m.r, np = m.np;
-        const UnitGeom g = unit_geom<MODE>(a, np, e, E, crank);
+        const UnitGeom g = unit_geom<MODE>(a, sm, np, e, crank);
         const int buf = iter & 1;
         const int cw = g.nb * kBoxCols;
         const int nt = (n + kNTok - 1) / kNTok;   // token tiles of 8

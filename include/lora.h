@@ -21,6 +21,13 @@
  *  - Every compute call is asynchronous on the given stream and does no
  *    host synchronisation.  Pointers named *_dev, and X, Y, V, ids, ranks,
  *    scales, page_table and ws, are device pointers; everything else is host.
+ *  - The library's kernels let the next kernel on the stream start its
+ *    preamble early (programmatic dependent launch).  ranks, scales and
+ *    page_table are slot state and may be read in that preamble, before the
+ *    kernels ahead on the stream have finished; every other input is read
+ *    only after they have.  So a kernel that writes ranks, scales or
+ *    page_table must not itself let its dependents start early (ordinary
+ *    kernels do not).
  *  - bf16 data is passed as uint16_t bit patterns.  Matrices are row-major.
  *  - Inputs are never modified, except Y (updated in place) and the outputs
  *    named in each call.
