@@ -266,6 +266,8 @@ PROFILE_FOR = {
     # workload -> (profile summary, kernel source it was captured from)
     "decode_q_proj_7b": ("profiles/gather_kernel_decode_q_proj_7b.md",
                          "heterogeneous_adapter_batching_b200/csrc/lora_gather.cu"),
+    "mixed_mlp_up": ("profiles/gather_kernel_mixed_mlp_up.md",
+                     "heterogeneous_adapter_batching_b200/csrc/lora_gather.cu"),
     "prefill": ("profiles/tiles_kernel_prefill.md", "heterogeneous_adapter_batching_b200/csrc/lora_tiles.cu"),
 }
 
