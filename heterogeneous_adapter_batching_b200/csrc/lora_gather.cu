@@ -60,7 +60,6 @@ constexpr int kMaxChunkCols = kStageBoxes * kBoxCols;   // chunk width with a si
 constexpr int kTableSlots = 128;             // page tables up to this many slots live in shared memory
 constexpr long long kWaitLimit = 2000000000LL;   // cycles (~1 s)
 constexpr int kMaxSplit = 64;                // most parts d_out is split into
-constexpr int kMTW = (kMaxChunkCols / 16 + kConsumerWarps - 1) / kConsumerWarps;   // a warp's 16-column tiles per chunk
 
 static_assert(kMaxJobTokens == LORA_MAX_JOB_TOKENS, "job size must be a whole number of MMA tiles");
 // After the shrink the X buffers hold the warps' partial sums (kRedBytes),
@@ -68,8 +67,14 @@ static_assert(kMaxJobTokens == LORA_MAX_JOB_TOKENS, "job size must be a whole nu
 constexpr int kRedBytes = kConsumerWarps * kMaxPages * kMaxNTiles * 128 * 4;
 constexpr int kPartFloats = kMaxJobTokens * LORA_MAX_RANK;
 constexpr int kVBytes = kMaxJobTokens * LORA_MAX_RANK * 2;   // one bf16 part of v
+// During the expand each warp turns its MMA results into rows of Y through a
+// 16-token x 16-column fp32 tile in the X buffers, after the two parts of v.
+constexpr int kYTileBytes = kMaxJobTokens * 16 * 4;
+constexpr int kYTileOff = 2 * kVBytes;
 static_assert(kRedBytes + kPartFloats * 4 <= 2 * kMaxJobTokens * kMaxChunkCols * 2,
               "the partial sums must fit in the X buffers");
+static_assert(kYTileOff + kConsumerWarps * kYTileBytes <= 2 * kMaxJobTokens * kMaxChunkCols * 2,
+              "the warps' Y tiles must fit in the X buffers");
 
 struct __align__(1024) GatherSmem {
     // stage s, box (page p, column block b) at (p * nb + b) * 2 KB, each box
@@ -467,36 +472,28 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         const int pitch = cw * 2;                   // bytes per token row of a staged X chunk
         if (kXchg && threadIdx.x == 0)   // the peers' partials of this unit: (kCS - 1) * n * r floats
             mbar_expect_tx(&sm.rbar[buf], (uint32_t)((kCS - 1) * n * r * 4));
-        // this thread's tokens in the expand's output fragments (columns 2 tig,
-        // 2 tig + 1 of each 8-token tile)
-        int otok[kMaxNTiles][2];
+        // Y is read and written in rows: lane = (token rt of an 8-token tile,
+        // 4-column group rc of a 16-column tile), one float4 each.
+        const int rt = lane >> 2, rc = lane & 3;
+        int rtok[kMaxNTiles];
 #pragma unroll
-        for (int j = 0; j < kMaxNTiles; ++j)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) otok[j][h] = job_token(a, tk, q0, n, j * kNTok + 2 * tig + h);
-        // Old Y of token tile 0 for this warp's 16-column tiles of an expand
-        // chunk, loaded ahead of use: chunk 0's before the exchange, chunk
-        // c + 1's while chunk c is computed.  Each (token, column) belongs to
-        // exactly one unit.
-        float ypf[kMTW][4];
-        auto load_y = [&](int c, int i) {
-            const int c0 = g.out0 + c * cw;
-            const int nmt = (min(cw, g.out1 - c0) + 15) >> 4;
-            int mt = warp - (c * (cw >> 4)) % kConsumerWarps;
-            if (mt < 0) mt += kConsumerWarps;
-            mt += i * kConsumerWarps;
-            const int colA = c0 + mt * 16 + g8, colB = colA + 8;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int tok = otok[0][h];
-                ypf[i][h] = (mt < nmt && tok >= 0 && colA < g.out1) ? a.Y[(size_t)tok * a.d_out + colA] : 0.f;
-                ypf[i][2 + h] = (mt < nmt && tok >= 0 && colB < g.out1) ? a.Y[(size_t)tok * a.d_out + colB] : 0.f;
-            }
+        for (int j = 0; j < kMaxNTiles; ++j) rtok[j] = job_token(a, tk, q0, n, j * kNTok + rt);
+        // Old Y of a 16-column tile, loaded ahead: token tile 0 two tiles
+        // ahead (the warp's first two tiles of the first expand chunk before
+        // the exchange), token tile 1 one tile ahead.  Each (token, column)
+        // belongs to exactly one unit.
+        auto load_y = [&](int c0, int mt, int nmt, int j) {
+            const int col = c0 + mt * 16 + 4 * rc;
+            return (mt < nmt && rtok[j] >= 0 && col < g.out1)
+                       ? *reinterpret_cast<const float4 *>(a.Y + (size_t)rtok[j] * a.d_out + col)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
         };
+        float4 ya = make_float4(0.f, 0.f, 0.f, 0.f), yb = ya;   // token tile 0 of this tile and the next
         auto load_y0 = [&]() {
             if (g.n_expand > 0) {
-#pragma unroll
-                for (int i = 0; i < kMTW; ++i) load_y(0, i);
+                const int nmt0 = (min(cw, g.out1 - g.out0) + 15) >> 4;
+                ya = load_y(g.out0, warp, nmt0, 0);
+                yb = load_y(g.out0, warp + kConsumerWarps, nmt0, 0);
             }
         };
 
@@ -664,70 +661,76 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         // tile: high part (matrices 0, 1) and low part (matrices 2, 3)
         const uint32_t vbase = smem_u32(&sm.xs) + ((lj >> 1) ? kVBytes : 0);
         const float sc = m.scale;
+        float *ytile = reinterpret_cast<float *>(reinterpret_cast<unsigned char *>(&sm.xs) + kYTileOff +
+                                                 warp * kYTileBytes);
         for (int c = 0; c < g.n_expand; ++c, ++chunk) {
             const int s = chunk % kStages;
             const int c0 = g.out0 + c * cw;
             const int nmt = (min(cw, g.out1 - c0) + 15) >> 4;
             mbar_wait(&sm.full[s], (chunk / kStages) & 1, sm, a.err);
             const uint32_t sb = smem_u32(sm.stage[s]);
-            int mt0 = warp - (c * (cw >> 4)) % kConsumerWarps;
-            if (mt0 < 0) mt0 += kConsumerWarps;
+            int mt = warp - (c * (cw >> 4)) % kConsumerWarps;
+            if (mt < 0) mt += kConsumerWarps;
+            if (c > 0) {
+                ya = load_y(c0, mt, nmt, 0);
+                yb = load_y(c0, mt + kConsumerWarps, nmt, 0);
+            }
+#pragma unroll 1
+            for (; mt < nmt; mt += kConsumerWarps) {
+                const float4 yc = load_y(c0, mt + 2 * kConsumerWarps, nmt, 0);   // two tiles ahead
+                const float4 y1 = (kMaxNTiles > 1 && nt > 1) ? load_y(c0, mt, nmt, kMaxNTiles - 1)
+                                                             : make_float4(0.f, 0.f, 0.f, 0.f);
+                const int col = c0 + mt * 16 + 4 * rc;
+                const bool ok = col < g.out1;
+                float d[kMaxNTiles][4];
 #pragma unroll
-            for (int i = 0; i < kMTW; ++i) {
-                const int mt = mt0 + i * kConsumerWarps;
-                if (mt < nmt) {
-                    const int colA = c0 + mt * 16 + g8, colB = colA + 8;
-                    const bool okA = colA < g.out1, okB = colB < g.out1;
-                    // old Y of token tile 1 (tile 0's was loaded ahead)
-                    float y1[4] = {0.f, 0.f, 0.f, 0.f};
-                    if (kMaxNTiles > 1 && nt > 1) {
+                for (int j = 0; j < kMaxNTiles; ++j)
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const int tok = otok[kMaxNTiles - 1][h];
-                            if (tok >= 0 && okA) y1[h] = a.Y[(size_t)tok * a.d_out + colA];
-                            if (tok >= 0 && okB) y1[2 + h] = a.Y[(size_t)tok * a.d_out + colB];
-                        }
-                    }
-                    float d[kMaxNTiles][4];
+                    for (int e2 = 0; e2 < 4; ++e2) d[j][e2] = 0.f;
+                const int b = mt >> 2, ms = mt & 3;
+                const int krow = li + 8 * (lj >> 1);
+#pragma unroll 1
+                for (int p = 0; p < np; ++p) {
+                    uint32_t af[4];
+                    ldsm_x4_t(sb + (uint32_t)((p * g.nb + b) * kBoxBytes + krow * 128 + (((2 * ms + (lj & 1)) ^ li) << 4)),
+                              af);
 #pragma unroll
-                    for (int j = 0; j < kMaxNTiles; ++j)
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) d[j][e2] = 0.f;
-                    const int b = mt >> 2, ms = mt & 3;
-#pragma unroll
-                    for (int p = 0; p < kMaxPages; ++p) {
-                        if (p < np) {
-                            uint32_t af[4];
-                            const int krow = li + 8 * (lj >> 1);
-                            ldsm_x4_t(sb + (uint32_t)((p * g.nb + b) * kBoxBytes + krow * 128 +
-                                                      (((2 * ms + (lj & 1)) ^ li) << 4)),
-                                      af);
-#pragma unroll
-                            for (int j = 0; j < kMaxNTiles; ++j) {
-                                if (j < nt) {
-                                    uint32_t bv[4];
-                                    ldsm_x4(vbase + swz(j * kNTok + li, LORA_MAX_RANK * 2, 2 * p + (lj & 1)), bv);
-                                    mma_bf16(d[j], af, bv[0], bv[1]);
-                                    mma_bf16(d[j], af, bv[2], bv[3]);
-                                }
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int tok0 = otok[0][h];
-                        if (tok0 >= 0 && okA) a.Y[(size_t)tok0 * a.d_out + colA] = fmaf(sc, d[0][h], ypf[i][h]);
-                        if (tok0 >= 0 && okB) a.Y[(size_t)tok0 * a.d_out + colB] = fmaf(sc, d[0][2 + h], ypf[i][2 + h]);
-                        if (kMaxNTiles > 1) {
-                            const int tok1 = otok[kMaxNTiles - 1][h];
-                            if (tok1 >= 0 && okA)
-                                a.Y[(size_t)tok1 * a.d_out + colA] = fmaf(sc, d[kMaxNTiles - 1][h], y1[h]);
-                            if (tok1 >= 0 && okB)
-                                a.Y[(size_t)tok1 * a.d_out + colB] = fmaf(sc, d[kMaxNTiles - 1][2 + h], y1[2 + h]);
+                    for (int j = 0; j < kMaxNTiles; ++j) {
+                        if (j < nt) {
+                            uint32_t bv[4];
+                            ldsm_x4(vbase + swz(j * kNTok + li, LORA_MAX_RANK * 2, 2 * p + (lj & 1)), bv);
+                            mma_bf16(d[j], af, bv[0], bv[1]);
+                            mma_bf16(d[j], af, bv[2], bv[3]);
                         }
                     }
                 }
-                if (c + 1 < g.n_expand) load_y(c + 1, i);   // this slot's tile of the next chunk
+                // fragments (column g8 / g8 + 8, tokens 2 tig, 2 tig + 1) -> rows:
+                // tile [token][16 columns], 4-column groups swizzled by token
+#pragma unroll
+                for (int j = 0; j < kMaxNTiles; ++j) {
+                    if (j < nt) {
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            const int t = j * kNTok + 2 * tig + (e2 & 1), cc = g8 + 8 * (e2 >> 1);
+                            ytile[t * 16 + (((cc >> 2) ^ (t & 3)) << 2) + (cc & 3)] = d[j][e2];
+                        }
+                    }
+                }
+                __syncwarp();
+#pragma unroll
+                for (int j = 0; j < kMaxNTiles; ++j) {
+                    const int t = j * kNTok + rt;
+                    const int tok = rtok[j];
+                    if (j < nt && tok >= 0 && ok) {
+                        const float4 dv = *reinterpret_cast<const float4 *>(ytile + t * 16 + ((rc ^ (t & 3)) << 2));
+                        const float4 y = (j == 0) ? ya : y1;
+                        *reinterpret_cast<float4 *>(a.Y + (size_t)tok * a.d_out + col) =
+                            make_float4(fmaf(sc, dv.x, y.x), fmaf(sc, dv.y, y.y), fmaf(sc, dv.z, y.z), fmaf(sc, dv.w, y.w));
+                    }
+                }
+                __syncwarp();   // the tile is rewritten for the next column tile
+                ya = yb;
+                yb = yc;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive_relaxed(&sm.empty[s]);

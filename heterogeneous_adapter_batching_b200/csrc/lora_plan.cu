@@ -77,6 +77,14 @@ __device__ __forceinline__ bool valid_id(int id, int S, const int32_t *ranks) {
 }
 
 // A break: token t starts a run of one slot, or has no valid adapter.
+// Gather jobs are ordered by rank class: 0 = 4 pages per matrix (rank 49-64;
+// an out-of-range rank counts here too), 1 = 3 pages, 2 = 2, 3 = 1 page.
+constexpr int kPlanRankClasses = 4;
+__device__ __forceinline__ int rank_class(int r) {
+    const int np = (r + LORA_PAGE_ROWS - 1) / LORA_PAGE_ROWS;
+    return np >= 4 ? 0 : (np <= 1 ? 3 : 4 - np);
+}
+
 __device__ __forceinline__ bool is_break(const int32_t *ids, int t, int id, bool ok) {
     return !ok || t == 0 || ids[t - 1] != id;
 }
@@ -295,34 +303,52 @@ plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ 
                 if (cand[i] <= job_tokens && s_total[6 + i] >= want) jt = cand[i];
             job_tokens = jt;
         }
-        int sh_local = 0, nj_local = 0, ns_local = 0;
+        // Jobs are written heaviest first: by pages per matrix (4, 3, 2, 1),
+        // then slot order.  The gather kernel hands units to clusters round
+        // robin, so this order places the long units first and the short ones
+        // fill in after them.
+        int sh_local = 0, ns_local = 0;
+        int njp[kPlanRankClasses] = {0, 0, 0, 0};
         for (int k = k0; k < k1; ++k) {
             const int c = scnt[k];
             sh_local += c;
-            if (c > 0) nj_local += (c + job_tokens - 1) / job_tokens;
+            if (c > 0) njp[rank_class(ranks[k])] += (c + job_tokens - 1) / job_tokens;
             if (out.seg_start[k + 1] > out.seg_start[k]) ++ns_local;
         }
         int sh_off = block_exclusive_scan(sh_local, warp_tot, &s_total[2]);
-        int j_off = block_exclusive_scan(nj_local, warp_tot, &s_total[3]);
+        int j_off[kPlanRankClasses];
+#pragma unroll
+        for (int i = 0; i < kPlanRankClasses; ++i) j_off[i] = block_exclusive_scan(njp[i], warp_tot, &s_total[6 + i]);
         (void)block_exclusive_scan(ns_local, warp_tot, &s_total[4]);
+        {
+            int base = 0;   // classes in order 0 (heaviest) .. 3
+#pragma unroll
+            for (int i = 0; i < kPlanRankClasses; ++i) {
+                j_off[i] += base;
+                base += s_total[6 + i];
+            }
+            if (tid == 0) s_total[3] = base;
+        }
         for (int k = k0; k < k1; ++k) {
             const int c = scnt[k];
             if (c > 0) {
                 const int nj = (c + job_tokens - 1) / job_tokens;
                 const int b = c / nj, rem = c % nj;
+                int &jo = j_off[rank_class(ranks[k])];
                 for (int j = 0; j < nj; ++j) {
                     const int cc = b + (j < rem ? 1 : 0);
                     const int q0 = sh_off + j * b + min(j, rem);
                     int tk[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) tk[i] = i < cc ? out.perm_short[q0 + i] : -1;
-                    out.jobs[2 * (j_off + j)] = make_int4(k, cc, q0, 0);
-                    out.jobs[2 * (j_off + j) + 1] = make_int4(tk[0], tk[1], tk[2], tk[3]);
+                    out.jobs[2 * (jo + j)] = make_int4(k, cc, q0, 0);
+                    out.jobs[2 * (jo + j) + 1] = make_int4(tk[0], tk[1], tk[2], tk[3]);
                 }
-                j_off += nj;
+                jo += nj;
             }
             sh_off += c;
         }
+        __syncthreads();   // s_total[3] (the job count) is read below
         // a token starts a tile when it lies in a long run at a multiple of kTileM
         // from the run's start
         int nt_local = 0;
