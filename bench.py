@@ -46,6 +46,8 @@ def parse():
     p.add_argument("--workload", default="decode_q_proj_7b",
                    help="decode_q_proj_7b | mixed_mlp_up | mixed_mlp_down | prefill | sweep_8b_one_T<n> | sweep_8b_distinct_T<n>")
     p.add_argument("--layers", type=int, default=0, help="ring size (0 = enough for > 4x L2)")
+    p.add_argument("--projections", type=int, default=1,
+                   help="layers that share one X and one launch (lora_apply_multi_planned), e.g. 3 for q/k/v")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -261,6 +263,28 @@ class Ring:
             n += self.H.lora_last_launch_count()
         return n
 
+    def step_groups(self, P: int, stream=None, plan: bool = True) -> int:
+        """Plan once, then one lora_apply_multi_planned per group of P layers that
+        read the same X (the group's first); returns the number of kernels launched."""
+        H = self.H
+        n = 0
+        if plan:
+            self.layers[0].plan(self.ids, ws=self.ws, stream=stream)
+            n += H.lora_last_launch_count()
+        for g in range(0, len(self.layers), P):
+            H.apply_multi(self.layers[g:g + P], self.X[g], self.Y[g:g + P], None, ws=self.ws, stream=stream)
+            n += H.lora_last_launch_count()
+        return n
+
+    def step_groups_separate(self, P: int, stream=None) -> int:
+        """The same work as step_groups(plan=False) with one launch per layer."""
+        n = 0
+        for g in range(0, len(self.layers), P):
+            for lay, Y in zip(self.layers[g:g + P], self.Y[g:g + P]):
+                lay.apply_planned(self.X[g], Y, ws=self.ws, stream=stream)
+                n += self.H.lora_last_launch_count()
+        return n
+
 
 PROFILE_FOR = {
     # workload -> (profile summary, kernel source it was captured from)
@@ -324,18 +348,21 @@ def run_gpu(args):
     wl, desc = workload_spec(args.workload)
     per_layer = (wl.pages_a * 16 * wl.d_in * 2 + wl.pages_b * 16 * wl.d_out * 2 + wl.T * (wl.d_in * 2 + wl.d_out * 4))
     n_layers = args.layers or max(8, min(256, math.ceil(4.2 * L2_BYTES / per_layer)))
+    P = max(1, args.projections)
+    n_layers = (n_layers + P - 1) // P * P
     ring = Ring(wl, n_layers, seed=1234 + rank, device=dev)
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
     # capture one step in a CUDA graph
+    step = ring.step if P == 1 else (lambda s: ring.step_groups(P, s))
     with torch.cuda.stream(stream):
         for _ in range(2):
-            ring.step(stream)
+            step(stream)
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
-        launches_per_step = ring.step(stream)
+        launches_per_step = step(stream)
     graph.replay()
     torch.cuda.synchronize()
     n_valid, n_seg, n_jobs, n_tiles = (int(x) for x in ring.ws[:16].cpu().numpy().view(np.int32)[:4])
@@ -348,7 +375,12 @@ def run_gpu(args):
         ring.layers[0].plan(ring.ids, ws=ring.ws, stream=stream)
     graph_apply = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph_apply, stream=stream):
-        apply_launches = ring.apply_only(stream)
+        apply_launches = ring.apply_only(stream) if P == 1 else ring.step_groups(P, stream, plan=False)
+    graph_sep = None
+    if P > 1:
+        graph_sep = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_sep, stream=stream):
+            ring.step_groups_separate(P, stream)
     H.lora_set_option(H.OPT_LONG_SEGMENT, old_thresh)
     torch.cuda.synchronize()
 
@@ -381,6 +413,16 @@ def run_gpu(args):
     a1.record(cur)
     torch.cuda.synchronize()
     apply_ms = a0.elapsed_time(a1)
+    sep_ms = None
+    if graph_sep is not None:
+        for _ in range(3):
+            graph_sep.replay()
+        a0.record(cur)
+        for _ in range(k_apply):
+            graph_sep.replay()
+        a1.record(cur)
+        torch.cuda.synchronize()
+        sep_ms = a0.elapsed_time(a1)
     clk = clocks.stop()
     if world > 1:
         t = torch.tensor([elapsed_ms], device=dev)
@@ -393,16 +435,16 @@ def run_gpu(args):
     value = tokens_per_step * world * args.steps / (elapsed_ms / 1000.0)
     ms_per_step = elapsed_ms / args.steps
 
-    # roofline of the gather kernel (one launch = one layer)
-    per_launch_ms = apply_ms / (k_apply * n_layers)
-    alg = algorithmic_bytes(wl)
+    # roofline of the gather kernel (one launch = one layer, or one group of P layers)
+    per_launch_ms = apply_ms / (k_apply * (n_layers // P))
+    alg = algorithmic_bytes(wl) * P
     achieved = alg / (per_launch_ms / 1000.0) / 1e9
     peak, peak_kind = measured_peaks()
     kname = "gather_kernel<apply>" if n_tiles == 0 else "gather_kernel<apply> + tiles_kernel"
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
             "traffic": profiled_traffic(args.workload), "peak_source": peak_kind, "kernel": kname,
             "kernel_us": per_launch_ms * 1000.0, "algorithmic_bytes_per_launch": alg,
-            "launches_per_layer": apply_launches // n_layers}
+            "launches_per_layer": apply_launches / n_layers}
 
     # end-to-end through the C ABI with host buffers (one layer per step)
     e2e = None
@@ -461,12 +503,17 @@ def run_gpu(args):
                        "l2": f"inputs larger than L2: ring of {n_layers} layer instances, "
                              f"{ring.footprint() / 1e6:.0f} MB > 4 x 126 MB",
                        "cuda_graph": True, "parallelism": f"replicas x{world} (no collective)"},
+
             "gpu_launches": int(launches_per_step * args.steps),
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "clocks": clk,
         }
+        if P > 1:
+            line["config"]["projections_per_launch"] = P
+            line["config"]["us_per_layer_one_launch_per_group"] = apply_ms * 1000.0 / (k_apply * n_layers)
+            line["config"]["us_per_layer_one_launch_per_layer"] = sep_ms * 1000.0 / (k_apply * n_layers)
         print(json.dumps(line), flush=True)
     return 0
 

@@ -34,13 +34,23 @@ OPT_LONG_SEGMENT = 1
 OPT_DECODE_JOB_TOKENS = 2
 NOALLOC_MAX_TOKENS = 32768
 NOALLOC_SCRATCH_BYTES = 2097152
+MAX_JOB_TOKENS = 16
+MAX_PROJECTIONS = 8
 
 EXPORTS = [
     "lora_pool_create", "lora_pool_destroy", "lora_pool_free_pages", "lora_pool_num_pages",
     "lora_pool_load", "lora_pool_evict", "lora_pool_read_row", "lora_workspace_size",
     "lora_plan", "lora_shrink", "lora_expand_add", "lora_apply", "lora_apply_planned", "lora_apply_noalloc",
+    "lora_apply_multi", "lora_apply_multi_planned",
     "lora_set_option", "lora_get_option", "lora_last_cuda_error", "lora_last_launch_count",
 ]
+
+
+class LoraProjection(ctypes.Structure):
+    """lora_projection_t: one projection of lora_apply_multi."""
+    _fields_ = [("Y", ctypes.c_void_p), ("d_out", ctypes.c_int), ("ranks", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("page_table", ctypes.c_void_p), ("pa", ctypes.c_void_p),
+                ("pb", ctypes.c_void_p)]
 
 
 class LoraError(RuntimeError):
@@ -79,6 +89,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lora_apply": (I, [V, V, I, I, I, V, I, V, V, V, V, V, V, Z, V, V]),
         "lora_apply_planned": (I, [V, V, I, I, I, I, V, V, V, V, V, V, Z, V, V]),
         "lora_apply_noalloc": (I, [V, V, I, I, I, V, I, V, V, V, V, V, V, V]),
+        "lora_apply_multi": (I, [V, I, I, V, I, ctypes.POINTER(LoraProjection), I, V, Z, V, V]),
+        "lora_apply_multi_planned": (I, [V, I, I, I, ctypes.POINTER(LoraProjection), I, V, Z, V, V]),
         "lora_set_option": (I, [I, I]),
         "lora_get_option": (I, [I]),
         "lora_last_cuda_error": (ctypes.c_char_p, []),
@@ -223,6 +235,27 @@ def lora_apply_noalloc(X, Y, T, d_in, d_out, ids, num_slots, ranks, scales, page
     _check("lora_apply_noalloc", load_library().lora_apply_noalloc(
         _p(X), _p(Y), T, d_in, d_out, _p(ids), num_slots, _p(ranks), _p(scales), _p(page_table),
         pa._h, pb._h, _p(err), _s(stream)))
+
+
+def _proj_array(projs):
+    arr = (LoraProjection * len(projs))()
+    for i, (Y, d_out, ranks, scales, page_table, pa, pb) in enumerate(projs):
+        arr[i] = LoraProjection(Y.data_ptr(), d_out, ranks.data_ptr(), scales.data_ptr(), page_table.data_ptr(),
+                                pa.handle, pb.handle)
+    return arr
+
+
+def lora_apply_multi(X, T, d_in, ids, num_slots, projs, ws, err=None, stream=None) -> None:
+    """projs: sequence of (Y, d_out, ranks, scales, page_table, pa: Pool, pb: Pool)."""
+    _check("lora_apply_multi", load_library().lora_apply_multi(
+        _p(X), T, d_in, _p(ids), num_slots, _proj_array(projs), len(projs), _p(ws), ws.numel() * ws.element_size(),
+        _p(err), _s(stream)))
+
+
+def lora_apply_multi_planned(X, T, d_in, num_slots, projs, ws, err=None, stream=None) -> None:
+    _check("lora_apply_multi_planned", load_library().lora_apply_multi_planned(
+        _p(X), T, d_in, num_slots, _proj_array(projs), len(projs), _p(ws), ws.numel() * ws.element_size(),
+        _p(err), _s(stream)))
 
 
 def lora_set_option(key: int, value: int) -> None:

@@ -265,25 +265,48 @@ static bool plan_uses_tiles(int T) {
     return tiles_supported() && opt_long_segment() > 0 && T >= opt_long_segment();
 }
 
-static int run_planned(const uint16_t *X, float *Y, int T, int d_in, int d_out, int num_slots,
-                       const int32_t *ranks, const float *scales, const int32_t *page_table, lora_pool_t pa,
-                       lora_pool_t pb, void *ws, int32_t *err_dev, cudaStream_t st) {
+static GatherProj gather_proj(float *Y, int d_out, const int32_t *ranks, const float *scales,
+                              const int32_t *page_table, const lora_pool_s *pa, const lora_pool_s *pb) {
+    GatherProj g = {};
+    g.Y = Y; g.d_out = d_out; g.ranks = ranks; g.scales = scales; g.pt = page_table;
+    g.rowsA = pa ? (long long)pa->num_pages * LORA_PAGE_ROWS : 0;
+    g.rowsB = pb ? (long long)pb->num_pages * LORA_PAGE_ROWS : 0;
+    return g;
+}
+
+// The apply kernels over a plan already in ws: one gather launch for every
+// projection, then (when the plan has long runs) one tile launch per projection.
+static int run_planned(const uint16_t *X, int T, int d_in, int num_slots, const lora_projection_t *pr, int nproj,
+                       void *ws, int32_t *err_dev, cudaStream_t st) {
     const PlanOut o = plan_out(ws, T, num_slots, nullptr, nullptr);
     GatherArgs a = {};
-    a.X = X; a.Y = Y; a.T = T; a.d_in = d_in; a.d_out = d_out; a.S = num_slots;
-    a.ranks = ranks; a.scales = scales; a.pt = page_table; a.poolA = pa->base; a.poolB = pb->base;
+    a.X = X; a.T = T; a.d_in = d_in; a.S = num_slots; a.nproj = nproj;
+    lora_pool_s *pa[LORA_MAX_PROJECTIONS], *pb[LORA_MAX_PROJECTIONS];
+    for (int p = 0; p < nproj; ++p) {
+        a.proj[p] = gather_proj(pr[p].Y, pr[p].d_out, pr[p].ranks, pr[p].scales, pr[p].page_table, pr[p].pa, pr[p].pb);
+        pa[p] = pr[p].pa;
+        pb[p] = pr[p].pb;
+    }
     a.perm = o.perm_short; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
-    a.rowsA = (long long)pa->num_pages * LORA_PAGE_ROWS; a.rowsB = (long long)pb->num_pages * LORA_PAGE_ROWS;
     if (int rc = launch_gather(kApply, a, pa, pb, st, true)) return rc;
     if (plan_uses_tiles(T)) {
-        TileArgs ta = {};
-        ta.X = X; ta.Y = Y; ta.T = T; ta.d_in = d_in; ta.d_out = d_out;
-        ta.ranks = ranks; ta.scales = scales; ta.pt = page_table; ta.pa = pa; ta.pb = pb;
-        ta.tiles = o.tiles; ta.hdr = o.header; ta.err = err_dev;
-        ta.rowsA = a.rowsA; ta.rowsB = a.rowsB; ta.long_thresh = opt_long_segment();
-        if (int rc = launch_tiles(ta, st, true)) return rc;
+        for (int p = 0; p < nproj; ++p) {
+            TileArgs ta = {};
+            ta.X = X; ta.Y = pr[p].Y; ta.T = T; ta.d_in = d_in; ta.d_out = pr[p].d_out;
+            ta.ranks = pr[p].ranks; ta.scales = pr[p].scales; ta.pt = pr[p].page_table; ta.pa = pr[p].pa;
+            ta.pb = pr[p].pb; ta.tiles = o.tiles; ta.hdr = o.header; ta.err = err_dev;
+            ta.rowsA = a.proj[p].rowsA; ta.rowsB = a.proj[p].rowsB; ta.long_thresh = opt_long_segment();
+            if (int rc = launch_tiles(ta, st, true)) return rc;
+        }
     }
     return LORA_OK;
+}
+
+static lora_projection_t one_proj(float *Y, int d_out, const int32_t *ranks, const float *scales,
+                                  const int32_t *page_table, lora_pool_t pa, lora_pool_t pb) {
+    lora_projection_t p;
+    p.Y = Y; p.d_out = d_out; p.ranks = ranks; p.scales = scales; p.page_table = page_table; p.pa = pa; p.pb = pb;
+    return p;
 }
 
 int lora_plan(const int32_t *ids, int T, const int32_t *ranks, int num_slots, int32_t *perm_out,
@@ -305,8 +328,8 @@ int lora_apply_planned(const uint16_t *X, float *Y, int T, int d_in, int d_out, 
     if (pa->width != d_in || pb->width != d_out) return LORA_ERR_WIDTH_MISMATCH;
     if (T == 0) return LORA_OK;
     if (!X || !Y || !scales || !page_table || !aligned(X, 16) || !aligned(Y, 16)) return LORA_ERR_INVALID_ARG;
-    return run_planned(X, Y, T, d_in, d_out, num_slots, ranks, scales, page_table, pa, pb, ws, err_dev,
-                       reinterpret_cast<cudaStream_t>(stream));
+    const lora_projection_t pr = one_proj(Y, d_out, ranks, scales, page_table, pa, pb);
+    return run_planned(X, T, d_in, num_slots, &pr, 1, ws, err_dev, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int lora_shrink(const uint16_t *X, int T, int d_in, const int32_t *ids, int num_slots, const int32_t *ranks,
@@ -322,11 +345,11 @@ int lora_shrink(const uint16_t *X, int T, int d_in, const int32_t *ids, int num_
     const PlanOut o = plan_out(ws, T, num_slots, nullptr, nullptr);
     if (int rc = launch_plan(ids, T, ranks, num_slots, 0, opt_job_tokens(), o, err_dev, st)) return rc;
     GatherArgs a = {};
-    a.X = X; a.V = V; a.T = T; a.d_in = d_in; a.d_out = 8; a.S = num_slots;
-    a.ranks = ranks; a.pt = page_table; a.poolA = pa->base;
+    a.X = X; a.V = V; a.T = T; a.d_in = d_in; a.S = num_slots; a.nproj = 1;
+    a.proj[0] = gather_proj(nullptr, 8, ranks, nullptr, page_table, pa, nullptr);
     a.perm = o.perm_short; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
-    a.rowsA = (long long)pa->num_pages * LORA_PAGE_ROWS;
-    return launch_gather(kShrink, a, pa, pa, st, true);
+    lora_pool_s *pp[1] = {pa};
+    return launch_gather(kShrink, a, pp, pp, st, true);
 }
 
 int lora_expand_add(const float *V, float *Y, int T, int d_out, const int32_t *ids, int num_slots,
@@ -342,11 +365,11 @@ int lora_expand_add(const float *V, float *Y, int T, int d_out, const int32_t *i
     const PlanOut o = plan_out(ws, T, num_slots, nullptr, nullptr);
     if (int rc = launch_plan(ids, T, ranks, num_slots, 0, opt_job_tokens(), o, err_dev, st)) return rc;
     GatherArgs a = {};
-    a.V = const_cast<float *>(V); a.Y = Y; a.T = T; a.d_in = 8; a.d_out = d_out; a.S = num_slots;
-    a.ranks = ranks; a.scales = scales; a.pt = page_table; a.poolB = pb->base;
+    a.V = const_cast<float *>(V); a.T = T; a.d_in = 8; a.S = num_slots; a.nproj = 1;
+    a.proj[0] = gather_proj(Y, d_out, ranks, scales, page_table, nullptr, pb);
     a.perm = o.perm_short; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
-    a.rowsB = (long long)pb->num_pages * LORA_PAGE_ROWS;
-    return launch_gather(kExpand, a, pb, pb, st, true);
+    lora_pool_s *pp[1] = {pb};
+    return launch_gather(kExpand, a, pp, pp, st, true);
 }
 
 int lora_apply(const uint16_t *X, float *Y, int T, int d_in, int d_out, const int32_t *ids, int num_slots,
@@ -362,7 +385,53 @@ int lora_apply(const uint16_t *X, float *Y, int T, int d_in, int d_out, const in
     const PlanOut o = plan_out(ws, T, num_slots, nullptr, nullptr);
     const int long_thresh = plan_uses_tiles(T) ? opt_long_segment() : 0;
     if (int rc = launch_plan(ids, T, ranks, num_slots, long_thresh, opt_job_tokens(), o, err_dev, st)) return rc;
-    return run_planned(X, Y, T, d_in, d_out, num_slots, ranks, scales, page_table, pa, pb, ws, err_dev, st);
+    const lora_projection_t pr = one_proj(Y, d_out, ranks, scales, page_table, pa, pb);
+    return run_planned(X, T, d_in, num_slots, &pr, 1, ws, err_dev, st);
+}
+
+// Checks of the projection list shared by the two multi-projection calls
+// (the sizes, ids and workspace are checked by the caller).
+static int check_projs(const uint16_t *X, int T, int d_in, const lora_projection_t *projs, int num_projs) {
+    for (int p = 0; p < num_projs; ++p) {
+        const lora_projection_t &q = projs[p];
+        if (!q.pa || !q.pb || !q.ranks) return LORA_ERR_INVALID_ARG;
+        if (q.pa->width != d_in || q.pb->width != q.d_out) return LORA_ERR_WIDTH_MISMATCH;
+    }
+    if (T == 0) return LORA_OK;
+    if (!X || !aligned(X, 16)) return LORA_ERR_INVALID_ARG;
+    for (int p = 0; p < num_projs; ++p) {
+        const lora_projection_t &q = projs[p];
+        if (!q.Y || !q.scales || !q.page_table || !aligned(q.Y, 16)) return LORA_ERR_INVALID_ARG;
+    }
+    return LORA_OK;
+}
+
+int lora_apply_multi_planned(const uint16_t *X, int T, int d_in, int num_slots, const lora_projection_t *projs,
+                             int num_projs, void *ws, size_t ws_bytes, int32_t *err_dev, lora_stream_t stream) {
+    reset_launch_count();
+    if (!projs || num_projs < 1 || num_projs > LORA_MAX_PROJECTIONS) return LORA_ERR_INVALID_ARG;
+    if (T < 0 || num_slots < 1 || num_slots > LORA_MAX_SLOTS) return LORA_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < ws_layout(T, num_slots).total || !aligned(ws, 256)) return LORA_ERR_WORKSPACE;
+    if (int rc = check_projs(X, T, d_in, projs, num_projs)) return rc;
+    if (T == 0) return LORA_OK;
+    return run_planned(X, T, d_in, num_slots, projs, num_projs, ws, err_dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int lora_apply_multi(const uint16_t *X, int T, int d_in, const int32_t *ids, int num_slots,
+                     const lora_projection_t *projs, int num_projs, void *ws, size_t ws_bytes, int32_t *err_dev,
+                     lora_stream_t stream) {
+    reset_launch_count();
+    if (!projs || num_projs < 1 || num_projs > LORA_MAX_PROJECTIONS) return LORA_ERR_INVALID_ARG;
+    if (int rc = check_common(T, num_slots, ids, projs[0].ranks, ws, ws_bytes)) return rc;
+    if (int rc = check_projs(X, T, d_in, projs, num_projs)) return rc;
+    if (T == 0) return LORA_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const PlanOut o = plan_out(ws, T, num_slots, nullptr, nullptr);
+    const int long_thresh = plan_uses_tiles(T) ? opt_long_segment() : 0;
+    if (int rc = launch_plan(ids, T, projs[0].ranks, num_slots, long_thresh, opt_job_tokens(), o, err_dev, st,
+                             num_projs))
+        return rc;
+    return run_planned(X, T, d_in, num_slots, projs, num_projs, ws, err_dev, st);
 }
 
 int lora_set_option(int key, int value) {

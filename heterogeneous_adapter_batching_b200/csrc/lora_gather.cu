@@ -93,11 +93,35 @@ struct __align__(1024) GatherSmem {
     int4 pt[kTableSlots * 2];                         // staged page-table rows (A pages, B pages)
     int ranks[kTableSlots];
     float scales[kTableSlots];
-    int ebound[kMaxSplit + 1];                        // d_out split: first 8-column group of part e
+    int ebound[LORA_MAX_PROJECTIONS][kMaxSplit + 1];  // d_out split: first 8-column group of part e
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t rbar[2];
     int abort;
+};
+
+static_assert(sizeof(GatherSmem) + 1024 <= 227 * 1024, "shared memory beyond the per-block limit");
+
+// Kernel parameters for launches of up to NP projections: single-projection
+// launches pass one record and one pair of TMA descriptors, not the maximum.
+template <int NP>
+struct GatherMaps {
+    CUtensorMap A[NP];
+    CUtensorMap B[NP];
+};
+
+template <int NP>
+struct KArgs {
+    const uint16_t *X;
+    float *V;
+    int T, d_in;
+    int S;
+    int nproj;
+    GatherProj proj[NP];
+    const int32_t *perm;
+    const int4 *jobs;
+    const PlanHeader *hdr;
+    int32_t *err;
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -237,20 +261,23 @@ struct SlotMeta {
     bool bad;
 };
 
-template <int MODE>
-__device__ __forceinline__ SlotMeta slot_meta(const GatherArgs &a, const GatherSmem &sm, bool staged, int slot) {
+template <int MODE, class Args>
+__device__ __forceinline__ SlotMeta slot_meta(const Args &a, const GatherSmem &sm, bool staged, int pj,
+                                              int slot) {
     SlotMeta m;
     int r;
+    const GatherProj &pr = a.proj[pj];
     if (staged) {
-        r = sm.ranks[slot];
-        m.pga = sm.pt[2 * slot];
-        m.pgb = sm.pt[2 * slot + 1];
-        m.scale = sm.scales[slot];
+        const int i = pj * a.S + slot;
+        r = sm.ranks[i];
+        m.pga = sm.pt[2 * i];
+        m.pgb = sm.pt[2 * i + 1];
+        m.scale = sm.scales[i];
     } else {
-        r = a.ranks[slot];
-        m.pga = reinterpret_cast<const int4 *>(a.pt)[2 * slot];
-        m.pgb = reinterpret_cast<const int4 *>(a.pt)[2 * slot + 1];
-        m.scale = (MODE == kShrink) ? 0.f : a.scales[slot];
+        r = pr.ranks[slot];
+        m.pga = reinterpret_cast<const int4 *>(pr.pt)[2 * slot];
+        m.pgb = reinterpret_cast<const int4 *>(pr.pt)[2 * slot + 1];
+        m.scale = (MODE == kShrink) ? 0.f : pr.scales[slot];
     }
     m.bad = r > LORA_MAX_RANK;
     if (r <= 0 || m.bad) r = 0;
@@ -260,8 +287,8 @@ __device__ __forceinline__ SlotMeta slot_meta(const GatherArgs &a, const GatherS
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
         if (p < np) {
-            if (MODE != kExpand && (pa[p] < 0 || (long long)(pa[p] + 1) * LORA_PAGE_ROWS > a.rowsA)) m.bad = true;
-            if (MODE != kShrink && (pb[p] < 0 || (long long)(pb[p] + 1) * LORA_PAGE_ROWS > a.rowsB)) m.bad = true;
+            if (MODE != kExpand && (pa[p] < 0 || (long long)(pa[p] + 1) * LORA_PAGE_ROWS > pr.rowsA)) m.bad = true;
+            if (MODE != kShrink && (pb[p] < 0 || (long long)(pb[p] + 1) * LORA_PAGE_ROWS > pr.rowsB)) m.bad = true;
         }
     }
     m.r = m.bad ? 0 : r;
@@ -277,14 +304,15 @@ struct UnitGeom {
     int n_shrink, n_expand;
 };
 
-template <int MODE>
-__device__ __forceinline__ UnitGeom unit_geom(const GatherArgs &a, const GatherSmem &sm, int np, int e, int crank) {
+template <int MODE, class Args>
+__device__ __forceinline__ UnitGeom unit_geom(const Args &a, const GatherSmem &sm, int pj, int np, int e,
+                                              int crank) {
     UnitGeom g;
     // 32-bit arithmetic: column groups fit easily (d <= 2^24 checked on the host)
     const unsigned Gi = (unsigned)a.d_in >> 3;
     g.in0 = 8 * (int)(Gi * crank / kCS);
     g.in1 = 8 * (int)(Gi * (crank + 1) / kCS);
-    const unsigned ge0 = (unsigned)sm.ebound[e], ge1 = (unsigned)sm.ebound[e + 1];
+    const unsigned ge0 = (unsigned)sm.ebound[pj][e], ge1 = (unsigned)sm.ebound[pj][e + 1];
     g.out0 = 8 * (int)(ge0 + (ge1 - ge0) * crank / kCS);
     g.out1 = 8 * (int)(ge0 + (ge1 - ge0) * (crank + 1) / kCS);
     // As many boxes per page as fit in a stage: the chunk width depends on the
@@ -311,22 +339,23 @@ __device__ __forceinline__ int ld_s32_now(const int *p) {
 
 // Token index t of a job: the first four are in the job record, the rest
 // in the plan's slot-ordered token list.  -1 past the job's end.
-__device__ __forceinline__ int job_token(const GatherArgs &a, const int4 &tk, int q0, int n, int t) {
+template <class Args>
+__device__ __forceinline__ int job_token(const Args &a, const int4 &tk, int q0, int n, int t) {
     if (t >= n) return -1;
     if (t < 4) return t == 0 ? tk.x : t == 1 ? tk.y : t == 2 ? tk.z : tk.w;
     return __ldg(a.perm + q0 + t);
 }
 
-template <int MODE>
+template <int MODE, int NP>
 __global__ void __launch_bounds__(kThreads, 1)
-gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GatherArgs a,
-              int e_max) {
+gather_kernel(const __grid_constant__ GatherMaps<NP> maps, const __grid_constant__ KArgs<NP> a, int e_max) {
     extern __shared__ unsigned char smem_raw[];
     GatherSmem &sm = *reinterpret_cast<GatherSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int crank = (int)cluster_rank();
     const int cluster_id = blockIdx.x / kCS;
     const int n_clusters = gridDim.x / kCS;
+    const int nproj = (NP == 1) ? 1 : a.nproj;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -348,25 +377,31 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     // Every launch's parameters sit in memory this SM has not read yet: fetch
     // them and both tensor maps now, while the previous kernel drains, rather
     // than on first use.
-    if (threadIdx.x == kConsumers) {
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+    if (warp == kConsumerWarps && lane < 2 * nproj) {
+        const CUtensorMap *m = (lane & 1) ? &maps.B[lane >> 1] : &maps.A[lane >> 1];
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
     }
-    asm volatile("" ::"l"(a.X), "l"(a.Y), "l"(a.V), "r"(a.T), "r"(a.d_in), "r"(a.d_out), "r"(a.S), "l"(a.ranks),
-                 "l"(a.scales), "l"(a.pt), "l"(a.perm), "l"(a.jobs), "l"(a.hdr), "l"(a.err), "l"(a.rowsA),
-                 "l"(a.rowsB), "r"(e_max));
+    asm volatile("" ::"l"(a.X), "l"(a.V), "r"(a.T), "r"(a.d_in), "r"(a.S), "r"(nproj), "l"(a.perm), "l"(a.jobs),
+                 "l"(a.hdr), "l"(a.err), "r"(e_max));
+    if (threadIdx.x < nproj) {
+        const GatherProj &pr = a.proj[threadIdx.x];
+        asm volatile("" ::"l"(pr.Y), "r"(pr.d_out), "l"(pr.ranks), "l"(pr.scales), "l"(pr.pt), "l"(pr.rowsA),
+                     "l"(pr.rowsB));
+    }
     // Small page tables, ranks and scales are staged in shared memory.  They
     // are the caller's slot state, not the plan's output, so they are read
     // before this kernel waits for the kernels ahead of it (the library's own
     // kernels, the only ones here that let a dependent start early, never
     // write them).
-    const bool staged = a.S <= kTableSlots;
+    const bool staged = nproj * a.S <= kTableSlots;
     if (staged) {
-        for (int i = threadIdx.x; i < a.S; i += kThreads) {
-            sm.pt[2 * i] = reinterpret_cast<const int4 *>(a.pt)[2 * i];
-            sm.pt[2 * i + 1] = reinterpret_cast<const int4 *>(a.pt)[2 * i + 1];
-            sm.ranks[i] = a.ranks[i];
-            sm.scales[i] = (MODE == kShrink) ? 0.f : a.scales[i];
+        for (int i = threadIdx.x; i < nproj * a.S; i += kThreads) {
+            const int pj = i / a.S, k = i - pj * a.S;
+            const GatherProj &pr = a.proj[pj];
+            sm.pt[2 * i] = reinterpret_cast<const int4 *>(pr.pt)[2 * k];
+            sm.pt[2 * i + 1] = reinterpret_cast<const int4 *>(pr.pt)[2 * k + 1];
+            sm.ranks[i] = pr.ranks[k];
+            sm.scales[i] = (MODE == kShrink) ? 0.f : pr.scales[k];
         }
     }
     // The plan kernel runs before this one; wait for its output.  Then let the
@@ -379,24 +414,28 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     // Issue the first job record (a guess that holds whenever there are at
     // least half as many jobs as clusters) and the job count together, so
     // their latencies overlap.
-    const int spec = cluster_id < a.T ? cluster_id : a.T - 1;
+    const int spec = min(cluster_id / nproj, a.T - 1);
     const int4 spec_job = ld_v4_now(a.jobs + 2 * spec);
     const int4 spec_tok = ld_v4_now(a.jobs + 2 * spec + 1);
     const int n_jobs = ld_s32_now(&a.hdr->n_jobs);
     int E = 1;
     if (MODE != kShrink && n_jobs > 0) {
-        E = n_clusters / n_jobs;
+        E = n_clusters / (n_jobs * nproj);
         E = E < 1 ? 1 : (E > e_max ? e_max : E);
         E = E > kMaxSplit ? kMaxSplit : E;
     }
-    // part e of the d_out split starts at 8-column group floor(Go * e / E)
-    if (threadIdx.x <= E) sm.ebound[threadIdx.x] = (int)((long long)(a.d_out >> 3) * threadIdx.x / E);
+    // part e of projection p's d_out split starts at 8-column group floor(Go * e / E)
+    for (int i = threadIdx.x; i < nproj * (E + 1); i += kThreads) {
+        const int pj = i / (E + 1), e = i - pj * (E + 1);
+        sm.ebound[pj][e] = (int)((long long)(a.proj[pj].d_out >> 3) * e / E);
+    }
     __syncthreads();
     if (n_jobs <= 0) {   // uniform over the grid; no peer traffic has happened
         cluster_wait();
         return;
     }
-    const int n_units = n_jobs * E;
+    const int upj = nproj * E;   // units per job: (projection, d_out part)
+    const int n_units = n_jobs * upj;
 
     // Cluster exchange of the shrink partials (apply and shrink modes).
     constexpr bool kXchg = MODE != kExpand;
@@ -408,11 +447,12 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         // ------------------------------------------------------------------
         int chunk = 0;
         for (int u = cluster_id; u < n_units; u += n_clusters) {
-            const int ji = u / E;
+            const int ji = u / upj;
             const int4 job = (ji == spec) ? spec_job : a.jobs[2 * ji];
-            const int e = u - ji * E;
-            const SlotMeta m = slot_meta<MODE>(a, sm, staged, job.x);
-            const UnitGeom g = unit_geom<MODE>(a, sm, m.np, e, crank);
+            const int pj = (NP == 1) ? 0 : (u - ji * upj) / E, e = u - ji * upj - pj * E;
+            const SlotMeta m = slot_meta<MODE>(a, sm, staged, pj, job.x);
+            const UnitGeom g = unit_geom<MODE>(a, sm, pj, m.np, e, crank);
+            const CUtensorMap *tmA = &maps.A[pj], *tmB = &maps.B[pj];
             // Shrink chunks, then expand chunks, in the order the consumers use
             // them; the ring lets the loads run up to kStages chunks ahead,
             // into the next unit.
@@ -429,7 +469,7 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 mbar_expect_tx(&sm.full[s], (uint32_t)(m.np * boxes * kBoxBytes));
                 for (int p = 0; p < m.np; ++p)
                     for (int b = 0; b < boxes; ++b)
-                        tma_load_box(sm.stage[s] + (size_t)(p * g.nb + b) * kBoxBytes, shrink ? &tmA : &tmB,
+                        tma_load_box(sm.stage[s] + (size_t)(p * g.nb + b) * kBoxBytes, shrink ? tmA : tmB,
                                      c0 + b * kBoxCols, (shrink ? pa[p] : pb[p]) * LORA_PAGE_ROWS, &sm.full[s]);
                 ++chunk;
             };
@@ -456,15 +496,17 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     int iter = 0;
     bool joined = false;   // passed the start-up cluster barrier
     for (int u = cluster_id; u < n_units; u += n_clusters, ++iter) {
-        const int ji = u / E;
+        const int ji = u / upj;
         const int4 job = (ji == spec) ? spec_job : a.jobs[2 * ji];
         const int4 tk = (ji == spec) ? spec_tok : a.jobs[2 * ji + 1];
-        const int e = u - ji * E;
+        const int pj = (NP == 1) ? 0 : (u - ji * upj) / E, e = u - ji * upj - pj * E;
         const int slot = job.x, n = min(job.y, kMaxJobTokens), q0 = job.z;
-        const SlotMeta m = slot_meta<MODE>(a, sm, staged, slot);
+        const SlotMeta m = slot_meta<MODE>(a, sm, staged, pj, slot);
         if (m.bad && threadIdx.x == 0 && crank == 0 && e == 0 && a.err) atomicOr(a.err, LORA_DEV_ERR_BAD_PAGE);
         const int r = m.r, np = m.np;
-        const UnitGeom g = unit_geom<MODE>(a, sm, np, e, crank);
+        const UnitGeom g = unit_geom<MODE>(a, sm, pj, np, e, crank);
+        float *const Yp = a.proj[pj].Y;
+        const int d_out = a.proj[pj].d_out;
         const int buf = iter & 1;
         const int cw = g.nb * kBoxCols;
         const int nt = (n + kNTok - 1) / kNTok;   // token tiles of 8
@@ -485,7 +527,7 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         auto load_y = [&](int c0, int mt, int nmt, int j) {
             const int col = c0 + mt * 16 + 4 * rc;
             return (mt < nmt && rtok[j] >= 0 && col < g.out1)
-                       ? *reinterpret_cast<const float4 *>(a.Y + (size_t)rtok[j] * a.d_out + col)
+                       ? *reinterpret_cast<const float4 *>(Yp + (size_t)rtok[j] * d_out + col)
                        : make_float4(0.f, 0.f, 0.f, 0.f);
         };
         float4 ya = make_float4(0.f, 0.f, 0.f, 0.f), yb = ya;   // token tile 0 of this tile and the next
@@ -724,7 +766,7 @@ gather_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                     if (j < nt && tok >= 0 && ok) {
                         const float4 dv = *reinterpret_cast<const float4 *>(ytile + t * 16 + ((rc ^ (t & 3)) << 2));
                         const float4 y = (j == 0) ? ya : y1;
-                        *reinterpret_cast<float4 *>(a.Y + (size_t)tok * a.d_out + col) =
+                        *reinterpret_cast<float4 *>(Yp + (size_t)tok * d_out + col) =
                             make_float4(fmaf(sc, dv.x, y.x), fmaf(sc, dv.y, y.y), fmaf(sc, dv.z, y.z), fmaf(sc, dv.w, y.w));
                     }
                 }
@@ -749,8 +791,9 @@ int max_clusters(int *out) {
     if (int rc = cuda_check(cudaGetDevice(&dev))) return rc;
     if (dev < 0 || dev >= 64) return LORA_ERR_INVALID_ARG;
     if (g_max_clusters[dev] == 0) {
-        const void *fns[3] = {(const void *)gather_kernel<kApply>, (const void *)gather_kernel<kShrink>,
-                              (const void *)gather_kernel<kExpand>};
+        const void *fns[4] = {(const void *)gather_kernel<kApply, 1>, (const void *)gather_kernel<kShrink, 1>,
+                              (const void *)gather_kernel<kExpand, 1>,
+                              (const void *)gather_kernel<kApply, LORA_MAX_PROJECTIONS>};
         for (const void *f : fns)
             if (int rc = cuda_check(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                          (int)kGatherSmemBytes)))
@@ -767,27 +810,42 @@ int max_clusters(int *out) {
         cfg.numAttrs = 1;
         cfg.gridDim = dim3(kCS * 256);
         int ncl = 0;
-        if (int rc = cuda_check(cudaOccupancyMaxActiveClusters(&ncl, gather_kernel<kApply>, &cfg))) return rc;
+        if (int rc = cuda_check(cudaOccupancyMaxActiveClusters(&ncl, gather_kernel<kApply, 1>, &cfg))) return rc;
         g_max_clusters[dev] = ncl > 0 ? ncl : 1;
     }
     *out = g_max_clusters[dev];
     return LORA_OK;
 }
 
-template <int MODE>
-int launch_mode(const GatherArgs &a, lora_pool_s *pa, lora_pool_s *pb, cudaStream_t st, bool pdl) {
+template <int MODE, int NP>
+int launch_mode(const GatherArgs &ga, lora_pool_s *const *pa, lora_pool_s *const *pb, cudaStream_t st, bool pdl) {
+    if (ga.nproj < 1 || ga.nproj > NP) return LORA_ERR_INVALID_ARG;
     int mcl = 1;
     if (int rc = max_clusters(&mcl)) return rc;
     const size_t smem = kGatherSmemBytes;
-    CUtensorMap ma, mb;
-    if (MODE != kExpand) {
-        if (int rc = pool_tensor_map(pa, &ma)) return rc;
+    KArgs<NP> a;
+    a.X = ga.X; a.V = ga.V; a.T = ga.T; a.d_in = ga.d_in; a.S = ga.S; a.nproj = ga.nproj;
+    for (int p = 0; p < NP; ++p) a.proj[p] = ga.proj[p < ga.nproj ? p : 0];
+    a.perm = ga.perm; a.jobs = ga.jobs; a.hdr = ga.hdr; a.err = ga.err;
+    GatherMaps<NP> maps;
+    int e_max = 1 << 30;
+    for (int p = 0; p < a.nproj; ++p) {
+        if (MODE != kExpand) {
+            if (int rc = pool_tensor_map(pa[p], &maps.A[p])) return rc;
+        }
+        if (MODE != kShrink) {
+            if (int rc = pool_tensor_map(pb[p], &maps.B[p])) return rc;
+        }
+        if (MODE == kExpand) maps.A[p] = maps.B[p];
+        if (MODE == kShrink) maps.B[p] = maps.A[p];
+        // a d_out part keeps at least kCS x 8 column groups (8 per CTA)
+        const int em = (a.proj[p].d_out >> 3) / (kCS * 8);
+        e_max = min(e_max, em < 1 ? 1 : em);
     }
-    if (MODE != kShrink) {
-        if (int rc = pool_tensor_map(pb, &mb)) return rc;
+    for (int p = a.nproj; p < NP; ++p) {   // unused slots: valid copies, never read
+        maps.A[p] = maps.A[0];
+        maps.B[p] = maps.B[0];
     }
-    if (MODE == kExpand) ma = mb;
-    if (MODE == kShrink) mb = ma;
 
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
@@ -802,15 +860,12 @@ int launch_mode(const GatherArgs &a, lora_pool_s *pa, lora_pool_s *pb, cudaStrea
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const int G = a.d_out >> 3;
-    int e_max = G / (kCS * 8);
-    if (e_max < 1) e_max = 1;
-    long long want = (long long)(a.T > 0 ? a.T : 1) * (MODE == kShrink ? 1 : e_max);
+    long long want = (long long)(a.T > 0 ? a.T : 1) * a.nproj * (MODE == kShrink ? 1 : e_max);
     int ncl = (int)(want < mcl ? want : mcl);
     if (ncl < 1) ncl = 1;
     cfg.gridDim = dim3(kCS * ncl);
     cfg.numAttrs = pdl ? 2 : 1;
-    if (int rc = cuda_check(cudaLaunchKernelEx(&cfg, gather_kernel<MODE>, ma, mb, a, e_max))) return rc;
+    if (int rc = cuda_check(cudaLaunchKernelEx(&cfg, gather_kernel<MODE, NP>, maps, a, e_max))) return rc;
     count_launch();
     return LORA_OK;
 }
@@ -819,11 +874,16 @@ int launch_mode(const GatherArgs &a, lora_pool_s *pa, lora_pool_s *pb, cudaStrea
 
 int gather_clusters(int *out) { return max_clusters(out); }
 
-int launch_gather(GatherMode mode, const GatherArgs &a, lora_pool_s *pa, lora_pool_s *pb, cudaStream_t st, bool pdl) {
+int launch_gather(GatherMode mode, const GatherArgs &a, lora_pool_s *const *pa, lora_pool_s *const *pb,
+                  cudaStream_t st, bool pdl) {
+    if (a.nproj > 1) {   // several projections: apply mode only
+        if (mode != kApply) return LORA_ERR_INVALID_ARG;
+        return launch_mode<kApply, LORA_MAX_PROJECTIONS>(a, pa, pb, st, pdl);
+    }
     switch (mode) {
-        case kApply: return launch_mode<kApply>(a, pa, pb, st, pdl);
-        case kShrink: return launch_mode<kShrink>(a, pa, pb, st, pdl);
-        case kExpand: return launch_mode<kExpand>(a, pa, pb, st, pdl);
+        case kApply: return launch_mode<kApply, 1>(a, pa, pb, st, pdl);
+        case kShrink: return launch_mode<kShrink, 1>(a, pa, pb, st, pdl);
+        case kExpand: return launch_mode<kExpand, 1>(a, pa, pb, st, pdl);
     }
     return LORA_ERR_INVALID_ARG;
 }

@@ -125,30 +125,39 @@ inline PlanOut plan_in_ws(void *ws, int T, int S) {
     o.seg_start_copy = nullptr;
     return o;
 }
+// units_per_job: gather units each job becomes (projections sharing the plan);
+// the job size rule then counts clusters / units_per_job.
 int launch_plan(const int32_t *ids, int T, const int32_t *ranks, int S, int long_thresh,
-                int job_tokens, const PlanOut &out, int32_t *err_dev, cudaStream_t st);
+                int job_tokens, const PlanOut &out, int32_t *err_dev, cudaStream_t st, int units_per_job = 1);
 
 enum GatherMode { kApply = 0, kShrink = 1, kExpand = 2 };
 
-struct GatherArgs {
-    const uint16_t *X;
-    float *Y;
-    float *V;
-    int T, d_in, d_out;
-    int S;              // slots in the page table
+// One adapted projection of a gather launch: its output and slot tables.
+struct GatherProj {
+    float *Y;           // [T][d_out] fp32, in place
+    int d_out;
     const int32_t *ranks;
     const float *scales;
     const int32_t *pt;
-    const uint16_t *poolA;
-    const uint16_t *poolB;
+    long long rowsA;    // rows in the A pool (pages * 16); 0 when unused
+    long long rowsB;
+};
+
+struct GatherArgs {
+    const uint16_t *X;
+    float *V;
+    int T, d_in;
+    int S;              // slots in every projection's tables
+    int nproj;          // projections sharing X and the plan (1..LORA_MAX_PROJECTIONS)
+    GatherProj proj[LORA_MAX_PROJECTIONS];
     const int32_t *perm;
     const int4 *jobs;
     const PlanHeader *hdr;
     int32_t *err;
-    long long rowsA;   // rows in the A pool (pages * 16); 0 when unused
-    long long rowsB;
 };
-int launch_gather(GatherMode mode, const GatherArgs &a, lora_pool_s *pa, lora_pool_s *pb, cudaStream_t st, bool pdl);
+// pa[p], pb[p]: the pools of projection p.
+int launch_gather(GatherMode mode, const GatherArgs &a, lora_pool_s *const *pa, lora_pool_s *const *pb,
+                  cudaStream_t st, bool pdl);
 // Clusters the gather kernel keeps resident on the current device (its grid
 // size in clusters when there is enough work).
 int gather_clusters(int *out);

@@ -77,18 +77,20 @@ extern "C" int lora_apply_noalloc(const uint16_t *X, float *Y, int T, int d_in, 
     if (int rc = launch_plan(ids, T, ranks, num_slots, long_thresh, opt_job_tokens(), o, err_dev, st)) return rc;
 
     GatherArgs a = {};
-    a.X = X; a.Y = Y; a.T = T; a.d_in = d_in; a.d_out = d_out; a.S = num_slots;
-    a.ranks = ranks; a.scales = scales; a.pt = page_table; a.poolA = pa->base; a.poolB = pb->base;
+    a.X = X; a.T = T; a.d_in = d_in; a.S = num_slots; a.nproj = 1;
+    a.proj[0].Y = Y; a.proj[0].d_out = d_out; a.proj[0].ranks = ranks; a.proj[0].scales = scales;
+    a.proj[0].pt = page_table;
+    a.proj[0].rowsA = (long long)pa->num_pages * LORA_PAGE_ROWS;
+    a.proj[0].rowsB = (long long)pb->num_pages * LORA_PAGE_ROWS;
     a.perm = o.perm_short; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
-    a.rowsA = (long long)pa->num_pages * LORA_PAGE_ROWS;
-    a.rowsB = (long long)pb->num_pages * LORA_PAGE_ROWS;
-    if (int rc = launch_gather(kApply, a, pa, pb, st, true)) return rc;
+    lora_pool_s *ppa[1] = {pa}, *ppb[1] = {pb};
+    if (int rc = launch_gather(kApply, a, ppa, ppb, st, true)) return rc;
     if (use_tiles) {
         TileArgs ta = {};
         ta.X = X; ta.Y = Y; ta.T = T; ta.d_in = d_in; ta.d_out = d_out;
         ta.ranks = ranks; ta.scales = scales; ta.pt = page_table; ta.pa = pa; ta.pb = pb;
         ta.tiles = o.tiles; ta.hdr = o.header; ta.err = err_dev;
-        ta.rowsA = a.rowsA; ta.rowsB = a.rowsB; ta.long_thresh = long_thresh;
+        ta.rowsA = a.proj[0].rowsA; ta.rowsB = a.proj[0].rowsB; ta.long_thresh = long_thresh;
         if (int rc = launch_tiles(ta, st, true)) return rc;
     }
     return LORA_OK;

@@ -384,7 +384,7 @@ plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ 
 }  // namespace
 
 int launch_plan(const int32_t *ids, int T, const int32_t *ranks, int S, int long_thresh, int job_tokens,
-                const PlanOut &out, int32_t *err_dev, cudaStream_t st) {
+                const PlanOut &out, int32_t *err_dev, cudaStream_t st, int units_per_job) {
     int W = 32;
     while (W > 1 && W * S > kTableEntries) W >>= 1;
     const size_t smem = sizeof(int) * ((size_t)S * W + (size_t)S);
@@ -400,6 +400,7 @@ int launch_plan(const int32_t *ids, int T, const int32_t *ranks, int S, int long
     }
     int clusters = 1;
     if (int rc = gather_clusters(&clusters)) return rc;
+    clusters = max(1, clusters / max(1, units_per_job));
     plan_kernel<<<1, kPlanThreads, smem, st>>>(ids, T, ranks, S, W, long_thresh, job_tokens, clusters, out, err_dev);
     count_launch();
     return cuda_check(cudaGetLastError());

@@ -74,3 +74,20 @@ class AdapterLayer:
              ws: Optional[torch.Tensor] = None, stream=None) -> None:
         B.lora_plan(ids, ids.shape[0], self.ranks, self.S, perm, seg_start, self.ws if ws is None else ws,
                     self.err, stream)
+
+
+def apply_multi(layers, X: torch.Tensor, Ys, ids: Optional[torch.Tensor], ws: Optional[torch.Tensor] = None,
+                err: Optional[torch.Tensor] = None, stream=None) -> None:
+    """One lora_apply_multi call over several AdapterLayer objects that read the
+    same X (same d_in and slot count): Ys[p] += branch of layers[p].  The plan
+    follows layers[0]'s ranks; ws and err default to layers[0]'s.  With
+    ids=None the plan already in ws is used (lora_apply_multi_planned)."""
+    l0 = layers[0]
+    projs = [(Y, l.d_out, l.ranks, l.scales, l.page_table, l.pool_a, l.pool_b) for l, Y in zip(layers, Ys)]
+    ws = l0.ws if ws is None else ws
+    err = l0.err if err is None else err
+    if ids is None:
+        B.lora_apply_multi_planned(X, X.shape[0], l0.d_in, l0.S, projs, ws, err, stream)
+    else:
+        B.lora_apply_multi(X, X.shape[0], l0.d_in, ids, l0.S, projs, ws, err, stream)
+

@@ -74,6 +74,7 @@ typedef struct lora_pool_s *lora_pool_t;        /* opaque host handle of one pag
 #define LORA_MAX_RANK             64
 #define LORA_MAX_PAGES_PER_MATRIX 4    /* LORA_MAX_RANK / LORA_PAGE_ROWS */
 #define LORA_MAX_JOB_TOKENS       16   /* most tokens one gather job serves (one weight read) */
+#define LORA_MAX_PROJECTIONS      8    /* most projections one lora_apply_multi call updates */
 #define LORA_MAX_SLOTS            4096
 
 /* ------------------------------------------------------------------------ */
@@ -197,6 +198,48 @@ int lora_apply_planned(const uint16_t *X, float *Y, int T, int d_in, int d_out, 
                        const int32_t *ranks, const float *scales, const int32_t *page_table,
                        lora_pool_t pa, lora_pool_t pb, void *ws, size_t ws_bytes,
                        int32_t *err_dev, lora_stream_t stream);
+
+/* One adapted projection of lora_apply_multi: its output Y [T][d_out] fp32
+ * (in place, 16-byte aligned), its slot tables (ranks, scales, page_table as
+ * for lora_apply) and its pools (pa of width d_in, pb of width d_out). */
+typedef struct {
+    float *Y;
+    int d_out;
+    const int32_t *ranks;
+    const float *scales;
+    const int32_t *page_table;
+    lora_pool_t pa;
+    lora_pool_t pb;
+} lora_projection_t;
+
+/* Several projections that read the same X, in one call: for every
+ * projection p and token t, Y_p[t] += s_{p,i} (X[t] A_{p,i}) B_{p,i}.
+ * Page "Multi-LoRA Serving Architecture ... (2026)", section "The memory
+ * arithmetic that makes it work": an all-linear adapter has A and B for each
+ * of a layer's seven projections (query, key and value read the same input,
+ * as do gate and up), each with its own output width.
+ *   projs: host array of num_projs (1..LORA_MAX_PROJECTIONS) projections;
+ *   the library reads it during the call only.  All share X, T, d_in, ids,
+ *   num_slots and one plan (made with projs[0].ranks: the error bits and the
+ *   tokens dropped follow projection 0; a slot that is empty in another
+ *   projection is skipped there).  Short segments of every projection are
+ *   handled by one gather launch; long runs get one tile launch per
+ *   projection.  ws as for lora_apply (lora_workspace_size(T, num_slots)).
+ * Each projection's result is bit-identical to lora_apply on that projection
+ * alone.  Errors: as lora_apply, checked for every projection before any
+ * work is enqueued; LORA_ERR_INVALID_ARG for num_projs out of range. */
+int lora_apply_multi(const uint16_t *X, int T, int d_in, const int32_t *ids, int num_slots,
+                     const lora_projection_t *projs, int num_projs, void *ws, size_t ws_bytes,
+                     int32_t *err_dev, lora_stream_t stream);
+
+/* The compute half of lora_apply_multi over the plan that lora_plan (or an
+ * earlier apply call on this batch) left in ws, as lora_apply_planned is for
+ * lora_apply: a model plans once per batch and applies every group of
+ * projections that share an input.  Same arguments and errors as
+ * lora_apply_multi without ids; launches only the compute kernels. */
+int lora_apply_multi_planned(const uint16_t *X, int T, int d_in, int num_slots,
+                             const lora_projection_t *projs, int num_projs, void *ws, size_t ws_bytes,
+                             int32_t *err_dev, lora_stream_t stream);
 
 /* lora_apply without a workspace argument, for callers that cannot allocate
  * device memory: e.g. a plug-in inside a host framework that owns all device

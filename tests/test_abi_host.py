@@ -101,6 +101,21 @@ def test_load_and_apply_validation_before_any_cuda_call(lib):
     # an empty batch is a no-op that launches nothing
     assert lib.lora_apply(fake, fake, 0, 64, 32, fake, 4, fake, fake, fake, pa, pb, ws,
                           lib.lora_workspace_size(0, 4), None, s) == 0
+    # lora_apply_multi: projection count, per-projection widths and workspace
+    from heterogeneous_adapter_batching_b200._binding import LoraProjection
+    good = LoraProjection(FAKE_DEV + (2 << 20), 32, FAKE_DEV + (2 << 20), FAKE_DEV + (2 << 20),
+                          FAKE_DEV + (2 << 20), pa.value, pb.value)
+    wrong = LoraProjection(FAKE_DEV + (2 << 20), 64, FAKE_DEV + (2 << 20), FAKE_DEV + (2 << 20),
+                           FAKE_DEV + (2 << 20), pa.value, pb.value)
+    arr = (LoraProjection * 9)(*([good] * 9))
+    assert lib.lora_apply_multi(fake, 8, 64, fake, 4, arr, 0, ws, ws_n, None, s) == -1
+    assert lib.lora_apply_multi(fake, 8, 64, fake, 4, arr, 9, ws, ws_n, None, s) == -1
+    assert lib.lora_apply_multi(fake, 8, 64, fake, 4, None, 1, ws, ws_n, None, s) == -1
+    assert lib.lora_apply_multi(fake, 8, 64, fake, 4, arr, 2, ws, ws_n - 1, None, s) == -7
+    two = (LoraProjection * 2)(good, wrong)
+    assert lib.lora_apply_multi(fake, 8, 64, fake, 4, two, 2, ws, ws_n, None, s) == -3
+    assert lib.lora_apply_multi(fake, 8, 32, fake, 4, arr, 1, ws, ws_n, None, s) == -3
+    assert lib.lora_apply_multi(fake, 0, 64, fake, 4, arr, 8, ws, lib.lora_workspace_size(0, 4), None, s) == 0
     assert lib.lora_last_launch_count() == 0
     assert lib.lora_shrink(fake, 8, 32, fake, 4, fake, fake, pa, fake, ws, ws_n, None, s) == -3
     assert lib.lora_expand_add(fake, fake, 8, 64, fake, 4, fake, fake, fake, pb, ws, ws_n, None, s) == -3
