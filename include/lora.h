@@ -170,7 +170,9 @@ int lora_shrink(const uint16_t *X, int T, int d_in, const int32_t *ids, int num_
 
 /* Expand-add: Y[t, c] += s_i * sum_{k < r_i} V[t, k] B_i[k, c], fp32.
  *   V [T][LORA_MAX_RANK] fp32, Y [T][d_out] fp32 in place, scales [num_slots]
- *   fp32 (alpha_i / r_i).  pb's width must be d_out. */
+ *   fp32 (alpha_i / r_i).  pb's width must be d_out.  The product runs on the
+ *   tensor cores with each V value split into a bf16 high part and a bf16
+ *   low part (about 16 significant bits of V), fp32 accumulation. */
 int lora_expand_add(const float *V, float *Y, int T, int d_out, const int32_t *ids, int num_slots,
                     const int32_t *ranks, const float *scales, const int32_t *page_table,
                     lora_pool_t pb, void *ws, size_t ws_bytes, int32_t *err_dev,
