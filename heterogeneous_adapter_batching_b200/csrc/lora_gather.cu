@@ -67,13 +67,13 @@ static_assert(kMaxJobTokens == LORA_MAX_JOB_TOKENS, "job size must be a whole nu
 constexpr int kRedBytes = kConsumerWarps * kMaxPages * kMaxNTiles * 128 * 4;
 constexpr int kPartFloats = kMaxJobTokens * LORA_MAX_RANK;
 constexpr int kVBytes = kMaxJobTokens * LORA_MAX_RANK * 2;   // one bf16 part of v
-// During the expand each warp turns its MMA results into rows of Y through a
-// 16-token x 16-column fp32 tile in the X buffers, after the two parts of v.
+// During the expand each warp turns its MMA results into rows of Y through two
+// 16-token x 16-column fp32 tiles in the X buffers, after the two parts of v.
 constexpr int kYTileBytes = kMaxJobTokens * 16 * 4;
 constexpr int kYTileOff = 2 * kVBytes;
 static_assert(kRedBytes + kPartFloats * 4 <= 2 * kMaxJobTokens * kMaxChunkCols * 2,
               "the partial sums must fit in the X buffers");
-static_assert(kYTileOff + kConsumerWarps * kYTileBytes <= 2 * kMaxJobTokens * kMaxChunkCols * 2,
+static_assert(kYTileOff + kConsumerWarps * 2 * kYTileBytes <= 2 * kMaxJobTokens * kMaxChunkCols * 2,
               "the warps' Y tiles must fit in the X buffers");
 
 struct __align__(1024) GatherSmem {
@@ -520,10 +520,10 @@ gather_kernel(const __grid_constant__ GatherMaps<NP> maps, const __grid_constant
         int rtok[kMaxNTiles];
 #pragma unroll
         for (int j = 0; j < kMaxNTiles; ++j) rtok[j] = job_token(a, tk, q0, n, j * kNTok + rt);
-        // Old Y of a 16-column tile, loaded ahead: token tile 0 two tiles
-        // ahead (the warp's first two tiles of the first expand chunk before
-        // the exchange), token tile 1 one tile ahead.  Each (token, column)
-        // belongs to exactly one unit.
+        // Old Y of a 16-column tile: token tile 0 one pair of tiles ahead (the
+        // warp's first pair of the first expand chunk before the exchange),
+        // token tile 1 with its pair.  Each (token, column) belongs to exactly
+        // one unit.
         auto load_y = [&](int c0, int mt, int nmt, int j) {
             const int col = c0 + mt * 16 + 4 * rc;
             return (mt < nmt && rtok[j] >= 0 && col < g.out1)
@@ -704,7 +704,7 @@ gather_kernel(const __grid_constant__ GatherMaps<NP> maps, const __grid_constant
         const uint32_t vbase = smem_u32(&sm.xs) + ((lj >> 1) ? kVBytes : 0);
         const float sc = m.scale;
         float *ytile = reinterpret_cast<float *>(reinterpret_cast<unsigned char *>(&sm.xs) + kYTileOff +
-                                                 warp * kYTileBytes);
+                                                 warp * 2 * kYTileBytes);
         for (int c = 0; c < g.n_expand; ++c, ++chunk) {
             const int s = chunk % kStages;
             const int c0 = g.out0 + c * cw;
@@ -717,62 +717,89 @@ gather_kernel(const __grid_constant__ GatherMaps<NP> maps, const __grid_constant
                 ya = load_y(c0, mt, nmt, 0);
                 yb = load_y(c0, mt + kConsumerWarps, nmt, 0);
             }
+            const int krow = li + 8 * (lj >> 1);
+            // The warp's tiles are taken in pairs (mt, mt + 15) whose fragment
+            // loads and MMAs interleave, so the two dependent chains overlap.
 #pragma unroll 1
-            for (; mt < nmt; mt += kConsumerWarps) {
-                const float4 yc = load_y(c0, mt + 2 * kConsumerWarps, nmt, 0);   // two tiles ahead
-                const float4 y1 = (kMaxNTiles > 1 && nt > 1) ? load_y(c0, mt, nmt, kMaxNTiles - 1)
-                                                             : make_float4(0.f, 0.f, 0.f, 0.f);
-                const int col = c0 + mt * 16 + 4 * rc;
-                const bool ok = col < g.out1;
-                float d[kMaxNTiles][4];
+            for (; mt < nmt; mt += 2 * kConsumerWarps) {
+                const int mtB = mt + kConsumerWarps;
+                const bool hasB = mtB < nmt;
+                // token tile 0 rows of the next pair; token tile 1 rows of this one
+                const float4 yc = load_y(c0, mt + 2 * kConsumerWarps, nmt, 0);
+                const float4 yd = load_y(c0, mt + 3 * kConsumerWarps, nmt, 0);
+                float4 y1[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+                if (kMaxNTiles > 1 && nt > 1) {
+                    y1[0] = load_y(c0, mt, nmt, kMaxNTiles - 1);
+                    y1[1] = load_y(c0, mtB, nmt, kMaxNTiles - 1);
+                }
+                float d[2][kMaxNTiles][4];
 #pragma unroll
-                for (int j = 0; j < kMaxNTiles; ++j)
+                for (int h = 0; h < 2; ++h)
 #pragma unroll
-                    for (int e2 = 0; e2 < 4; ++e2) d[j][e2] = 0.f;
-                const int b = mt >> 2, ms = mt & 3;
-                const int krow = li + 8 * (lj >> 1);
+                    for (int jj = 0; jj < kMaxNTiles; ++jj)
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) d[h][jj][e2] = 0.f;
+                const uint32_t offA = (uint32_t)((mt >> 2) * kBoxBytes + krow * 128 + (((2 * (mt & 3) + (lj & 1)) ^ li) << 4));
+                const uint32_t offB = (uint32_t)((mtB >> 2) * kBoxBytes + krow * 128 + (((2 * (mtB & 3) + (lj & 1)) ^ li) << 4));
 #pragma unroll 1
                 for (int p = 0; p < np; ++p) {
-                    uint32_t af[4];
-                    ldsm_x4_t(sb + (uint32_t)((p * g.nb + b) * kBoxBytes + krow * 128 + (((2 * ms + (lj & 1)) ^ li) << 4)),
-                              af);
+                    const uint32_t pb0 = sb + (uint32_t)(p * g.nb * kBoxBytes);
+                    uint32_t afA[4], afB[4] = {0u, 0u, 0u, 0u};
+                    ldsm_x4_t(pb0 + offA, afA);
+                    if (hasB) ldsm_x4_t(pb0 + offB, afB);
 #pragma unroll
-                    for (int j = 0; j < kMaxNTiles; ++j) {
-                        if (j < nt) {
+                    for (int jj = 0; jj < kMaxNTiles; ++jj) {
+                        if (jj < nt) {
                             uint32_t bv[4];
-                            ldsm_x4(vbase + swz(j * kNTok + li, LORA_MAX_RANK * 2, 2 * p + (lj & 1)), bv);
-                            mma_bf16(d[j], af, bv[0], bv[1]);
-                            mma_bf16(d[j], af, bv[2], bv[3]);
+                            ldsm_x4(vbase + swz(jj * kNTok + li, LORA_MAX_RANK * 2, 2 * p + (lj & 1)), bv);
+                            mma_bf16(d[0][jj], afA, bv[0], bv[1]);
+                            if (hasB) mma_bf16(d[1][jj], afB, bv[0], bv[1]);
+                            mma_bf16(d[0][jj], afA, bv[2], bv[3]);
+                            if (hasB) mma_bf16(d[1][jj], afB, bv[2], bv[3]);
                         }
                     }
                 }
                 // fragments (column g8 / g8 + 8, tokens 2 tig, 2 tig + 1) -> rows:
-                // tile [token][16 columns], 4-column groups swizzled by token
+                // per tile [token][16 columns], 4-column groups swizzled by token
 #pragma unroll
-                for (int j = 0; j < kMaxNTiles; ++j) {
-                    if (j < nt) {
+                for (int h = 0; h < 2; ++h) {
+                    if (h == 0 || hasB) {
 #pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            const int t = j * kNTok + 2 * tig + (e2 & 1), cc = g8 + 8 * (e2 >> 1);
-                            ytile[t * 16 + (((cc >> 2) ^ (t & 3)) << 2) + (cc & 3)] = d[j][e2];
+                        for (int jj = 0; jj < kMaxNTiles; ++jj) {
+                            if (jj < nt) {
+#pragma unroll
+                                for (int e2 = 0; e2 < 4; ++e2) {
+                                    const int t = jj * kNTok + 2 * tig + (e2 & 1), cc = g8 + 8 * (e2 >> 1);
+                                    ytile[h * (kYTileBytes / 4) + t * 16 + (((cc >> 2) ^ (t & 3)) << 2) + (cc & 3)] =
+                                        d[h][jj][e2];
+                                }
+                            }
                         }
                     }
                 }
                 __syncwarp();
 #pragma unroll
-                for (int j = 0; j < kMaxNTiles; ++j) {
-                    const int t = j * kNTok + rt;
-                    const int tok = rtok[j];
-                    if (j < nt && tok >= 0 && ok) {
-                        const float4 dv = *reinterpret_cast<const float4 *>(ytile + t * 16 + ((rc ^ (t & 3)) << 2));
-                        const float4 y = (j == 0) ? ya : y1;
-                        *reinterpret_cast<float4 *>(Yp + (size_t)tok * d_out + col) =
-                            make_float4(fmaf(sc, dv.x, y.x), fmaf(sc, dv.y, y.y), fmaf(sc, dv.z, y.z), fmaf(sc, dv.w, y.w));
+                for (int h = 0; h < 2; ++h) {
+                    const int col = c0 + (mt + h * kConsumerWarps) * 16 + 4 * rc;
+                    if ((h == 0 || hasB) && col < g.out1) {
+#pragma unroll
+                        for (int jj = 0; jj < kMaxNTiles; ++jj) {
+                            const int t = jj * kNTok + rt;
+                            const int tok = rtok[jj];
+                            if (jj < nt && tok >= 0) {
+                                const float4 dv = *reinterpret_cast<const float4 *>(
+                                    ytile + h * (kYTileBytes / 4) + t * 16 + ((rc ^ (t & 3)) << 2));
+                                const float4 y = (jj == 0) ? (h == 0 ? ya : yb) : y1[h];
+                                *reinterpret_cast<float4 *>(Yp + (size_t)tok * d_out + col) =
+                                    make_float4(fmaf(sc, dv.x, y.x), fmaf(sc, dv.y, y.y), fmaf(sc, dv.z, y.z),
+                                                fmaf(sc, dv.w, y.w));
+                            }
+                        }
                     }
                 }
-                __syncwarp();   // the tile is rewritten for the next column tile
-                ya = yb;
-                yb = yc;
+                __syncwarp();   // the tiles are rewritten for the next pair
+                ya = yc;
+                yb = yd;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive_relaxed(&sm.empty[s]);
