@@ -246,3 +246,25 @@ def test_expand_add_matches_oracle(H):
     torch.cuda.synchronize()
     ref, _ = O.lora_expand_add(Vh, wl.Y_base, wl.ids, [a.B for a in wl.adapters], wl.scales_f32())
     U.assert_parity(Y.cpu().numpy(), ref, wl.Y_base)
+
+
+def test_max_slots(H):
+    """LORA_MAX_SLOTS = 4096 resident slots: the plan's smallest per-warp table
+    and slot tables read from global memory (too many to stage)."""
+    wl = W.random_small(seed=61, T=300, d_in=64, d_out=72, S=4096, ranks=(1, 4, 16, 64), p_none=0.05)
+    Y, err, _ = _run_apply(H, wl)
+    ref, rerr = U.oracle_full(wl)
+    assert err == rerr == 0
+    U.assert_parity(Y, ref, wl.Y_base)
+
+
+def test_many_tokens(H):
+    """32768 decode-style tokens over 64 slots: tens of thousands of gather jobs
+    over the persistent clusters (no long runs at this id mix)."""
+    wl = W.random_small(seed=62, T=32768, d_in=128, d_out=136, S=64, ranks=(4, 8, 16, 33, 64), p_none=0.1)
+    Y, err, layer = _run_apply(H, wl)
+    ref, rerr = U.oracle_full(wl)
+    assert err == rerr == 0
+    U.assert_parity(Y, ref, wl.Y_base)
+    jt = U.plan_job_tokens(layer.ws)
+    assert U.plan_counts(layer.ws)[2] == U.expected_work(wl.ids, wl.ranks(), H.lora_get_option(H.OPT_LONG_SEGMENT), jt)[0]
