@@ -186,15 +186,18 @@ def run_reference(args):
     if rank != 0:
         return 0
     wl, desc = workload_spec(args.workload)
+    # one step = oracle calls on the workload's batch (its first tokens when the
+    # batch is large) for at least 20 ms; the value is the median step rate
     per_step = []
     for _ in range(max(args.warmup, 0)):
-        time_oracle(wl, 0.0)
+        time_oracle(wl, 0.02)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        v, threads, sample = time_oracle(wl, 0.0)
+        v, threads, sample = time_oracle(wl, 0.02)
         per_step.append(v)
     el = time.perf_counter() - t0
     value = statistics.median(per_step)
+    sample = f"{args.steps} steps, each {sample}"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * el / max(1, args.steps),
