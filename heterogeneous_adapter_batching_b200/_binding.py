@@ -20,7 +20,7 @@ LORA_OK = 0
 ERR_NAMES = {
     -1: "LORA_ERR_INVALID_ARG", -2: "LORA_ERR_BAD_RANK", -3: "LORA_ERR_WIDTH_MISMATCH",
     -4: "LORA_ERR_POOL_OOM", -5: "LORA_ERR_BAD_SLOT", -6: "LORA_ERR_CUDA", -7: "LORA_ERR_WORKSPACE",
-    -8: "LORA_ERR_TOO_LARGE",
+    -8: "LORA_ERR_TOO_LARGE", -9: "LORA_ERR_ALL_PINNED",
 }
 DEV_ERR_BAD_ID = 1
 DEV_ERR_EMPTY_SLOT = 2
@@ -42,6 +42,8 @@ EXPORTS = [
     "lora_pool_load", "lora_pool_evict", "lora_pool_read_row", "lora_workspace_size",
     "lora_plan", "lora_shrink", "lora_expand_add", "lora_apply", "lora_apply_planned", "lora_apply_noalloc",
     "lora_apply_multi", "lora_apply_multi_planned",
+    "lora_slot_cache_create", "lora_slot_cache_destroy", "lora_slot_cache_acquire", "lora_slot_cache_unpin",
+    "lora_slot_cache_invalidate", "lora_slot_cache_lookup", "lora_slot_cache_stats",
     "lora_set_option", "lora_get_option", "lora_last_cuda_error", "lora_last_launch_count",
 ]
 
@@ -91,6 +93,15 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lora_apply_noalloc": (I, [V, V, I, I, I, V, I, V, V, V, V, V, V, V]),
         "lora_apply_multi": (I, [V, I, I, V, I, ctypes.POINTER(LoraProjection), I, V, Z, V, V]),
         "lora_apply_multi_planned": (I, [V, I, I, I, ctypes.POINTER(LoraProjection), I, V, Z, V, V]),
+        "lora_slot_cache_create": (I, [I, ctypes.POINTER(V)]),
+        "lora_slot_cache_destroy": (I, [V]),
+        "lora_slot_cache_acquire": (I, [V, ctypes.c_int64, I, ctypes.POINTER(I), ctypes.POINTER(I),
+                                        ctypes.POINTER(ctypes.c_int64)]),
+        "lora_slot_cache_unpin": (I, [V, I]),
+        "lora_slot_cache_invalidate": (I, [V, I]),
+        "lora_slot_cache_lookup": (I, [V, ctypes.c_int64, ctypes.POINTER(I)]),
+        "lora_slot_cache_stats": (I, [V, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64),
+                                      ctypes.POINTER(ctypes.c_int64)]),
         "lora_set_option": (I, [I, I]),
         "lora_get_option": (I, [I]),
         "lora_last_cuda_error": (ctypes.c_char_p, []),
@@ -256,6 +267,50 @@ def lora_apply_multi_planned(X, T, d_in, num_slots, projs, ws, err=None, stream=
     _check("lora_apply_multi_planned", load_library().lora_apply_multi_planned(
         _p(X), T, d_in, num_slots, _proj_array(projs), len(projs), _p(ws), ws.numel() * ws.element_size(),
         _p(err), _s(stream)))
+
+
+class SlotCache:
+    """lora_slot_cache_t: which adapter key lives in which slot (exact LRU over
+    the slots no running batch pins).  Host bookkeeping only."""
+
+    def __init__(self, num_slots: int):
+        h = ctypes.c_void_p()
+        _check("lora_slot_cache_create", load_library().lora_slot_cache_create(num_slots, ctypes.byref(h)))
+        self.handle = h.value
+        self.num_slots = num_slots
+        self._slot, self._hit, self._ev = ctypes.c_int(), ctypes.c_int(), ctypes.c_int64()
+
+    def __del__(self):
+        try:
+            if self.handle and _lib is not None:
+                _lib.lora_slot_cache_destroy(ctypes.c_void_p(self.handle))
+                self.handle = 0
+        except Exception:
+            pass
+
+    def acquire(self, key: int, pin: bool = False):
+        """-> (slot, hit, evicted_key or -1)."""
+        _check("lora_slot_cache_acquire", _lib.lora_slot_cache_acquire(
+            ctypes.c_void_p(self.handle), key, 1 if pin else 0, ctypes.byref(self._slot), ctypes.byref(self._hit),
+            ctypes.byref(self._ev)))
+        return self._slot.value, bool(self._hit.value), self._ev.value
+
+    def unpin(self, slot: int) -> None:
+        _check("lora_slot_cache_unpin", _lib.lora_slot_cache_unpin(ctypes.c_void_p(self.handle), slot))
+
+    def invalidate(self, slot: int) -> None:
+        _check("lora_slot_cache_invalidate", _lib.lora_slot_cache_invalidate(ctypes.c_void_p(self.handle), slot))
+
+    def lookup(self, key: int) -> int:
+        _check("lora_slot_cache_lookup", _lib.lora_slot_cache_lookup(ctypes.c_void_p(self.handle), key,
+                                                                     ctypes.byref(self._slot)))
+        return self._slot.value
+
+    def stats(self):
+        h, m, e = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+        _check("lora_slot_cache_stats", _lib.lora_slot_cache_stats(ctypes.c_void_p(self.handle), ctypes.byref(h),
+                                                                   ctypes.byref(m), ctypes.byref(e)))
+        return h.value, m.value, e.value
 
 
 def lora_set_option(key: int, value: int) -> None:

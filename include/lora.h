@@ -61,6 +61,7 @@ typedef struct lora_pool_s *lora_pool_t;        /* opaque host handle of one pag
 #define LORA_ERR_CUDA           -6   /* a CUDA runtime call failed; see lora_last_cuda_error() */
 #define LORA_ERR_WORKSPACE      -7   /* ws is NULL or ws_bytes < lora_workspace_size(...) */
 #define LORA_ERR_TOO_LARGE      -8   /* lora_apply_noalloc: T or num_slots beyond its fixed scratch */
+#define LORA_ERR_ALL_PINNED     -9   /* slot cache: every slot is held by a running batch */
 
 /* Device error word bits. */
 #define LORA_DEV_ERR_BAD_ID      1   /* some id < -1 or id >= num_slots */
@@ -270,6 +271,51 @@ int lora_apply_noalloc(const uint16_t *X, float *Y, int T, int d_in, int d_out, 
                        int num_slots, const int32_t *ranks, const float *scales,
                        const int32_t *page_table, lora_pool_t pa, lora_pool_t pb,
                        int32_t *err_dev, lora_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Slot manager (host bookkeeping of which adapter lives in which slot)       */
+/* ------------------------------------------------------------------------ */
+/* Page "LoRA Adapters at Serve Time with vLLM Multi-LoRA", section "The
+ * Inference Mechanism: A Worked Scenario", step "Eviction": when every slot is
+ * taken the least recently used adapter is swapped out; page "Multi-LoRA
+ * Serving Architecture ... (2026)", section "An adapter-cache LRU simulator":
+ * an LRU over a fixed slot count judged by its hit rate, where in a batching
+ * engine the slots hold the running batch's adapters (here: pinned slots).
+ * The manager is host-only and thread-safe; it never touches device memory:
+ * on a miss the caller evicts the returned key's pages and loads the new
+ * adapter into the returned slot with lora_pool_evict / lora_pool_load, on the
+ * stream of its choice (a second stream overlaps the load with compute). */
+typedef struct lora_slot_cache_s *lora_slot_cache_t;
+
+/* num_slots in [1, LORA_MAX_SLOTS], all initially empty. */
+int lora_slot_cache_create(int num_slots, lora_slot_cache_t *out);
+int lora_slot_cache_destroy(lora_slot_cache_t c);
+
+/* Make adapter `key` (>= 0, the caller's id) resident and most recently used.
+ *   *hit_out = 1: it already was, in *slot_out.
+ *   *hit_out = 0: it now owns *slot_out: the lowest-numbered never-used slot,
+ *   else the most recently emptied one, else the least recently used slot
+ *   whose pin count is 0; *evicted_key_out is the key that slot held (-1 if
+ *   none).  The caller must load the adapter before a batch uses the slot.
+ * pin != 0 adds one to the slot's pin count (a running batch uses it).
+ * Errors: LORA_ERR_ALL_PINNED when a miss finds every slot pinned (nothing
+ * changes); LORA_ERR_INVALID_ARG for key < 0 or NULL outputs. */
+int lora_slot_cache_acquire(lora_slot_cache_t c, int64_t key, int pin, int *slot_out, int *hit_out,
+                            int64_t *evicted_key_out);
+
+/* Drop one pin of `slot` (the batch that used it finished).  LORA_ERR_BAD_SLOT
+ * for a slot out of range, LORA_ERR_INVALID_ARG when it holds no pin. */
+int lora_slot_cache_unpin(lora_slot_cache_t c, int slot);
+
+/* Mark `slot` empty (its adapter was evicted by the caller); it is the next
+ * slot a miss takes.  LORA_ERR_ALL_PINNED if the slot is pinned. */
+int lora_slot_cache_invalidate(lora_slot_cache_t c, int slot);
+
+/* Slot of `key`, or -1, without touching the recency order. */
+int lora_slot_cache_lookup(lora_slot_cache_t c, int64_t key, int *slot_out);
+
+/* Counters since creation: acquire hits, misses, and misses that evicted. */
+int lora_slot_cache_stats(lora_slot_cache_t c, int64_t *hits, int64_t *misses, int64_t *evictions);
 
 /* ------------------------------------------------------------------------ */
 /* Options and diagnostics (process-wide)                                   */
