@@ -23,7 +23,7 @@ bf16-rounded inputs the GPU path receives.  Sources (page title, section):
 * same page, "The memory arithmetic that makes it work": an adapter on a
   projection costs r*(d_in + d_out) parameters.
 
-Readings where the pages are silent (listed in the design doc as well):
+Readings where the pages are silent:
   * orientation follows the llms.blog page (row vectors); the column-vector
     form on the iotdigitaltwinplm page is its transpose;
   * the scale alpha/r is part of the method (the ashishsrivastav page drops
