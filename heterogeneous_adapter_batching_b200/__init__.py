@@ -5,4 +5,4 @@ include/lora.h; this package only marshals torch tensors into those calls.
 """
 from . import _binding
 from ._binding import *  # noqa: F401,F403
-from .layer import AdapterLayer, apply_multi  # noqa: F401
+from .layer import AdapterCache, AdapterLayer, apply_multi  # noqa: F401

@@ -91,3 +91,43 @@ def apply_multi(layers, X: torch.Tensor, Ys, ids: Optional[torch.Tensor], ws: Op
     else:
         B.lora_apply_multi(X, X.shape[0], l0.d_in, ids, l0.S, projs, ws, err, stream)
 
+
+
+class AdapterCache:
+    """A working set of adapters kept resident in one AdapterLayer's pools.
+
+    `host` maps an adapter key to (a_t_bits [r, d_in], b_bits [r, d_out], alpha)
+    (bf16 tensors, host or device).  map_batch() turns the per-token keys of a
+    batch into slot ids, loading the adapters that are not resident into the
+    slots the LRU slot manager (lora_slot_cache_*) picks and pinning every slot
+    the batch uses; release() unpins them once the batch has run.
+    """
+
+    def __init__(self, layer: AdapterLayer, host):
+        self.layer = layer
+        self.host = host
+        self.slots = B.SlotCache(layer.S)
+
+    def map_batch(self, keys, stream=None):
+        """keys: per-token adapter keys (-1 = base model only).
+        Returns (ids int32 tensor on the layer's device, pinned slot list)."""
+        slot_of, pinned = {}, []
+        for k in keys:
+            k = int(k)
+            if k < 0 or k in slot_of:
+                continue
+            slot, hit, evicted = self.slots.acquire(k, pin=True)
+            pinned.append(slot)
+            if not hit:
+                if evicted >= 0:
+                    self.layer.evict(slot, stream=stream)
+                at, b, alpha = self.host[k]
+                self.layer.load(slot, at.shape[0], alpha, at, b, stream=stream)
+            slot_of[k] = slot
+        ids = torch.tensor([slot_of.get(int(k), -1) for k in keys], dtype=torch.int32,
+                           device=self.layer.device)
+        return ids, pinned
+
+    def release(self, pinned) -> None:
+        for s in pinned:
+            self.slots.unpin(s)
