@@ -10,8 +10,9 @@
 // weights are read straight out of the physical pages the page table names.
 //
 // Work unit = one gather job (an adapter slot and up to 16 of its tokens, from
-// the plan kernel) times one part e of an E-way split of d_out.  A cluster of
-// kCS CTAs (one per SM) runs one unit at a time and loops over the units
+// the plan kernel) times one projection (a launch may cover up to 8 that read
+// the same X) times one part e of an E-way split of d_out.  A cluster of kCS
+// CTAs (one per SM) runs one unit at a time and loops over the units
 // (persistent grid sized from the occupancy of the cluster shape).  Per CTA:
 //   * a producer warp streams the adapter's pages into a ring of shared-memory
 //     stages with 2D TMA loads of 16 rank rows x 64 columns (128-byte
@@ -23,20 +24,23 @@
 //   * 15 consumer warps copy the tokens' X columns of each chunk into shared
 //     memory (cp.async, issued one chunk ahead) and run the shrink on the
 //     tensor cores with warp-level bf16 MMAs (m16n8k16, fp32 accumulate): a
-//     page's 16 rank rows are the M side, up to 8 tokens the N side, and each
-//     warp owns every 15th 16-column step of the slice.  The warps' partial
-//     sums are added in warp order, the CTAs exchange theirs through
-//     distributed shared memory after one hardware cluster barrier, and each
-//     CTA adds the kCS partials in rank order, so all CTAs hold the same fp32
-//     v and a token's result does not depend on the job it landed in;
+//     page's 16 rank rows are the M side, 8 tokens the N side (two N tiles
+//     for a 16-token job), and each warp owns every 15th 16-column step of
+//     the slice.  The warps' partial sums are added in warp order; each CTA
+//     pushes its partial into its peers' shared memory with asynchronous
+//     DSMEM stores that complete on the peer's mbarrier, and adds the kCS
+//     partials in rank order, so all CTAs hold the same fp32 v and a token's
+//     result does not depend on the job it landed in;
 //   * v is split into a bf16 high part and a bf16 low part (v - high), and the
 //     expand runs as two MMAs per page (output columns on the M side, read
 //     with transposing ldmatrix), which keeps v to about 16 significant bits;
-//     each warp owns every 15th 16-column tile of the d_out slice and adds
-//     scale * (v B) to Y in place.
-// Small page tables (<= 256 slots) are staged in shared memory before the
-// kernel waits for the plan, so a unit's metadata costs one global read (the
-// job record).  Every wait is bounded; a wait that runs out sets
+//     each warp owns every 15th 16-column tile of the d_out slice, takes its
+//     tiles in pairs whose MMA chains interleave, turns the results into rows
+//     through small shared tiles and updates Y in place with float4 rows.
+// Slot tables of up to 128 (projection, slot) entries are staged in shared
+// memory before the kernel waits for its predecessor, so a unit's metadata
+// costs one global read (the job record).  The hardware cluster barrier is
+// used once, at start-up.  Every wait is bounded; a wait that runs out sets
 // LORA_DEV_ERR_TIMEOUT in the error word and the kernel runs to completion
 // without trapping.  No cluster multicast is used.
 #include "lora_internal.cuh"
