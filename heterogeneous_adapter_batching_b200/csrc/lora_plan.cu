@@ -18,12 +18,16 @@
 //   perm_short          perm without the tokens of such runs (a stable
 //                       compaction, so still grouped by slot);
 //   jobs                the short tokens of every slot, split into gather
-//                       jobs of at most job_tokens (<= LORA_MAX_JOB_TOKENS),
-//                       balanced in size: two int4 per job, {slot, count,
-//                       first index into perm_short, 0} and the job's first
-//                       four token indices (-1 padded), so a decode consumer
-//                       needs a single read to know its work (a larger job's
-//                       further tokens follow in perm_short).
+//                       jobs of balanced size, at most the size chosen for
+//                       the batch (4, 8 or the cap job_tokens <=
+//                       LORA_MAX_JOB_TOKENS, from the job counts and the
+//                       gather kernel's cluster count), heaviest rank class
+//                       first: two int4 per job, {slot, count, first index
+//                       into perm_short, 0} and the job's first four token
+//                       indices (-1 padded), so a decode consumer needs a
+//                       single read to know its work (a larger job's further
+//                       tokens follow in perm_short); the header records the
+//                       job size chosen.
 // Invalid ids (outside [-1, S) or an empty slot) are dropped and flagged.
 //
 // One CTA of 1024 threads.  W warps (W * S <= 16384) own contiguous token
