@@ -80,10 +80,12 @@ def workload_spec(name: str):
 
 
 def algorithmic_bytes(wl) -> int:
-    """Each distinct adapter read once (A and B, bf16), X read in bf16, Y read and written in fp32."""
+    """Each distinct adapter read once (A and B, bf16), X read in bf16, Y read and written in fp32,
+    over the tokens whose slot holds an adapter."""
     ids = wl.ids
-    valid = ids[(ids >= 0) & (ids < wl.S)]
     rk = wl.ranks()
+    inr = (ids >= 0) & (ids < wl.S)
+    valid = ids[inr][rk[ids[inr]] > 0]
     distinct = np.unique(valid)
     w = int(sum(2 * int(rk[i]) * (wl.d_in + wl.d_out) for i in distinct))
     return w + len(valid) * (2 * wl.d_in + 8 * wl.d_out)
@@ -91,8 +93,9 @@ def algorithmic_bytes(wl) -> int:
 
 def algorithmic_flops(wl) -> int:
     ids = wl.ids
-    valid = ids[(ids >= 0) & (ids < wl.S)]
     rk = wl.ranks()
+    inr = (ids >= 0) & (ids < wl.S)
+    valid = ids[inr][rk[ids[inr]] > 0]
     return int(sum(2 * int(rk[i]) * (wl.d_in + wl.d_out) for i in valid))
 
 
