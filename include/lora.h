@@ -37,6 +37,10 @@
  *    means "base model only" and is not an error.  Kernels never trap.
  *  - The library keeps no device memory of its own: scratch space comes
  *    from the caller's workspace (ws, ws_bytes).
+ *  - Host threads: calls may come from several threads.  A pool's free list,
+ *    a slot cache and the options are guarded inside the library; a
+ *    workspace, an error word and the device tables belong to whoever passes
+ *    them, and calls that share one must be ordered on one stream.
  */
 #ifndef LORA_H_
 #define LORA_H_
