@@ -238,7 +238,8 @@ class Ring:
                     continue
                 at = (torch.randn((r, wl.d_in), generator=g, device=device) / math.sqrt(wl.d_in)).to(torch.bfloat16)
                 b = (torch.randn((r, wl.d_out), generator=g, device=device) / math.sqrt(r)).to(torch.bfloat16)
-                lay.load(i, r, 2.0 * r, at, b, page_ids=torch.from_numpy(np.ascontiguousarray(wl.page_ids[i])))
+                lay.load(i, r, float(wl.adapters.alpha_of[i]), at, b,
+                         page_ids=torch.from_numpy(np.ascontiguousarray(wl.page_ids[i])))
             self.layers.append(lay)
             self.X.append((torch.randn((wl.T, wl.d_in), generator=g, device=device) / math.sqrt(wl.d_in)).to(torch.bfloat16))
             self.Y.append(torch.randn((wl.T, wl.d_out), generator=g, device=device))

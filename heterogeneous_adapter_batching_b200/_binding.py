@@ -33,7 +33,7 @@ MAX_SLOTS = 4096
 OPT_LONG_SEGMENT = 1
 OPT_DECODE_JOB_TOKENS = 2
 NOALLOC_MAX_TOKENS = 32768
-NOALLOC_SCRATCH_BYTES = 2097152
+NOALLOC_SCRATCH_BYTES = 2162688
 MAX_JOB_TOKENS = 16
 MAX_PROJECTIONS = 8
 

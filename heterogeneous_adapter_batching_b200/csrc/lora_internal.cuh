@@ -32,10 +32,11 @@ struct WsLayout {
     size_t header, seg_start, perm, perm_short, run_start, run_end, jobs, tiles, total;
 };
 
-inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-inline WsLayout ws_layout(int T, int S) {
-    WsLayout l;
+// constexpr so that the fixed scratch of lora_apply_noalloc can be sized from it.
+constexpr WsLayout ws_layout(int T, int S) {
+    WsLayout l{};
     const size_t t = (size_t)(T > 0 ? T : 1);
     size_t o = 0;
     l.header = o;     o = align_up(o + sizeof(PlanHeader), 256);

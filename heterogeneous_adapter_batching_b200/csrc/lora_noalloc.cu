@@ -23,11 +23,19 @@ namespace {
 // once per device with cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[LORA_NOALLOC_SCRATCH_BYTES];
 
+// The scratch holds the whole plan of the largest call the entry point admits.
+static_assert(ws_layout(LORA_NOALLOC_MAX_TOKENS, LORA_MAX_SLOTS).total <= (size_t)LORA_NOALLOC_SCRATCH_BYTES,
+              "LORA_NOALLOC_SCRATCH_BYTES is smaller than the plan of LORA_NOALLOC_MAX_TOKENS tokens and "
+              "LORA_MAX_SLOTS slots");
+
 std::mutex g_noalloc_mu;
 void *g_noalloc_ptr[64] = {};
 
 // Device address of the scratch array on the current device, looked up on the
-// first call made on that device.
+// first call made on that device and kept for the life of the process.  The
+// address belongs to the device's primary context: a cudaDeviceReset makes it
+// stale, so a process that resets a device must not call this entry point on
+// that device again.
 int noalloc_scratch(void **out) {
     int dev = 0;
     if (int rc = cuda_check(cudaGetDevice(&dev))) return rc;

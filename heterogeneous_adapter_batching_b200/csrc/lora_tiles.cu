@@ -163,6 +163,7 @@ __device__ __forceinline__ bool epi_all(bool ok) {
 struct UnitInfo {
     int slot, row0, ntok, r, n1, np, j0, j1;
     bool skip;
+    bool bad;    // rank above 64 or a page outside its pool (LORA_DEV_ERR_BAD_PAGE); rank 0 is not bad
 };
 
 __device__ __forceinline__ UnitInfo unit_info(const TileArgs &a, int tile, int j0, int j1) {
@@ -174,13 +175,15 @@ __device__ __forceinline__ UnitInfo unit_info(const TileArgs &a, int tile, int j
     ui.j0 = j0;
     ui.j1 = j1;
     int r = a.ranks[ui.slot];
-    bool bad = r <= 0 || r > LORA_MAX_RANK;
-    const int np = bad ? 0 : (r + 15) >> 4;
+    bool bad = r > LORA_MAX_RANK;
+    const int np = (bad || r <= 0) ? 0 : (r + 15) >> 4;
     for (int p = 0; p < np; ++p) {
         const int pa = a.pt[ui.slot * 8 + p], pb = a.pt[ui.slot * 8 + 4 + p];
         if (pa < 0 || (long long)(pa + 1) * LORA_PAGE_ROWS > a.rowsA) bad = true;
         if (pb < 0 || (long long)(pb + 1) * LORA_PAGE_ROWS > a.rowsB) bad = true;
     }
+    ui.bad = bad;
+    bad = bad || r <= 0;
     ui.skip = bad || ui.j0 >= ui.j1;
     ui.r = bad ? 0 : r;
     ui.np = bad ? 0 : np;
@@ -271,6 +274,7 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
         UnitIter ur = unit_range(n_tiles, nj);
         UnitInfo ui;
         while (next_unit(a, ur, ui) && !aborted(sm)) {
+            if (ui.bad && a.err) atomicOr(a.err, LORA_DEV_ERR_BAD_PAGE);
             if (ui.skip) continue;
             int pg[4];
             for (int p = 0; p < 4; ++p) pg[p] = p < ui.np ? a.pt[ui.slot * 8 + p] : 0;

@@ -35,8 +35,11 @@
  *    LORA_DEV_ERR_* bits.  A token whose id is outside [-1, S) or names an
  *    empty slot (rank 0) is skipped: its Y row is left untouched.  id = -1
  *    means "base model only" and is not an error.  Kernels never trap.
- *  - The library keeps no device memory of its own: scratch space comes
- *    from the caller's workspace (ws, ws_bytes).
+ *  - Scratch space comes from the caller's workspace (ws, ws_bytes).  The one
+ *    exception is lora_apply_noalloc, for callers that cannot allocate: its
+ *    plan lives in a fixed static device array of the library
+ *    (LORA_NOALLOC_SCRATCH_BYTES per GPU that loads the library, held until
+ *    the process exits).  No call allocates device memory.
  *  - Host threads: calls may come from several threads.  A pool's free list,
  *    a slot cache and the options are guarded inside the library; a
  *    workspace, an error word and the device tables belong to whoever passes
@@ -129,6 +132,11 @@ int lora_pool_load(lora_pool_t pa, lora_pool_t pb, int slot, int num_slots, int 
 
 /* Return the pages of (page_table_dev, slot) to the free lists and mark the
  * slot empty on the device (rank 0, scale 0, page entries -1) on `stream`.
+ * Page "LoRA Adapters at Serve Time with vLLM Multi-LoRA", section "The
+ * Inference Mechanism: A Worked Scenario", step "Eviction": a resident
+ * adapter is swapped out to make room; page "Multi-LoRA Serving in
+ * Production", section "Unified Paging Architecture": its pages go back to
+ * the shared pool.
  * Pages are reused in stream order: a later load on the same stream is safe;
  * a caller using several streams must order them itself. */
 int lora_pool_evict(lora_pool_t pa, lora_pool_t pb, int slot, int num_slots,
@@ -167,6 +175,9 @@ int lora_plan(const int32_t *ids, int T, const int32_t *ranks, int num_slots,
               void *ws, size_t ws_bytes, int32_t *err_dev, lora_stream_t stream);
 
 /* Shrink: V[t, k] = sum_j X[t, j] A_i[j, k] for k < r_i, fp32 accumulate.
+ * Page "Multi-LoRA Serving in Production", section "Segmented Gather
+ * Matrix-Vector Multiplication (SGMV)": the first of the two steps projects
+ * each token onto its own adapter's rank-r_i space (v = x A).
  *   X [T][d_in] bf16, V [T][LORA_MAX_RANK] fp32 (columns >= r_i and rows of
  *   tokens without a valid adapter are left untouched).  pa's width must be d_in. */
 int lora_shrink(const uint16_t *X, int T, int d_in, const int32_t *ids, int num_slots,
@@ -174,6 +185,10 @@ int lora_shrink(const uint16_t *X, int T, int d_in, const int32_t *ids, int num_
                 float *V, void *ws, size_t ws_bytes, int32_t *err_dev, lora_stream_t stream);
 
 /* Expand-add: Y[t, c] += s_i * sum_{k < r_i} V[t, k] B_i[k, c], fp32.
+ * Page "Multi-LoRA Serving in Production", section "Segmented Gather
+ * Matrix-Vector Multiplication (SGMV)": the second step expands v back to the
+ * output width through B, scales it by alpha/r and adds it to the base
+ * output.
  *   V [T][LORA_MAX_RANK] fp32, Y [T][d_out] fp32 in place, scales [num_slots]
  *   fp32 (alpha_i / r_i).  pb's width must be d_out.  The product runs on the
  *   tensor cores with each V value split into a bf16 high part and a bf16
@@ -264,13 +279,15 @@ int lora_apply_multi_planned(const uint16_t *X, int T, int d_in, int num_slots,
  * LORA_MAX_SLOTS; larger sizes return LORA_ERR_TOO_LARGE before any work is
  * enqueued.  The first call on a device looks up the scratch's device
  * address (cudaGetSymbolAddress) with that device current; make that first
- * call before any stream capture.  All calls share the one array (it keeps the
+ * call before any stream capture.  The address is kept for the process's
+ * life and belongs to the device's primary context: after cudaDeviceReset on
+ * a device, do not call lora_apply_noalloc on that device again.  All calls share the one array (it keeps the
  * last call's contents; each call writes everything it reads, so nothing needs
  * clearing), so calls whose kernels overlap on the GPU - on different streams
  * or from different host threads without ordering - race and give undefined
  * results: order them on one stream. */
 #define LORA_NOALLOC_MAX_TOKENS    32768
-#define LORA_NOALLOC_SCRATCH_BYTES 2097152   /* 2 MiB */
+#define LORA_NOALLOC_SCRATCH_BYTES 2162688   /* 2 MiB + 64 KiB: the plan of 32768 tokens and 4096 slots */
 int lora_apply_noalloc(const uint16_t *X, float *Y, int T, int d_in, int d_out, const int32_t *ids,
                        int num_slots, const int32_t *ranks, const float *scales,
                        const int32_t *page_table, lora_pool_t pa, lora_pool_t pb,

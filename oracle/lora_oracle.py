@@ -138,7 +138,11 @@ def lora_expand_add(V, Y_base, ids, B, scales, ranks=None):
 
 
 def merged_weight(W0, A, B, scale):
-    """W' = W0 + s * A B, the single-tenant pre-merged matrix (fp64)."""
+    """W' = W0 + s * A B, the single-tenant pre-merged matrix (fp64).
+
+    "Multi-LoRA Serving in Production", "The Mathematical Anatomy of
+    Heterogeneous Batches": merging folds the low-rank product into the base
+    weight; the unmerged branch must give X W' for every token."""
     return np.asarray(W0, np.float64) + np.float64(np.float32(scale)) * (
         np.asarray(A, np.float64) @ np.asarray(B, np.float64))
 

@@ -44,7 +44,7 @@ def test_working_set_through_the_slot_manager():
         # the reference uses the adapters by key
         A = [ad[k].A for k in range(n_adapters)]
         Bm = [ad[k].B for k in range(n_adapters)]
-        sc = np.array([2.0] * n_adapters, dtype=np.float32)
+        sc = ad.alpha_of / ranks.astype(np.float32)      # each adapter's own alpha / r
         ref, _ = OC.lora_apply_c(X, Yb, np.array(keys, dtype=np.int32), A, Bm, sc)
         got = Yd.cpu().numpy()
         assert np.all(np.abs(got - ref) <= 2e-3 + 1e-2 * np.abs(ref)), bi

@@ -194,7 +194,8 @@ def test_all_tokens_one_adapter_matches_dense(H):
     Y, err, _ = _run_apply(H, wl)
     i = int(wl.ids[0])
     a = wl.adapters[i]
-    ref = wl.Y_base.astype(np.float64) + 2.0 * (wl.X.astype(np.float64) @ a.A.astype(np.float64)) @ a.B.astype(np.float64)
+    s = np.float64(wl.scales_f32()[i])
+    ref = wl.Y_base.astype(np.float64) + s * (wl.X.astype(np.float64) @ a.A.astype(np.float64)) @ a.B.astype(np.float64)
     assert err == 0
     U.assert_parity(Y, ref, wl.Y_base, delta_rel=U.DELTA_REL_TENSOR)
 
@@ -268,3 +269,79 @@ def test_many_tokens(H):
     U.assert_parity(Y, ref, wl.Y_base)
     jt = U.plan_job_tokens(layer.ws)
     assert U.plan_counts(layer.ws)[2] == U.expected_work(wl.ids, wl.ranks(), H.lora_get_option(H.OPT_LONG_SEGMENT), jt)[0]
+
+
+# ---------------------------------------------------------------------------
+# Slot tables that name memory outside the pool (LORA_DEV_ERR_BAD_PAGE)
+# ---------------------------------------------------------------------------
+
+def _corrupt_and_apply(H, wl, corrupt, thresh=None):
+    """Run lora_apply on a clean layer, then again after `corrupt(layer)` edits the
+    device slot tables; returns (clean Y, corrupted Y, error word)."""
+    import torch
+    if thresh is not None:
+        H.lora_set_option(H.OPT_LONG_SEGMENT, thresh)
+    Yc, err, layer = _run_apply(H, wl)
+    assert err == 0
+    corrupt(layer)
+    X, Y, ids = U.dev_inputs(wl)
+    layer.err.zero_()
+    layer.apply(X, Y, ids)
+    torch.cuda.synchronize()
+    return Yc, Y.cpu().numpy(), int(layer.err.item())
+
+
+@pytest.mark.parametrize("kind", ["a_page_past_pool", "b_page_negative", "rank_above_64"])
+@pytest.mark.parametrize("thresh", [None, 16])
+def test_bad_page_skips_tokens_and_sets_bit(H, kind, thresh):
+    """A page id outside the pool (or -1 inside the rank), or a rank above 64,
+    written straight into the device tables: the kernels check every page before
+    any load, leave that slot's rows at Y_base, set LORA_DEV_ERR_BAD_PAGE and
+    give every other token the clean result bit for bit.  thresh = 16 puts the
+    long runs on the tensor-core tiles."""
+    if thresh is None:
+        wl = W.random_small(seed=71, T=60, d_in=256, d_out=200, S=6, ranks=(16, 33, 64), p_none=0.0)
+    else:
+        wl = W.segments(72, [40, 200, 17, 130], 256, 200, S=6, ranks=(16, 33, 64))
+    bad_slot = int(wl.ids[len(wl.ids) // 2])
+
+    def corrupt(layer):
+        if kind == "a_page_past_pool":
+            layer.page_table[bad_slot, 0, 0] = H.lora_pool_num_pages(layer.pool_a) + 3
+        elif kind == "b_page_negative":
+            layer.page_table[bad_slot, 1, 0] = -1
+        else:
+            layer.ranks[bad_slot] = 65
+
+    Yc, Yb, err = _corrupt_and_apply(H, wl, corrupt, thresh)
+    assert err == H.DEV_ERR_BAD_PAGE
+    rows = wl.ids == bad_slot
+    assert rows.any() and (~rows).any()
+    assert np.array_equal(Yb[rows], wl.Y_base[rows])
+    assert np.array_equal(Yb[~rows], Yc[~rows])
+
+
+def test_distinct_scales_reach_every_slot(H):
+    """Every slot carries its own alpha / r, and the result of each slot's tokens
+    follows that slot's scale: rescaling one slot's alpha changes only its rows,
+    by exactly the expected factor within the tolerance."""
+    import torch
+    wl = W.random_small(seed=73, T=48, d_in=128, d_out=96, S=8, ranks=(4, 16, 33), p_none=0.0)
+    sc = wl.scales_f32()
+    used = np.unique(wl.ids)
+    assert len(np.unique(sc[used])) >= 3           # the generator gives slots different scales
+    Y1, err, layer = _run_apply(H, wl)
+    assert err == 0
+    ref, _ = U.oracle_full(wl)
+    U.assert_parity(Y1, ref, wl.Y_base)
+    k = int(used[0])
+    layer.scales[k] = float(sc[k]) * 3.0
+    X, Y, ids = U.dev_inputs(wl)
+    layer.apply(X, Y, ids)
+    torch.cuda.synchronize()
+    Y2 = Y.cpu().numpy()
+    rows = wl.ids == k
+    assert np.array_equal(Y2[~rows], Y1[~rows])
+    d1 = Y1[rows].astype(np.float64) - wl.Y_base[rows]
+    d2 = Y2[rows].astype(np.float64) - wl.Y_base[rows]
+    assert np.abs(d2 - 3.0 * d1).max() <= 1e-4 * np.abs(d1).max() + 1e-6

@@ -88,7 +88,7 @@ def pin_merge_identity(apply, seed=11):
     ok = err == 0
     for t in range(X.shape[0]):
         i = ids[t]
-        Wm = W0 + np.float64(sc[i]) * (A[i].astype(np.float64) @ B[i].astype(np.float64))
+        Wm = O.merged_weight(W0, A[i], B[i], sc[i])
         ref = X[t].astype(np.float64) @ Wm - (X[t].astype(np.float64) @ W0) + Yb32[t]
         ok &= np.allclose(Y[t], ref, rtol=1e-12, atol=1e-12)
     return bool(ok)
@@ -195,6 +195,34 @@ PINS = [pin_hand_example, pin_merge_identity, pin_one_adapter_dense, pin_zero_b,
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
 def test_oracle_pin(impl, pin):
     assert pin(IMPLS[impl])
+
+
+def test_merged_weight_selector_closed_form():
+    """merged_weight(W0, [I_r; 0], [I_r 0], s) = W0 + s E_r, with E_r the identity on
+    the leading r x r block and zero elsewhere (d_in != d_out, s not 1)."""
+    rng = np.random.default_rng(31)
+    d_in, d_out, r, s = 11, 9, 4, np.float32(0.375)
+    W0 = rng.standard_normal((d_in, d_out))
+    A = np.zeros((d_in, r), np.float32)
+    A[:r, :r] = np.eye(r)
+    B = np.zeros((r, d_out), np.float32)
+    B[:r, :r] = np.eye(r)
+    E = np.zeros((d_in, d_out))
+    E[:r, :r] = np.eye(r)
+    assert np.array_equal(O.merged_weight(W0, A, B, s), W0 + 0.375 * E)
+
+
+def test_merged_weight_rank1_closed_form():
+    """A rank-1 adapter a b^T merges to W0 + s a b^T, element by element."""
+    rng = np.random.default_rng(32)
+    a = W.bf16_round(rng.standard_normal((7, 1)).astype(np.float32))
+    b = W.bf16_round(rng.standard_normal((1, 5)).astype(np.float32))
+    W0 = rng.standard_normal((7, 5))
+    s = np.float32(1.25)
+    got = O.merged_weight(W0, a, b, s)
+    for j in range(7):
+        for c in range(5):
+            assert got[j, c] == W0[j, c] + 1.25 * (float(a[j, 0]) * float(b[0, c]))
 
 
 def test_c_and_numpy_oracles_agree_on_generated_workload():
@@ -339,13 +367,15 @@ def _mutant(kind):
             if kind == "first_token_adapter":
                 j = int(ids[0]) if int(ids[0]) >= 0 else i
                 a, b = A[j].astype(np.float64), B[j].astype(np.float64)
+            if kind == "neighbour_scale":
+                s = np.float64(sc[(i + 1) % S])
             Y[t] += s * ((x @ a) @ b)
         return Y, err
     return apply
 
 
 MUTANTS = ["no_scale", "scale_times_r", "sign", "drop_last_rank", "rank_shift",
-           "reversed_x", "neighbour_adapter", "skip_ybase", "first_token_adapter"]
+           "reversed_x", "neighbour_adapter", "skip_ybase", "first_token_adapter", "neighbour_scale"]
 
 
 @pytest.mark.parametrize("kind", MUTANTS)

@@ -16,7 +16,11 @@ Shapes follow the workloads of the pages:
 
 Value recipe (all configs): X, A, B ~ N(0,1)/sqrt(fan_in) rounded to bf16 by
 round-to-nearest-even (torch ``.to(bfloat16)``), fan_in = d_in for X and A and
-r for B; Y_base ~ N(0,1) in fp32; alpha = 2r so alpha/r = 2.
+r for B; Y_base ~ N(0,1) in fp32.  alpha: the tiny correctness case fixes
+alpha = 2r; elsewhere the configs leave it open, and every slot draws its own
+alpha from {r/2, 3r/2, 3r, 7, 2.9r} (fp32 values), so that neighbouring slots
+carry different scales alpha/r and a kernel that reads another slot's scale
+fails parity.
 """
 from __future__ import annotations
 
@@ -56,13 +60,28 @@ class Adapter:
     B: np.ndarray  # [r, d_out] float32 holding bf16 values
 
 
+def draw_alphas(seed: int, ranks) -> np.ndarray:
+    """One alpha per slot (fp32), drawn from {r/2, 3r/2, 3r, 7, 2.9r}; 0 for an empty slot."""
+    r = np.asarray(ranks, dtype=np.int32)
+    rf = r.astype(np.float32)
+    table = np.stack([np.float32(0.5) * rf, np.float32(1.5) * rf, np.float32(3.0) * rf,
+                      np.full_like(rf, np.float32(7.0)), np.float32(2.9) * rf]).astype(np.float32)
+    pick = np.random.default_rng([seed, 7]).integers(0, table.shape[0], size=len(r))
+    a = table[pick, np.arange(len(r))].astype(np.float32)
+    a[r <= 0] = 0
+    return a
+
+
 class Adapters:
     """Per-slot adapters, each drawn from its own seed on first access, so a
-    large resident pool never has to be held in host memory at once."""
+    large resident pool never has to be held in host memory at once.
+    alphas: fp32 alpha per slot (default: draw_alphas(seed, ranks))."""
 
-    def __init__(self, seed: int, d_in: int, d_out: int, ranks: np.ndarray, cache: bool = True):
+    def __init__(self, seed: int, d_in: int, d_out: int, ranks: np.ndarray, cache: bool = True, alphas=None):
         self.seed, self.d_in, self.d_out = seed, d_in, d_out
         self.rank_of = np.asarray(ranks, dtype=np.int32)
+        self.alpha_of = (draw_alphas(seed, self.rank_of) if alphas is None
+                         else np.asarray(alphas, dtype=np.float32).copy())
         self._cache = {} if cache else None
 
     def __len__(self) -> int:
@@ -78,7 +97,7 @@ class Adapters:
         rng = np.random.default_rng([self.seed, 100, i])
         A = bf16_round(rng.standard_normal((self.d_in, r), dtype=np.float32) / np.float32(np.sqrt(self.d_in)))
         B = bf16_round(rng.standard_normal((r, self.d_out), dtype=np.float32) / np.float32(np.sqrt(r)))
-        ad = Adapter(rank=r, alpha=2.0 * r, A=A, B=B)
+        ad = Adapter(rank=r, alpha=float(self.alpha_of[i]), A=A, B=B)
         if self._cache is not None:
             self._cache[i] = ad
         return ad
@@ -112,12 +131,16 @@ class Workload:
     def ranks(self) -> np.ndarray:
         return self.adapters.rank_of.copy()
 
+    def alphas(self) -> np.ndarray:
+        return self.adapters.alpha_of.copy()
+
     def scales_f32(self) -> np.ndarray:
-        """alpha/r per slot (alpha = 2r), rounded once to fp32; both sides widen this value."""
+        """alpha/r per slot, one fp32 division (as the library's loader does it);
+        both sides widen this value."""
         r = self.adapters.rank_of
         out = np.zeros(len(r), dtype=np.float32)
         nz = r > 0
-        out[nz] = np.float32(2.0) * r[nz].astype(np.float32) / r[nz].astype(np.float32)
+        out[nz] = self.adapters.alpha_of[nz] / r[nz].astype(np.float32)
         return out
 
     def distinct(self) -> int:
@@ -143,7 +166,7 @@ def _assign_pages(seed: int, ranks: np.ndarray, extra_pages: int = 3):
     return pid, n_pool, n_pool
 
 
-def _finish(name, seed, d_in, d_out, ids, ranks) -> Workload:
+def _finish(name, seed, d_in, d_out, ids, ranks, alphas=None) -> Workload:
     T = len(ids)
     rx = np.random.default_rng([seed, 2])
     X = bf16_round(rx.standard_normal((T, d_in), dtype=np.float32) / np.float32(np.sqrt(d_in)))
@@ -153,7 +176,7 @@ def _finish(name, seed, d_in, d_out, ids, ranks) -> Workload:
     pid, na, nb = _assign_pages(seed, ranks)
     return Workload(name=name, d_in=d_in, d_out=d_out, X=X, Y_base=Y_base,
                     ids=np.ascontiguousarray(ids, dtype=np.int32),
-                    adapters=Adapters(seed, d_in, d_out, ranks, cache=len(ranks) <= 256),
+                    adapters=Adapters(seed, d_in, d_out, ranks, cache=len(ranks) <= 256, alphas=alphas),
                     page_ids=pid, pages_a=na, pages_b=nb)
 
 
@@ -162,10 +185,12 @@ def _finish(name, seed, d_in, d_out, ids, ranks) -> Workload:
 # ---------------------------------------------------------------------------
 
 def tiny(seed: int = 0) -> Workload:
-    """d_in = d_out = 256, 8 decode tokens, 3 adapters of rank 4, 8, 16, uniform ids."""
+    """d_in = d_out = 256, 8 decode tokens, 3 adapters of rank 4, 8, 16, uniform ids,
+    alpha = 2r (the one config that fixes alpha)."""
     rng = np.random.default_rng([seed, 1])
     ids = rng.integers(0, 3, size=8)
-    return _finish("tiny_d256_T8", seed, 256, 256, ids, [4, 8, 16])
+    ranks = [4, 8, 16]
+    return _finish("tiny_d256_T8", seed, 256, 256, ids, ranks, alphas=[2.0 * r for r in ranks])
 
 
 def decode_q_proj_7b(seed: int = 1, T: int = 64) -> Workload:
