@@ -9,9 +9,13 @@ layer).  The ring's footprint is more than 4x the L2 cache, so every layer's
 weights and activations come from HBM.  The step is captured once in a CUDA
 graph and replayed.  value = tokens x layers x steps / device time.
 
-Default workload: 7B decode q_proj, d_in = d_out = 4096, 64 tokens (one per
-sequence), 32 resident rank-16 adapters with Zipf(1.0) popularity, bf16
-weights in 16-row pages with shuffled page order, fp32 Y_base.
+Default (headline) workload: the largest single-GPU configuration, the 8B
+sweep with every token on a distinct adapter at T = 1024 (d_in = 4096,
+d_out = 14336, rank 64, 512 resident adapters, 1.33 GB of algorithmic bytes
+per layer).  The same JSON line carries `per_config`: kernel time, algorithmic
+bytes and the fraction of the measured HBM peak for every other configuration
+(7B decode q_proj, mixed-rank MLP up and down, prefill with its tensor-pipe
+fraction, the 8B sweep at T = 1, 64, 1024 in both regimes).
 
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of the same workload.
@@ -43,7 +47,7 @@ def parse():
     p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="decode_q_proj_7b",
+    p.add_argument("--workload", default="sweep_8b_distinct_T1024",
                    help="decode_q_proj_7b | mixed_mlp_up | mixed_mlp_down | prefill | sweep_8b_one_T<n> | sweep_8b_distinct_T<n>")
     p.add_argument("--layers", type=int, default=0, help="ring size (0 = enough for > 4x L2)")
     p.add_argument("--projections", type=int, default=1,
@@ -51,7 +55,16 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-per-config", action="store_true")
+    p.add_argument("--per-config", default=",".join(PER_CONFIG),
+                   help="comma-separated workloads measured into the per_config object")
     return p.parse_args()
+
+
+# Every configuration of the workload list; the headline is the largest.
+PER_CONFIG = ["decode_q_proj_7b", "mixed_mlp_up", "mixed_mlp_down", "prefill",
+              "sweep_8b_one_T1", "sweep_8b_one_T64", "sweep_8b_one_T1024",
+              "sweep_8b_distinct_T1", "sweep_8b_distinct_T64", "sweep_8b_distinct_T1024"]
 
 
 # ---------------------------------------------------------------------------
@@ -157,7 +170,7 @@ class ClockSampler:
 # CPU oracle timing (cpu_baseline and --impl reference)
 # ---------------------------------------------------------------------------
 
-def time_oracle(wl, seconds: float):
+def time_oracle(wl, seconds: float, max_flops: float = 2.5e8):
     """Run the fp64 C oracle on the workload's batch until `seconds` of work
     (at least one call); returns (tokens/s per layer, threads, sample text)."""
     from oracle import build_oracle as OC
@@ -165,8 +178,8 @@ def time_oracle(wl, seconds: float):
     # bounded sample: whole batch when small, else the first tokens of it
     n_tok = T
     est = algorithmic_flops(wl)
-    if est > 4e9:
-        n_tok = max(1, int(T * 4e9 / est))
+    if est > max_flops:
+        n_tok = max(1, int(T * max_flops / est))
     tok = np.arange(n_tok)
     import workloads as W
     X, Yb, ids, A, B, sc = W.subset_for_tokens(wl, tok)
@@ -182,6 +195,21 @@ def time_oracle(wl, seconds: float):
     value = n_tok * calls / el
     sample = f"{calls} oracle calls of {n_tok} tokens ({wl.name}), {el:.1f} s"
     return value, threads, sample
+
+
+def ring_layers(wl, layers_arg: int = 0, factor: float = 4.2) -> int:
+    """Independent layer instances so that one step's footprint exceeds factor x L2."""
+    per_layer = (wl.pages_a * 16 * wl.d_in * 2 + wl.pages_b * 16 * wl.d_out * 2
+                 + wl.T * (wl.d_in * 2 + wl.d_out * 4))
+    return layers_arg or max(8, min(256, math.ceil(factor * L2_BYTES / per_layer)))
+
+
+def bench_config(wl, desc: str, layers_arg: int = 0) -> dict:
+    """The workload's config object, identical on both arms."""
+    n = ring_layers(wl, layers_arg)
+    return {"workload": desc, "tokens": wl.T, "distinct_adapters": wl.distinct(),
+            "l2": f"inputs larger than L2: a ring of {n} independent layer instances "
+                  f"(over 4 x the 126 MB L2) replayed back to back"}
 
 
 def run_reference(args):
@@ -205,7 +233,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * el / max(1, args.steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": desc},
+        "config": bench_config(wl, desc),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -283,6 +311,23 @@ class Ring:
             n += H.lora_last_launch_count()
         return n
 
+    def plan_only(self, reps: int, stream=None) -> int:
+        """The batch's plan, `reps` times (timing of the plan kernel)."""
+        n = 0
+        for _ in range(reps):
+            self.layers[0].plan(self.ids, ws=self.ws, stream=stream)
+            n += self.H.lora_last_launch_count()
+        return n
+
+    def apply_calls(self, reps: int, stream=None) -> int:
+        """lora_apply (plan + compute in one call) on the first min(reps, layers) layers."""
+        n = 0
+        for lay, X, Y in list(zip(self.layers, self.X, self.Y))[:reps]:
+            self.H.lora_apply(X, Y, self.T, lay.d_in, lay.d_out, self.ids, lay.S, lay.ranks, lay.scales,
+                              lay.page_table, lay.pool_a, lay.pool_b, self.ws, lay.err, stream)
+            n += self.H.lora_last_launch_count()
+        return n
+
     def step_groups_separate(self, P: int, stream=None) -> int:
         """The same work as step_groups(plan=False) with one launch per layer."""
         n = 0
@@ -293,44 +338,138 @@ class Ring:
         return n
 
 
+# workload -> profile summary of its dominant kernel (each names the kernel source it was captured from)
 PROFILE_FOR = {
-    # workload -> (profile summary, kernel source it was captured from)
-    "decode_q_proj_7b": ("profiles/gather_kernel_decode_q_proj_7b.md",
-                         "heterogeneous_adapter_batching_b200/csrc/lora_gather.cu"),
-    "mixed_mlp_up": ("profiles/gather_kernel_mixed_mlp_up.md",
-                     "heterogeneous_adapter_batching_b200/csrc/lora_gather.cu"),
-    "prefill": ("profiles/tiles_kernel_prefill.md", "heterogeneous_adapter_batching_b200/csrc/lora_tiles.cu"),
+    "decode_q_proj_7b": "profiles/gather_kernel_decode_q_proj_7b.md",
+    "mixed_mlp_up": "profiles/gather_kernel_mixed_mlp_up.md",
+    "prefill": "profiles/tiles_kernel_prefill.md",
 }
+
+
+def source_digest(path: str) -> str:
+    """sha256 of a CUDA source with its comments and blank lines removed, so that
+    a comment-only edit keeps the digest of the code a profile was taken from."""
+    import hashlib
+    import re
+    text = open(path, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    lines = [ln.rstrip() for ln in text.splitlines() if ln.strip()]
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()
+
+
+def profile_fields(prof_rel: str) -> dict:
+    fields = {}
+    for line in open(os.path.join(ROOT, prof_rel)):
+        if ":" in line and not line.startswith(("#", "|", " ")):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    return fields
 
 
 def profiled_traffic(workload: str):
     """DRAM bytes per launch of the dominant kernel from the committed ncu summary,
-    or None when there is none or the kernel source changed since the capture."""
-    import hashlib
+    or None when there is none or the kernel's code changed since the capture."""
     if workload not in PROFILE_FOR:
         return None
-    prof, src = (os.path.join(ROOT, x) for x in PROFILE_FOR[workload])
     try:
-        fields = {}
-        for line in open(prof):
-            if ":" in line and not line.startswith(("#", "|", " ")):
-                k, v = line.split(":", 1)
-                fields[k.strip()] = v.strip()
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
-        if fields.get("source_sha256") != sha:
+        f = profile_fields(PROFILE_FOR[workload])
+        if f.get("source_digest") != source_digest(os.path.join(ROOT, f["source"])):
             return None
-        return int(fields["traffic_bytes_per_launch"])
+        return int(f["traffic_bytes_per_launch"])
     except Exception:
         return None
 
 
 def measured_peaks():
+    """(HBM GB/s, bf16 TFLOP/s sustained, source)."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
+        tf = d.get("bf16_tflops_sustained", d.get("bf16_tflops"))
+        return float(d["hbm_gbs"]), float(tf), "measured"
     except Exception:
-        return 6650.0, "fallback"
+        return 6650.0, 1400.0, "fallback"
+
+
+def _time_graph(graph, reps: int, stream) -> float:
+    """Mean ms per replay of a captured graph, CUDA events on the replay stream."""
+    import torch
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream()
+    e0.record(cur)
+    for _ in range(reps):
+        graph.replay()
+    e1.record(cur)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def _capture(fn, stream):
+    import torch
+    with torch.cuda.stream(stream):
+        fn(stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        n = fn(stream)
+    torch.cuda.synchronize()
+    return g, n
+
+
+def kernel_times(ring, stream, reps: int, H, P: int = 1):
+    """Per-layer device times, at the library's default options, of the ring's
+    compute launches (the plan already in ring.ws), of the plan alone, and of one
+    lora_apply call (plan + compute)."""
+    n_valid, n_seg, n_jobs, n_tiles = (int(x) for x in ring.ws[:16].cpu().numpy().view(np.int32)[:4])
+    fn = ring.apply_only if P == 1 else (lambda s: ring.step_groups(P, s, plan=False))
+    g_apply, launches = _capture(fn, stream)
+    n_layers = len(ring.layers)
+    apply_ms = _time_graph(g_apply, reps, stream)
+    g_plan, _ = _capture(lambda s: ring.plan_only(8, s), stream)
+    plan_ms = _time_graph(g_plan, reps, stream) / 8
+    g_one, _ = _capture(lambda s: ring.apply_calls(8, s), stream)
+    one_ms = _time_graph(g_one, reps, stream) / min(8, n_layers)
+    del g_apply, g_plan, g_one
+    ring.layers[0].plan(ring.ids, ws=ring.ws, stream=stream)
+    torch_sync()
+    return {"kernel_us": apply_ms * 1000.0 / n_layers, "plan_us": plan_ms * 1000.0,
+            "lora_apply_us": one_ms * 1000.0, "launches_per_layer": launches / n_layers,
+            "gather_jobs": n_jobs, "tensor_tiles": n_tiles}
+
+
+def torch_sync():
+    import torch
+    torch.cuda.synchronize()
+
+
+def measure_config(name: str, dev, stream, H, reps: int, peak_gbs: float, peak_tf: float) -> dict:
+    """One per_config entry: a ring over 2.5 x L2, the plan once, the compute launches timed."""
+    import torch
+    wl, desc = workload_spec(name)
+    ring = Ring(wl, ring_layers(wl, 0, factor=2.5), seed=4321, device=dev)
+    with torch.cuda.stream(stream):
+        ring.layers[0].plan(ring.ids, ws=ring.ws, stream=stream)
+    torch.cuda.synchronize()
+    kt = kernel_times(ring, stream, reps, H)
+    alg = algorithmic_bytes(wl)
+    flops = algorithmic_flops(wl)
+    us = kt["kernel_us"]
+    out = {"tokens": wl.T, "distinct_adapters": wl.distinct(), "layers": len(ring.layers),
+           "kernel_us": us, "algorithmic_bytes": alg, "achieved_gbs": alg / (us * 1e-6) / 1e9,
+           "frac": alg / (us * 1e-6) / 1e9 / peak_gbs, "tokens_per_s": wl.T / (us * 1e-6),
+           "plan_us": kt["plan_us"], "lora_apply_us": kt["lora_apply_us"],
+           "launches_per_layer": kt["launches_per_layer"],
+           "plan": {"gather_jobs": kt["gather_jobs"], "tensor_tiles": kt["tensor_tiles"]}}
+    if kt["tensor_tiles"] > 0:
+        out["tensor_tflops"] = flops / (us * 1e-6) / 1e12
+        out["tensor_frac"] = out["tensor_tflops"] / peak_tf
+    del ring
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_gpu(args):
@@ -353,44 +492,18 @@ def run_gpu(args):
     H.load_library()
 
     wl, desc = workload_spec(args.workload)
-    per_layer = (wl.pages_a * 16 * wl.d_in * 2 + wl.pages_b * 16 * wl.d_out * 2 + wl.T * (wl.d_in * 2 + wl.d_out * 4))
-    n_layers = args.layers or max(8, min(256, math.ceil(4.2 * L2_BYTES / per_layer)))
     P = max(1, args.projections)
+    n_layers = ring_layers(wl, args.layers)
     n_layers = (n_layers + P - 1) // P * P
     ring = Ring(wl, n_layers, seed=1234 + rank, device=dev)
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
-    # capture one step in a CUDA graph
+    # one step = the plan of the batch + every layer's compute, captured once
     step = ring.step if P == 1 else (lambda s: ring.step_groups(P, s))
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            step(stream)
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        launches_per_step = step(stream)
+    graph, launches_per_step = _capture(step, stream)
     graph.replay()
     torch.cuda.synchronize()
-    n_valid, n_seg, n_jobs, n_tiles = (int(x) for x in ring.ws[:16].cpu().numpy().view(np.int32)[:4])
-    # The dominant kernel is timed alone: the gather kernel when the plan has no
-    # tiles (the tile launch is then skipped by planning with no long segments),
-    # else the pair of compute launches of every layer.
-    old_thresh = H.lora_get_option(H.OPT_LONG_SEGMENT)
-    if n_tiles == 0:
-        H.lora_set_option(H.OPT_LONG_SEGMENT, 0)
-        ring.layers[0].plan(ring.ids, ws=ring.ws, stream=stream)
-    graph_apply = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_apply, stream=stream):
-        apply_launches = ring.apply_only(stream) if P == 1 else ring.step_groups(P, stream, plan=False)
-    graph_sep = None
-    if P > 1:
-        graph_sep = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph_sep, stream=stream):
-            ring.step_groups_separate(P, stream)
-    H.lora_set_option(H.OPT_LONG_SEGMENT, old_thresh)
-    torch.cuda.synchronize()
-
     for _ in range(max(args.warmup, 3)):
         graph.replay()
     torch.cuda.synchronize()
@@ -409,27 +522,8 @@ def run_gpu(args):
     ev1.record(cur)
     torch.cuda.synchronize()
     elapsed_ms = ev0.elapsed_time(ev1)
-    # dominant kernel: the fused gather kernel, one launch per layer (plan excluded)
-    for _ in range(3):
-        graph_apply.replay()
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    k_apply = max(10, args.steps)
-    a0.record(cur)
-    for _ in range(k_apply):
-        graph_apply.replay()
-    a1.record(cur)
-    torch.cuda.synchronize()
-    apply_ms = a0.elapsed_time(a1)
-    sep_ms = None
-    if graph_sep is not None:
-        for _ in range(3):
-            graph_sep.replay()
-        a0.record(cur)
-        for _ in range(k_apply):
-            graph_sep.replay()
-        a1.record(cur)
-        torch.cuda.synchronize()
-        sep_ms = a0.elapsed_time(a1)
+    # the dominant kernels alone: one layer's compute launches (plan excluded)
+    kt = kernel_times(ring, stream, max(10, args.steps), H, P)
     clk = clocks.stop()
     if world > 1:
         t = torch.tensor([elapsed_ms], device=dev)
@@ -442,18 +536,19 @@ def run_gpu(args):
     value = tokens_per_step * world * args.steps / (elapsed_ms / 1000.0)
     ms_per_step = elapsed_ms / args.steps
 
-    # roofline of the gather kernel (one launch = one layer, or one group of P layers)
-    per_launch_ms = apply_ms / (k_apply * (n_layers // P))
+    peak, peak_tf, peak_kind = measured_peaks()
+    per_launch_us = kt["kernel_us"] * P
     alg = algorithmic_bytes(wl) * P
-    achieved = alg / (per_launch_ms / 1000.0) / 1e9
-    peak, peak_kind = measured_peaks()
-    kname = "gather_kernel<apply>" if n_tiles == 0 else "gather_kernel<apply> + tiles_kernel"
+    achieved = alg / (per_launch_us * 1e-6) / 1e9
+    kname = "compute launches of one layer (plan excluded)"
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
             "traffic": profiled_traffic(args.workload), "peak_source": peak_kind, "kernel": kname,
-            "kernel_us": per_launch_ms * 1000.0, "algorithmic_bytes_per_launch": alg,
-            "launches_per_layer": apply_launches / n_layers}
+            "kernel_us": per_launch_us, "algorithmic_bytes_per_launch": alg,
+            "launches_per_layer": kt["launches_per_layer"], "plan_us": kt["plan_us"],
+            "lora_apply_us": kt["lora_apply_us"],
+            "plan": {"gather_jobs": kt["gather_jobs"], "tensor_tiles": kt["tensor_tiles"]}}
 
-    # end-to-end through the C ABI with host buffers (one layer per step)
+    # end to end through the C ABI with host buffers (one layer per step)
     e2e = None
     if not args.no_e2e:
         lay = ring.layers[0]
@@ -487,7 +582,18 @@ def run_gpu(args):
         h2d = Xh.numel() * 2 + Yh.numel() * 4 + Ih.numel() * 4
         e2e = {"value": T * world / (e2e_ms / 1000.0), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(Yout.numel() * 4), "ms_per_step": e2e_ms,
-               "path": "pinned H2D of X, Y_base, ids -> lora_apply (plan + fused kernel) -> D2H of Y, one layer"}
+               "path": "pinned H2D of X, Y_base, ids -> lora_apply (plan + compute kernels) -> D2H of Y, one layer"}
+
+    del graph
+    ring_footprint = ring.footprint()
+    del ring
+    torch.cuda.empty_cache()
+
+    per_config = None
+    if not args.no_per_config and world == 1:
+        per_config = {}
+        for name in [n for n in args.per_config.split(",") if n]:
+            per_config[name] = measure_config(name, dev, stream, H, max(10, args.steps), peak, peak_tf)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -496,7 +602,6 @@ def run_gpu(args):
 
     if world > 1:
         dist.barrier()
-        del graph, graph_apply
         dist.destroy_process_group()
 
     if rank == 0:
@@ -504,23 +609,17 @@ def run_gpu(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": desc, "tokens": T, "distinct_adapters": wl.distinct(),
-                       "plan": {"gather_jobs": n_jobs, "tensor_tiles": n_tiles},
-                       "layers_per_step": n_layers, "plans_per_step": 1,
-                       "l2": f"inputs larger than L2: ring of {n_layers} layer instances, "
-                             f"{ring.footprint() / 1e6:.0f} MB > 4 x 126 MB",
-                       "cuda_graph": True, "parallelism": f"replicas x{world} (no collective)"},
-
+            "config": bench_config(wl, desc, args.layers),
             "gpu_launches": int(launches_per_step * args.steps),
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "clocks": clk,
+            "step": {"layers_per_step": n_layers, "plans_per_step": 1, "cuda_graph": True,
+                     "ring_bytes": ring_footprint, "parallelism": f"replicas x{world} (no collective)",
+                     "projections_per_launch": P},
+            "per_config": per_config,
         }
-        if P > 1:
-            line["config"]["projections_per_launch"] = P
-            line["config"]["us_per_layer_one_launch_per_group"] = apply_ms * 1000.0 / (k_apply * n_layers)
-            line["config"]["us_per_layer_one_launch_per_layer"] = sep_ms * 1000.0 / (k_apply * n_layers)
         print(json.dumps(line), flush=True)
     return 0
 

@@ -51,4 +51,27 @@ def test_reference_arm_json_line():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
-    assert line["config"]["workload"].startswith("7B decode q_proj")
+    bench = _bench()
+    wl, desc = bench.workload_spec("sweep_8b_distinct_T1024")
+    assert line["config"] == bench.bench_config(wl, desc)      # the GPU arm prints the same object
+    assert line["config"]["workload"].startswith("8B sweep distinct")
+
+
+def test_source_digest_ignores_comments(tmp_path):
+    """A profile's traffic stays valid across comment-only edits of the kernel source
+    and is dropped when the code changes."""
+    bench = _bench()
+    a, b, c = tmp_path / "a.cu", tmp_path / "b.cu", tmp_path / "c.cu"
+    a.write_text("// head\nint f(int x) {  // tail\n  return x + 1;\n}\n")
+    b.write_text("/* another\n   block */\nint f(int x) {\n\n  return x + 1;   \n}\n")
+    c.write_text("int f(int x) {\n  return x + 2;\n}\n")
+    assert bench.source_digest(str(a)) == bench.source_digest(str(b)) != bench.source_digest(str(c))
+
+
+def test_profiled_traffic_matches_only_the_captured_code():
+    bench = _bench()
+    for wl_name, prof in bench.PROFILE_FOR.items():
+        f = bench.profile_fields(prof)
+        assert f["source"].endswith(".cu") and len(f["source_digest"]) == 64 and int(f["traffic_bytes_per_launch"]) > 0
+        same = bench.source_digest(os.path.join(ROOT, f["source"])) == f["source_digest"]
+        assert (bench.profiled_traffic(wl_name) is not None) == same
