@@ -11,6 +11,7 @@ namespace lora {
 namespace {
 std::atomic<int> g_long_segment{128};
 std::atomic<int> g_job_tokens{LORA_MAX_JOB_TOKENS};
+std::atomic<int> g_gather_path{LORA_GATHER_AUTO};
 thread_local int t_launches = 0;
 thread_local const char *t_last_cuda_error = "no error";
 
@@ -39,6 +40,7 @@ __global__ void read_row_kernel(const uint16_t *pool, int width, const int32_t *
 
 int opt_long_segment() { return g_long_segment.load(); }
 int opt_job_tokens() { return g_job_tokens.load(); }
+int opt_gather_path() { return g_gather_path.load(); }
 
 int cuda_check(cudaError_t e) {
     if (e == cudaSuccess) return LORA_OK;
@@ -274,11 +276,49 @@ static GatherProj gather_proj(float *Y, int d_out, const int32_t *ranks, const f
     return g;
 }
 
-// The apply kernels over a plan already in ws: one gather launch for every
-// projection, then (when the plan has long runs) one tile launch per projection.
+// The tensor-core launches of a plan with long runs: one per projection.
+static int run_tiles(const uint16_t *X, int T, int d_in, const lora_projection_t *pr, int nproj, const PlanOut &o,
+                     int32_t *err_dev, cudaStream_t st) {
+    if (!plan_uses_tiles(T)) return LORA_OK;
+    for (int p = 0; p < nproj; ++p) {
+        TileArgs ta = {};
+        ta.X = X; ta.Y = pr[p].Y; ta.T = T; ta.d_in = d_in; ta.d_out = pr[p].d_out;
+        ta.ranks = pr[p].ranks; ta.scales = pr[p].scales; ta.pt = pr[p].page_table; ta.pa = pr[p].pa;
+        ta.pb = pr[p].pb; ta.tiles = o.tiles; ta.hdr = o.header; ta.err = err_dev;
+        ta.rowsA = (long long)pr[p].pa->num_pages * LORA_PAGE_ROWS;
+        ta.rowsB = (long long)pr[p].pb->num_pages * LORA_PAGE_ROWS;
+        ta.long_thresh = opt_long_segment();
+        if (int rc = launch_tiles(ta, st, true)) return rc;
+    }
+    return LORA_OK;
+}
+
+// Which gather path a call takes (both give bit-identical results).
+static bool use_split(int nproj) {
+    const int p = opt_gather_path();
+    if (p == LORA_GATHER_SPLIT) return true;
+    if (p == LORA_GATHER_CLUSTER) return false;
+    return nproj == 1;
+}
+
+// The apply kernels over a plan already in ws: the short segments of every
+// projection through the gather path (one cluster-kernel launch for all
+// projections, or a shrink + expand pair per projection), then (when the plan
+// has long runs) one tile launch per projection.
 static int run_planned(const uint16_t *X, int T, int d_in, int num_slots, const lora_projection_t *pr, int nproj,
                        void *ws, int32_t *err_dev, cudaStream_t st) {
     const PlanOut o = plan_out(ws, T, num_slots, nullptr, nullptr);
+    if (use_split(nproj)) {
+        float *vpart = reinterpret_cast<float *>(static_cast<char *>(ws) + ws_layout(T, num_slots).vpart);
+        for (int p = 0; p < nproj; ++p) {
+            SplitArgs s = {};
+            s.X = X; s.Y = pr[p].Y; s.T = T; s.d_in = d_in; s.d_out = pr[p].d_out; s.S = num_slots;
+            s.ranks = pr[p].ranks; s.scales = pr[p].scales; s.pt = pr[p].page_table;
+            s.perm = o.perm_short; s.jobs = o.jobs; s.hdr = o.header; s.vpart = vpart; s.err = err_dev;
+            if (int rc = launch_split(s, pr[p].pa, pr[p].pb, st)) return rc;
+        }
+        return run_tiles(X, T, d_in, pr, nproj, o, err_dev, st);
+    }
     GatherArgs a = {};
     a.X = X; a.T = T; a.d_in = d_in; a.S = num_slots; a.nproj = nproj;
     lora_pool_s *pa[LORA_MAX_PROJECTIONS], *pb[LORA_MAX_PROJECTIONS];
@@ -289,17 +329,7 @@ static int run_planned(const uint16_t *X, int T, int d_in, int num_slots, const 
     }
     a.perm = o.perm_short; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
     if (int rc = launch_gather(kApply, a, pa, pb, st, true)) return rc;
-    if (plan_uses_tiles(T)) {
-        for (int p = 0; p < nproj; ++p) {
-            TileArgs ta = {};
-            ta.X = X; ta.Y = pr[p].Y; ta.T = T; ta.d_in = d_in; ta.d_out = pr[p].d_out;
-            ta.ranks = pr[p].ranks; ta.scales = pr[p].scales; ta.pt = pr[p].page_table; ta.pa = pr[p].pa;
-            ta.pb = pr[p].pb; ta.tiles = o.tiles; ta.hdr = o.header; ta.err = err_dev;
-            ta.rowsA = a.proj[p].rowsA; ta.rowsB = a.proj[p].rowsB; ta.long_thresh = opt_long_segment();
-            if (int rc = launch_tiles(ta, st, true)) return rc;
-        }
-    }
-    return LORA_OK;
+    return run_tiles(X, T, d_in, pr, nproj, o, err_dev, st);
 }
 
 static lora_projection_t one_proj(float *Y, int d_out, const int32_t *ranks, const float *scales,
@@ -444,6 +474,10 @@ int lora_set_option(int key, int value) {
             if (value < 1 || value > LORA_MAX_JOB_TOKENS) return LORA_ERR_INVALID_ARG;
             g_job_tokens.store(value);
             return LORA_OK;
+        case LORA_OPT_GATHER_PATH:
+            if (value < LORA_GATHER_AUTO || value > LORA_GATHER_SPLIT) return LORA_ERR_INVALID_ARG;
+            g_gather_path.store(value);
+            return LORA_OK;
     }
     return LORA_ERR_INVALID_ARG;
 }
@@ -452,6 +486,7 @@ int lora_get_option(int key) {
     switch (key) {
         case LORA_OPT_LONG_SEGMENT: return g_long_segment.load();
         case LORA_OPT_DECODE_JOB_TOKENS: return g_job_tokens.load();
+        case LORA_OPT_GATHER_PATH: return g_gather_path.load();
     }
     return LORA_ERR_INVALID_ARG;
 }

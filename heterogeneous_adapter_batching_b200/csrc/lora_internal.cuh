@@ -29,7 +29,10 @@ struct PlanHeader {
 };
 
 struct WsLayout {
-    size_t header, seg_start, perm, perm_short, run_start, run_end, jobs, tiles, total;
+    size_t header, seg_start, perm, perm_short, run_start, run_end, jobs, tiles;
+    size_t plan_total;   // bytes of the plan (everything above)
+    size_t vpart;        // split gather path: fp32 partials [4][T][LORA_MAX_RANK]
+    size_t total;
 };
 
 constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -47,6 +50,8 @@ constexpr WsLayout ws_layout(int T, int S) {
     l.run_end = o;    o = align_up(o + sizeof(int32_t) * t, 256);
     l.jobs = o;       o = align_up(o + 2 * sizeof(int4) * t, 256);   // two int4 per job
     l.tiles = o;      o = align_up(o + sizeof(int4) * t, 256);
+    l.plan_total = o;
+    l.vpart = o;      o = align_up(o + 4 * t * LORA_MAX_RANK * sizeof(float), 256);
     l.total = o;
     return l;
 }
@@ -87,6 +92,7 @@ int pool_tensor_map(lora_pool_s *pool, CUtensorMap *out);
 // Process-wide options.
 int opt_long_segment();
 int opt_job_tokens();
+int opt_gather_path();
 
 // Record a CUDA error and return LORA_ERR_CUDA, or LORA_OK.
 int cuda_check(cudaError_t e);
@@ -181,5 +187,22 @@ struct TileArgs {
 };
 int launch_tiles(const TileArgs &a, cudaStream_t st, bool pdl);
 bool tiles_supported();
+
+// Split gather path (shrink kernel writing per-quarter partials, then an
+// expand kernel), bit-identical to the cluster gather kernel in apply mode.
+struct SplitArgs {
+    const uint16_t *X;
+    float *Y;
+    int T, d_in, d_out, S;
+    const int32_t *ranks;
+    const float *scales;
+    const int32_t *pt;
+    const int32_t *perm;     // the plan's short-token list
+    const int4 *jobs;
+    const PlanHeader *hdr;
+    float *vpart;            // workspace region WsLayout::vpart
+    int32_t *err;
+};
+int launch_split(const SplitArgs &s, lora_pool_s *pa, lora_pool_s *pb, cudaStream_t st);
 
 }  // namespace lora

@@ -24,7 +24,7 @@ namespace {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[LORA_NOALLOC_SCRATCH_BYTES];
 
 // The scratch holds the whole plan of the largest call the entry point admits.
-static_assert(ws_layout(LORA_NOALLOC_MAX_TOKENS, LORA_MAX_SLOTS).total <= (size_t)LORA_NOALLOC_SCRATCH_BYTES,
+static_assert(ws_layout(LORA_NOALLOC_MAX_TOKENS, LORA_MAX_SLOTS).plan_total <= (size_t)LORA_NOALLOC_SCRATCH_BYTES,
               "LORA_NOALLOC_SCRATCH_BYTES is smaller than the plan of LORA_NOALLOC_MAX_TOKENS tokens and "
               "LORA_MAX_SLOTS slots");
 
@@ -65,7 +65,7 @@ extern "C" int lora_apply_noalloc(const uint16_t *X, float *Y, int T, int d_in, 
     if (T < 0 || num_slots < 1 || num_slots > LORA_MAX_SLOTS) return LORA_ERR_INVALID_ARG;
     if (T > LORA_NOALLOC_MAX_TOKENS) return LORA_ERR_TOO_LARGE;
     const WsLayout l = ws_layout(T, num_slots);
-    if (l.total > (size_t)LORA_NOALLOC_SCRATCH_BYTES) return LORA_ERR_TOO_LARGE;
+    if (l.plan_total > (size_t)LORA_NOALLOC_SCRATCH_BYTES) return LORA_ERR_TOO_LARGE;
     if (T > 0 && (!ids || !ranks)) return LORA_ERR_INVALID_ARG;
     if (!pa || !pb) return LORA_ERR_INVALID_ARG;
     if (pa->width != d_in || pb->width != d_out) return LORA_ERR_WIDTH_MISMATCH;
@@ -76,9 +76,12 @@ extern "C" int lora_apply_noalloc(const uint16_t *X, float *Y, int T, int d_in, 
     if (int rc = noalloc_scratch(&ws)) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
-    // Same launch sequence as lora_apply, with the plan kept in the scratch.
-    // Every word the compute kernels read is written by the plan kernel of the
-    // same call first, so nothing in the scratch has to start at zero.
+    // The launch sequence of lora_apply with the cluster gather kernel, which
+    // needs nothing beyond the plan (lora_apply may take the split gather path
+    // instead, whose result is bit-identical), and the plan kept in the
+    // scratch.  Every word the compute kernels read is written by the plan
+    // kernel of the same call first, so nothing in the scratch has to start at
+    // zero.
     const PlanOut o = plan_in_ws(ws, T, num_slots);
     const bool use_tiles = tiles_supported() && opt_long_segment() > 0 && T >= opt_long_segment();
     const int long_thresh = use_tiles ? opt_long_segment() : 0;
