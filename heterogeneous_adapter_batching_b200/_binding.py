@@ -42,7 +42,7 @@ MAX_PROJECTIONS = 8
 EXPORTS = [
     "lora_pool_create", "lora_pool_destroy", "lora_pool_free_pages", "lora_pool_num_pages",
     "lora_pool_load", "lora_pool_evict", "lora_pool_read_row", "lora_workspace_size",
-    "lora_plan", "lora_shrink", "lora_expand_add", "lora_apply", "lora_apply_planned", "lora_apply_noalloc",
+    "lora_plan", "lora_shrink", "lora_expand_add", "lora_expand_add_strided", "lora_apply", "lora_apply_planned", "lora_apply_noalloc",
     "lora_apply_multi", "lora_apply_multi_planned",
     "lora_slot_cache_create", "lora_slot_cache_destroy", "lora_slot_cache_acquire", "lora_slot_cache_unpin",
     "lora_slot_cache_invalidate", "lora_slot_cache_lookup", "lora_slot_cache_stats",
@@ -90,6 +90,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lora_plan": (I, [V, I, V, I, V, V, V, Z, V, V]),
         "lora_shrink": (I, [V, I, I, V, I, V, V, V, V, V, Z, V, V]),
         "lora_expand_add": (I, [V, V, I, I, V, I, V, V, V, V, V, Z, V, V]),
+        "lora_expand_add_strided": (I, [V, V, I, I, I, V, I, V, V, V, V, V, Z, V, V]),
         "lora_apply": (I, [V, V, I, I, I, V, I, V, V, V, V, V, V, Z, V, V]),
         "lora_apply_planned": (I, [V, V, I, I, I, I, V, V, V, V, V, V, Z, V, V]),
         "lora_apply_noalloc": (I, [V, V, I, I, I, V, I, V, V, V, V, V, V, V]),
@@ -224,6 +225,14 @@ def lora_expand_add(V, Y, T, d_out, ids, num_slots, ranks, scales, page_table, p
                     stream=None) -> None:
     _check("lora_expand_add", load_library().lora_expand_add(
         _p(V), _p(Y), T, d_out, _p(ids), num_slots, _p(ranks), _p(scales), _p(page_table), pb._h, _p(ws),
+        ws.numel() * ws.element_size(), _p(err), _s(stream)))
+
+
+def lora_expand_add_strided(V, Y, ldy, T, d_out, ids, num_slots, ranks, scales, page_table, pb: Pool, ws, err=None,
+                            stream=None) -> None:
+    """Y: a [T, d_out] column block of a wider fp32 tensor whose rows are ldy apart."""
+    _check("lora_expand_add_strided", load_library().lora_expand_add_strided(
+        _p(V), _p(Y), ldy, T, d_out, _p(ids), num_slots, _p(ranks), _p(scales), _p(page_table), pb._h, _p(ws),
         ws.numel() * ws.element_size(), _p(err), _s(stream)))
 
 

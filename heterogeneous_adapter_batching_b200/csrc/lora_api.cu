@@ -270,7 +270,7 @@ static bool plan_uses_tiles(int T) {
 static GatherProj gather_proj(float *Y, int d_out, const int32_t *ranks, const float *scales,
                               const int32_t *page_table, const lora_pool_s *pa, const lora_pool_s *pb) {
     GatherProj g = {};
-    g.Y = Y; g.d_out = d_out; g.ranks = ranks; g.scales = scales; g.pt = page_table;
+    g.Y = Y; g.d_out = d_out; g.ldy = d_out; g.ranks = ranks; g.scales = scales; g.pt = page_table;
     g.rowsA = pa ? (long long)pa->num_pages * LORA_PAGE_ROWS : 0;
     g.rowsB = pb ? (long long)pb->num_pages * LORA_PAGE_ROWS : 0;
     return g;
@@ -385,10 +385,18 @@ int lora_shrink(const uint16_t *X, int T, int d_in, const int32_t *ids, int num_
 int lora_expand_add(const float *V, float *Y, int T, int d_out, const int32_t *ids, int num_slots,
                     const int32_t *ranks, const float *scales, const int32_t *page_table, lora_pool_t pb, void *ws,
                     size_t ws_bytes, int32_t *err_dev, lora_stream_t stream) {
+    return lora_expand_add_strided(V, Y, d_out, T, d_out, ids, num_slots, ranks, scales, page_table, pb, ws, ws_bytes,
+                                   err_dev, stream);
+}
+
+int lora_expand_add_strided(const float *V, float *Y, int ldy, int T, int d_out, const int32_t *ids, int num_slots,
+                            const int32_t *ranks, const float *scales, const int32_t *page_table, lora_pool_t pb,
+                            void *ws, size_t ws_bytes, int32_t *err_dev, lora_stream_t stream) {
     reset_launch_count();
     if (int rc = check_common(T, num_slots, ids, ranks, ws, ws_bytes)) return rc;
     if (!pb) return LORA_ERR_INVALID_ARG;
     if (pb->width != d_out) return LORA_ERR_WIDTH_MISMATCH;
+    if (ldy < d_out || (ldy % 4) != 0) return LORA_ERR_INVALID_ARG;
     if (T == 0) return LORA_OK;
     if (!V || !Y || !scales || !page_table || !aligned(Y, 16)) return LORA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -397,6 +405,7 @@ int lora_expand_add(const float *V, float *Y, int T, int d_out, const int32_t *i
     GatherArgs a = {};
     a.V = const_cast<float *>(V); a.T = T; a.d_in = 8; a.S = num_slots; a.nproj = 1;
     a.proj[0] = gather_proj(Y, d_out, ranks, scales, page_table, nullptr, pb);
+    a.proj[0].ldy = ldy;
     a.perm = o.perm_short; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
     lora_pool_s *pp[1] = {pb};
     return launch_gather(kExpand, a, pp, pp, st, true);

@@ -389,7 +389,7 @@ gather_kernel(const __grid_constant__ GatherMaps<NP> maps, const __grid_constant
                  "l"(a.hdr), "l"(a.err), "r"(e_max));
     if (threadIdx.x < nproj) {
         const GatherProj &pr = a.proj[threadIdx.x];
-        asm volatile("" ::"l"(pr.Y), "r"(pr.d_out), "l"(pr.ranks), "l"(pr.scales), "l"(pr.pt), "l"(pr.rowsA),
+        asm volatile("" ::"l"(pr.Y), "r"(pr.d_out), "r"(pr.ldy), "l"(pr.ranks), "l"(pr.scales), "l"(pr.pt), "l"(pr.rowsA),
                      "l"(pr.rowsB));
     }
     // Small page tables, ranks and scales are staged in shared memory.  They
@@ -510,7 +510,7 @@ gather_kernel(const __grid_constant__ GatherMaps<NP> maps, const __grid_constant
         const int r = m.r, np = m.np;
         const UnitGeom g = unit_geom<MODE>(a, sm, pj, np, e, crank);
         float *const Yp = a.proj[pj].Y;
-        const int d_out = a.proj[pj].d_out;
+        const int ldy = a.proj[pj].ldy;   // row stride of Y (d_out unless the caller passed a column block)
         const int buf = iter & 1;
         const int cw = g.nb * kBoxCols;
         const int nt = (n + kNTok - 1) / kNTok;   // token tiles of 8
@@ -531,7 +531,7 @@ gather_kernel(const __grid_constant__ GatherMaps<NP> maps, const __grid_constant
         auto load_y = [&](int c0, int mt, int nmt, int j) {
             const int col = c0 + mt * 16 + 4 * rc;
             return (mt < nmt && rtok[j] >= 0 && col < g.out1)
-                       ? *reinterpret_cast<const float4 *>(Yp + (size_t)rtok[j] * d_out + col)
+                       ? *reinterpret_cast<const float4 *>(Yp + (size_t)rtok[j] * ldy + col)
                        : make_float4(0.f, 0.f, 0.f, 0.f);
         };
         float4 ya = make_float4(0.f, 0.f, 0.f, 0.f), yb = ya;   // token tile 0 of this tile and the next
@@ -794,7 +794,7 @@ gather_kernel(const __grid_constant__ GatherMaps<NP> maps, const __grid_constant
                                 const float4 dv = *reinterpret_cast<const float4 *>(
                                     ytile + h * (kYTileBytes / 4) + t * 16 + ((rc ^ (t & 3)) << 2));
                                 const float4 y = (jj == 0) ? (h == 0 ? ya : yb) : y1[h];
-                                *reinterpret_cast<float4 *>(Yp + (size_t)tok * d_out + col) =
+                                *reinterpret_cast<float4 *>(Yp + (size_t)tok * ldy + col) =
                                     make_float4(fmaf(sc, dv.x, y.x), fmaf(sc, dv.y, y.y), fmaf(sc, dv.z, y.z),
                                                 fmaf(sc, dv.w, y.w));
                             }

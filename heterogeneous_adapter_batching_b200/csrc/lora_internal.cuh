@@ -141,8 +141,9 @@ enum GatherMode { kApply = 0, kShrink = 1, kExpand = 2 };
 
 // One adapted projection of a gather launch: its output and slot tables.
 struct GatherProj {
-    float *Y;           // [T][d_out] fp32, in place
+    float *Y;           // [T][ldy] fp32, columns [0, d_out) updated in place
     int d_out;
+    int ldy;            // row stride of Y in elements (>= d_out, a multiple of 4)
     const int32_t *ranks;
     const float *scales;
     const int32_t *pt;

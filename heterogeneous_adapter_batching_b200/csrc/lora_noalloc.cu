@@ -89,7 +89,8 @@ extern "C" int lora_apply_noalloc(const uint16_t *X, float *Y, int T, int d_in, 
 
     GatherArgs a = {};
     a.X = X; a.T = T; a.d_in = d_in; a.S = num_slots; a.nproj = 1;
-    a.proj[0].Y = Y; a.proj[0].d_out = d_out; a.proj[0].ranks = ranks; a.proj[0].scales = scales;
+    a.proj[0].Y = Y; a.proj[0].d_out = d_out; a.proj[0].ldy = d_out; a.proj[0].ranks = ranks;
+    a.proj[0].scales = scales;
     a.proj[0].pt = page_table;
     a.proj[0].rowsA = (long long)pa->num_pages * LORA_PAGE_ROWS;
     a.proj[0].rowsB = (long long)pb->num_pages * LORA_PAGE_ROWS;

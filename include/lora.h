@@ -198,6 +198,18 @@ int lora_expand_add(const float *V, float *Y, int T, int d_out, const int32_t *i
                     lora_pool_t pb, void *ws, size_t ws_bytes, int32_t *err_dev,
                     lora_stream_t stream);
 
+/* lora_expand_add into a column block of a wider output: row t of the block
+ * starts at Y + t * ldy (ldy >= d_out, a multiple of 4; Y 16-byte aligned),
+ * and only its first d_out columns are updated.  Page "Multi-LoRA Serving in
+ * Production", section "S-LoRA TP Communication Optimization": for small
+ * ranks a row-parallel layer splits B by columns and exchanges the rank-r
+ * vector v; each rank then adds s v B_k into its own column block of the
+ * partial output before the layer's all-reduce.  LORA_ERR_INVALID_ARG for a
+ * bad ldy; otherwise as lora_expand_add. */
+int lora_expand_add_strided(const float *V, float *Y, int ldy, int T, int d_out, const int32_t *ids, int num_slots,
+                            const int32_t *ranks, const float *scales, const int32_t *page_table, lora_pool_t pb,
+                            void *ws, size_t ws_bytes, int32_t *err_dev, lora_stream_t stream);
+
 /* Fused shrink + expand-add: Y[t] += s_i (X[t] A_i) B_i for every token.
  *   X [T][d_in] bf16, Y [T][d_out] fp32 (holds Y_base = X W0 on entry, computed
  *   by the caller; page "Multi-LoRA Serving Architecture ... (2026)", section

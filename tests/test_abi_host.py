@@ -119,6 +119,11 @@ def test_load_and_apply_validation_before_any_cuda_call(lib):
     assert lib.lora_last_launch_count() == 0
     assert lib.lora_shrink(fake, 8, 32, fake, 4, fake, fake, pa, fake, ws, ws_n, None, s) == -3
     assert lib.lora_expand_add(fake, fake, 8, 64, fake, 4, fake, fake, fake, pb, ws, ws_n, None, s) == -3
+    # the strided expand: the pool's width must be d_out, the row stride >= d_out and a multiple of 4
+    assert lib.lora_expand_add_strided(fake, fake, 64, 8, 64, fake, 4, fake, fake, fake, pb, ws, ws_n, None, s) == -3
+    assert lib.lora_expand_add_strided(fake, fake, 30, 8, 32, fake, 4, fake, fake, fake, pb, ws, ws_n, None, s) == -1
+    assert lib.lora_expand_add_strided(fake, fake, 34, 8, 32, fake, 4, fake, fake, fake, pb, ws, ws_n, None, s) == -1
+    assert lib.lora_last_launch_count() == 0
     lib.lora_pool_destroy(pa)
     lib.lora_pool_destroy(pb)
 
