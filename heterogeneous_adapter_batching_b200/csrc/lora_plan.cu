@@ -30,7 +30,11 @@
 //                       job size chosen.
 // Invalid ids (outside [-1, S) or an empty slot) are dropped and flagged.
 //
-// One CTA of 1024 threads.  W warps (W * S <= 16384) own contiguous token
+// One CTA (256 threads for up to 1024 tokens, 512 up to 4096, 1024 beyond).
+// Up to 4096 tokens the kernel keeps ids, ranks, perm, perm_short, the run
+// bounds and seg_start in shared memory: the inputs cross from global memory
+// once and the outputs are written once, so the plan costs one memory round
+// trip plus its barriers.  W warps (W * S <= 16384) own contiguous token
 // ranges; per-warp counts live in a [slot][warp] table in shared memory whose
 // exclusive scan in slot-major order gives every warp the first output
 // position of its tokens of each slot; __match_any_sync ranks the lanes that
@@ -46,41 +50,58 @@
 namespace lora {
 namespace {
 
-constexpr int kPlanThreads = 1024;
+constexpr int kPlanMaxThreads = 1024;
 constexpr int kTableEntries = 16384;
+constexpr int kSmemTokens = 4096;      // batches up to this size plan in shared memory
+constexpr int kScanVals = 8;           // most values one block scan carries
 
-__device__ __forceinline__ int block_exclusive_scan(int v, int *warp_tot, int *total) {
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    int x = v;
+// Exclusive scan of N values per thread across the block (thread order);
+// totals[i] receives the sum of value i.  Every thread must call it.
+template <int N>
+__device__ __forceinline__ void block_scan(int (&v)[N], int *wsum, int *totals) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int x[N];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) warp_tot[wid] = x;
-    __syncthreads();
-    if (wid == 0) {
-        int w = (lane < (int)(blockDim.x >> 5)) ? warp_tot[lane] : 0;
-        int s = w;
+    for (int i = 0; i < N; ++i) {
+        x[i] = v[i];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            int y = __shfl_up_sync(0xffffffffu, s, o);
-            if (lane >= o) s += y;
+            const int y = __shfl_up_sync(0xffffffffu, x[i], o);
+            if (lane >= o) x[i] += y;
         }
-        warp_tot[lane] = s - w;  // exclusive warp offsets
-        if (lane == 31) *total = s;
+        if (lane == 31) wsum[i * 32 + wid] = x[i];
     }
     __syncthreads();
-    int r = warp_tot[wid] + x - v;
+    if (wid == 0) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+            const int w = lane < nw ? wsum[i * 32 + lane] : 0;
+            int s = w;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, s, o);
+                if (lane >= o) s += y;
+            }
+            wsum[i * 32 + lane] = s - w;   // exclusive warp offsets
+            if (lane == 31) totals[i] = s;
+        }
+    }
     __syncthreads();
-    return r;
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] = wsum[i * 32 + wid] + x[i] - v[i];
+    __syncthreads();   // wsum is reused by the next scan
+}
+
+__device__ __forceinline__ int block_exclusive_scan(int v, int *wsum, int *total) {
+    int a[1] = {v};
+    block_scan<1>(a, wsum, total);
+    return a[0];
 }
 
 __device__ __forceinline__ bool valid_id(int id, int S, const int32_t *ranks) {
     return id >= 0 && id < S && ranks[id] > 0;
 }
 
-// A break: token t starts a run of one slot, or has no valid adapter.
 // Gather jobs are ordered by rank class: 0 = 4 pages per matrix (rank 49-64;
 // an out-of-range rank counts here too), 1 = 3 pages, 2 = 2, 3 = 1 page.
 constexpr int kPlanRankClasses = 4;
@@ -89,12 +110,19 @@ __device__ __forceinline__ int rank_class(int r) {
     return np >= 4 ? 0 : (np <= 1 ? 3 : 4 - np);
 }
 
+// A break: token t starts a run of one slot, or has no valid adapter.
 __device__ __forceinline__ bool is_break(const int32_t *ids, int t, int id, bool ok) {
     return !ok || t == 0 || ids[t - 1] != id;
 }
 
-__global__ void __launch_bounds__(kPlanThreads, 1)
-plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ ranks, int S, int W,
+// Dynamic shared memory of the kernel (ints).
+__host__ __device__ constexpr size_t plan_smem_ints(int T, int S, int W, bool in_smem) {
+    return (size_t)S * W + (size_t)S + (in_smem ? (size_t)5 * T + 2 * (size_t)S + 1 : 0);
+}
+
+template <bool SMEM>
+__global__ void __launch_bounds__(kPlanMaxThreads, 1)
+plan_kernel(const int32_t *__restrict__ ids_g, int T, const int32_t *__restrict__ ranks_g, int S, int W,
             int long_thresh, int job_tokens, int clusters, PlanOut out, int32_t *err_dev) {
     // Let the dependent kernel's CTAs get resident while the plan runs; they
     // wait for this grid's completion before reading its output.
@@ -103,16 +131,35 @@ plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ 
     extern __shared__ int smem[];
     int *cnt = smem;                       // [S][W] per-warp counts, then scan offsets
     int *scnt = cnt + (size_t)S * W;       // [S] short tokens per slot
-    __shared__ int warp_tot[32];
-    __shared__ int s_total[12];
+    int *ids_s = scnt + S;                 // SMEM only: [T] ids, [S] ranks, [T] perm, [T] perm_short,
+    int *ranks_s = ids_s + T;              //   [T] run starts, [T] run ends, [S + 1] seg_start
+    int *perm_s = ranks_s + S;
+    int *psh_s = perm_s + T;
+    int *rs_s = psh_s + T;
+    int *re_s = rs_s + T;
+    int *seg_s = re_s + T;
+    __shared__ int wsum[kScanVals * 32];
+    __shared__ int s_total[16];
     __shared__ int wfirst[32], wlast[32], carry_l[32], carry_r[32];
 
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nthr = blockDim.x;
     const int n_entries = S * W;
     const bool runs = long_thresh > 0 && T >= long_thresh;
 
-    for (int e = tid; e < n_entries; e += blockDim.x) cnt[e] = 0;
-    for (int k = tid; k < S; k += blockDim.x) scnt[k] = 0;
+    const int32_t *ids = SMEM ? ids_s : ids_g;
+    const int32_t *ranks = SMEM ? ranks_s : ranks_g;
+    int32_t *perm = SMEM ? perm_s : out.perm;
+    int32_t *perm_short = SMEM ? psh_s : out.perm_short;
+    int32_t *run_start = SMEM ? rs_s : out.run_start;
+    int32_t *run_end = SMEM ? re_s : out.run_end;
+    int32_t *seg_start = SMEM ? seg_s : out.seg_start;
+
+    if (SMEM) {
+        for (int t = tid; t < T; t += nthr) ids_s[t] = ids_g[t];
+        for (int k = tid; k < S; k += nthr) ranks_s[k] = ranks_g[k];
+    }
+    for (int e = tid; e < n_entries; e += nthr) cnt[e] = 0;
+    for (int k = tid; k < S; k += nthr) scnt[k] = 0;
     __syncthreads();
 
     const int chunk = ((T + W - 1) / W + 31) / 32 * 32;
@@ -155,11 +202,11 @@ plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ 
 
     // Phase 2: exclusive scan of cnt in slot-major order; carries of the run scans.
     {
-        const int per = (n_entries + blockDim.x - 1) / blockDim.x;
+        const int per = (n_entries + nthr - 1) / nthr;
         const int e0 = tid * per, e1 = min(n_entries, e0 + per);
         int local = 0;
         for (int e = e0; e < e1; ++e) local += cnt[e];
-        int run = block_exclusive_scan(local, warp_tot, &s_total[0]);
+        int run = block_exclusive_scan(local, wsum, &s_total[0]);
         for (int e = e0; e < e1; ++e) { int c = cnt[e]; cnt[e] = run; run += c; }
         if (tid < W) {
             int cl = -1, cr = T;
@@ -171,13 +218,15 @@ plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ 
     }
     __syncthreads();
     const int n_valid = s_total[0];
-    for (int k = tid; k < S; k += blockDim.x) {
+    for (int k = tid; k < S; k += nthr) {
         const int st = cnt[k * W];
-        out.seg_start[k] = st;
+        seg_start[k] = st;
+        if (SMEM) out.seg_start[k] = st;
         if (out.seg_start_copy) out.seg_start_copy[k] = st;
     }
     if (tid == 0) {
-        out.seg_start[S] = n_valid;
+        seg_start[S] = n_valid;
+        if (SMEM) out.seg_start[S] = n_valid;
         if (out.seg_start_copy) out.seg_start_copy[S] = n_valid;
     }
     __syncthreads();   // the scatter below advances cnt in place
@@ -199,7 +248,7 @@ plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ 
             if (ok) {
                 m = __match_any_sync(act, id);
                 const int pos = cnt[id * W + wid] + __popc(m & lt_mask);
-                out.perm[pos] = t;
+                perm[pos] = t;
                 if (out.perm_copy) out.perm_copy[pos] = t;
             }
             __syncwarp();
@@ -222,7 +271,7 @@ plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ 
                     if (lane >= o) v = max(v, y);
                 }
                 v = max(v, carry);
-                if (t < hi) out.run_start[t] = v;
+                if (t < hi) run_start[t] = v;
                 carry = __shfl_sync(0xffffffffu, v, 31);
             }
             // next break after every token: suffix min, right to left.  The same
@@ -250,8 +299,8 @@ plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ 
                 nxt = min(nxt, rc);
                 if (t < hi) {
                     int end = -1;
-                    if (ok && nxt - out.run_start[t] >= long_thresh) end = nxt - 1;
-                    out.run_end[t] = end;
+                    if (ok && nxt - run_start[t] >= long_thresh) end = nxt - 1;
+                    run_end[t] = end;
                 }
                 rc = min(rc, __shfl_sync(0xffffffffu, incl, 0));
             }
@@ -262,19 +311,21 @@ plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ 
     // Phase 4: compact perm to the tokens outside long runs (perm_short) and
     // count them per slot.
     {
-        const int per = (n_valid + blockDim.x - 1) / blockDim.x;
+        const int per = (n_valid + nthr - 1) / nthr;
         const int p0 = tid * per, p1 = min(n_valid, p0 + per);
         int local = 0;
         for (int p = p0; p < p1; ++p) {
-            const int t = out.perm[p];
-            if (!runs || out.run_end[t] < 0) ++local;
+            const int t = perm[p];
+            if (!runs || run_end[t] < 0) ++local;
         }
-        int pos = block_exclusive_scan(local, warp_tot, &s_total[1]);
+        int pos = block_exclusive_scan(local, wsum, &s_total[1]);
         for (int p = p0; p < p1; ++p) {
-            const int t = out.perm[p];
-            if (!runs || out.run_end[t] < 0) {
-                out.perm_short[pos++] = t;
+            const int t = perm[p];
+            if (!runs || run_end[t] < 0) {
+                perm_short[pos] = t;
+                if (SMEM) out.perm_short[pos] = t;
                 atomicAdd(&scnt[ids[t]], 1);
+                ++pos;
             }
         }
     }
@@ -282,7 +333,7 @@ plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ 
 
     // Phase 5: gather jobs (per slot) and tensor tiles (per long run, token order).
     {
-        const int per = (S + blockDim.x - 1) / blockDim.x;   // <= 4 for S <= 4096
+        const int per = (S + nthr - 1) / nthr;
         const int k0 = tid * per, k1 = min(S, k0 + per);
         // Job size: the candidates are 4, 8 and the cap job_tokens (each at
         // most the cap).  The largest is taken that still gives min(jobs at
@@ -297,8 +348,7 @@ plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ 
             for (int i = 0; i < 3; ++i)
                 if (c > 0) njc[i] += (c + cand[i] - 1) / cand[i];
         }
-#pragma unroll
-        for (int i = 0; i < 3; ++i) (void)block_exclusive_scan(njc[i], warp_tot, &s_total[6 + i]);
+        block_scan<3>(njc, wsum, &s_total[6]);
         {
             const int want = min(s_total[6], clusters);
             int jt = cand[0];
@@ -308,30 +358,31 @@ plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ 
             job_tokens = jt;
         }
         // Jobs are written heaviest first: by pages per matrix (4, 3, 2, 1),
-        // then slot order.  The gather kernel hands units to clusters round
-        // robin, so this order places the long units first and the short ones
-        // fill in after them.
-        int sh_local = 0, ns_local = 0;
-        int njp[kPlanRankClasses] = {0, 0, 0, 0};
+        // then slot order.  The gather kernels hand units out round robin, so
+        // this order places the long units first and the short ones fill in
+        // after them.  One scan carries the short tokens before each slot, the
+        // jobs of each rank class before it and the slots present.
+        int vals[kPlanRankClasses + 2] = {0, 0, 0, 0, 0, 0};   // jobs per class, short tokens, slots present
         for (int k = k0; k < k1; ++k) {
             const int c = scnt[k];
-            sh_local += c;
-            if (c > 0) njp[rank_class(ranks[k])] += (c + job_tokens - 1) / job_tokens;
-            if (out.seg_start[k + 1] > out.seg_start[k]) ++ns_local;
+            vals[kPlanRankClasses] += c;
+            if (c > 0) vals[rank_class(ranks[k])] += (c + job_tokens - 1) / job_tokens;
+            if (seg_start[k + 1] > seg_start[k]) ++vals[kPlanRankClasses + 1];
         }
-        int sh_off = block_exclusive_scan(sh_local, warp_tot, &s_total[2]);
+        block_scan<kPlanRankClasses + 2>(vals, wsum, &s_total[6]);
+        int sh_off = vals[kPlanRankClasses];
         int j_off[kPlanRankClasses];
-#pragma unroll
-        for (int i = 0; i < kPlanRankClasses; ++i) j_off[i] = block_exclusive_scan(njp[i], warp_tot, &s_total[6 + i]);
-        (void)block_exclusive_scan(ns_local, warp_tot, &s_total[4]);
         {
             int base = 0;   // classes in order 0 (heaviest) .. 3
 #pragma unroll
             for (int i = 0; i < kPlanRankClasses; ++i) {
-                j_off[i] += base;
+                j_off[i] = vals[i] + base;
                 base += s_total[6 + i];
             }
-            if (tid == 0) s_total[3] = base;
+            if (tid == 0) {
+                s_total[3] = base;
+                s_total[4] = s_total[6 + kPlanRankClasses + 1];
+            }
         }
         for (int k = k0; k < k1; ++k) {
             const int c = scnt[k];
@@ -344,7 +395,7 @@ plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ 
                     const int q0 = sh_off + j * b + min(j, rem);
                     int tk[4];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) tk[i] = i < cc ? out.perm_short[q0 + i] : -1;
+                    for (int i = 0; i < 4; ++i) tk[i] = i < cc ? perm_short[q0 + i] : -1;
                     out.jobs[2 * (jo + j)] = make_int4(k, cc, q0, 0);
                     out.jobs[2 * (jo + j) + 1] = make_int4(tk[0], tk[1], tk[2], tk[3]);
                 }
@@ -352,23 +403,23 @@ plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ 
             }
             sh_off += c;
         }
-        __syncthreads();   // s_total[3] (the job count) is read below
+        __syncthreads();   // s_total[3], s_total[4] are read below
         // a token starts a tile when it lies in a long run at a multiple of kTileM
         // from the run's start
         int nt_local = 0;
-        const int tper = (T + blockDim.x - 1) / blockDim.x;
+        const int tper = (T + nthr - 1) / nthr;
         const int t0 = tid * tper, t1 = min(T, t0 + tper);
         if (runs) {
             for (int t = t0; t < t1; ++t) {
-                const int e = out.run_end[t];
-                if (e >= 0 && ((t - out.run_start[t]) % kTileM) == 0) ++nt_local;
+                const int e = run_end[t];
+                if (e >= 0 && ((t - run_start[t]) % kTileM) == 0) ++nt_local;
             }
         }
-        int t_off = block_exclusive_scan(nt_local, warp_tot, &s_total[5]);
+        int t_off = block_exclusive_scan(nt_local, wsum, &s_total[5]);
         if (runs) {
             for (int t = t0; t < t1; ++t) {
-                const int e = out.run_end[t];
-                if (e >= 0 && ((t - out.run_start[t]) % kTileM) == 0)
+                const int e = run_end[t];
+                if (e >= 0 && ((t - run_start[t]) % kTileM) == 0)
                     out.tiles[t_off++] = make_int4(ids[t], t, min(kTileM, e - t + 1), 0);
             }
         }
@@ -389,23 +440,33 @@ plan_kernel(const int32_t *__restrict__ ids, int T, const int32_t *__restrict__ 
 
 int launch_plan(const int32_t *ids, int T, const int32_t *ranks, int S, int long_thresh, int job_tokens,
                 const PlanOut &out, int32_t *err_dev, cudaStream_t st, int units_per_job) {
-    int W = 32;
+    const bool in_smem = T <= kSmemTokens;
+    const int threads = T <= 1024 ? 256 : (in_smem ? 512 : kPlanMaxThreads);
+    int W = threads / 32;
     while (W > 1 && W * S > kTableEntries) W >>= 1;
-    const size_t smem = sizeof(int) * ((size_t)S * W + (size_t)S);
+    const size_t smem = sizeof(int) * plan_smem_ints(T, S, W, in_smem);
     static bool attr_set[64] = {};
     int dev = 0;
     if (int rc = cuda_check(cudaGetDevice(&dev))) return rc;
     if (dev < 0 || dev >= 64) return LORA_ERR_INVALID_ARG;
     if (!attr_set[dev]) {
-        int rc = cuda_check(cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)(sizeof(int) * (kTableEntries + LORA_MAX_SLOTS))));
-        if (rc) return rc;
+        // the largest each variant asks for: a full table (W * S = 16384) and, in
+        // shared memory, kSmemTokens tokens and LORA_MAX_SLOTS slots
+        const int big = (int)(sizeof(int) * (kTableEntries + LORA_MAX_SLOTS));
+        const int big_s = (int)(sizeof(int) * (kTableEntries + LORA_MAX_SLOTS + 5 * kSmemTokens + 2 * LORA_MAX_SLOTS + 1));
+        if (int rc = cuda_check(cudaFuncSetAttribute(plan_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, big)))
+            return rc;
+        if (int rc = cuda_check(cudaFuncSetAttribute(plan_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, big_s)))
+            return rc;
         attr_set[dev] = true;
     }
     int clusters = 1;
     if (int rc = gather_clusters(&clusters)) return rc;
     clusters = max(1, clusters / max(1, units_per_job));
-    plan_kernel<<<1, kPlanThreads, smem, st>>>(ids, T, ranks, S, W, long_thresh, job_tokens, clusters, out, err_dev);
+    if (in_smem)
+        plan_kernel<true><<<1, threads, smem, st>>>(ids, T, ranks, S, W, long_thresh, job_tokens, clusters, out, err_dev);
+    else
+        plan_kernel<false><<<1, threads, smem, st>>>(ids, T, ranks, S, W, long_thresh, job_tokens, clusters, out, err_dev);
     count_launch();
     return cuda_check(cudaGetLastError());
 }

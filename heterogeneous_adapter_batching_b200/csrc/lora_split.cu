@@ -416,6 +416,18 @@ shrink_part_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     }
 }
 
+// Quarters of d_in that hold columns (d_in below 32 leaves some empty; an
+// empty quarter adds +0 to v in the cluster kernel, so skipping it in the sum
+// gives the same bits).
+__device__ __forceinline__ unsigned quarter_mask(int d_in) {
+    const unsigned Gi = (unsigned)d_in >> 3;
+    unsigned m = 0;
+#pragma unroll
+    for (int q = 0; q < kSlices; ++q)
+        if (Gi * (q + 1) / kSlices > Gi * q / kSlices) m |= 1u << q;
+    return m;
+}
+
 // d_out parts per job for this launch: enough units to fill the grid, few
 // enough that each unit still streams a long run of B columns.
 __device__ __forceinline__ int choose_parts(int n_jobs, int grid, int e_max) {
@@ -469,6 +481,7 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
         const int E = n_jobs > 0 ? choose_parts(n_jobs, gridDim.x, a.e_max) : 1;
         const int n_units = n_jobs * E;
         const long long Go = a.d_out >> 3;
+        const unsigned qmask = quarter_mask(a.d_in);
         int chunk = 0, nv = 0;
         bool ok = true, waited = false;
         auto wait_shrink = [&]() {
@@ -496,9 +509,9 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
             const int vb = nv & 1;
             auto issue_v = [&]() {
                 if (!wait_w(&sm.vempty[vb], ((nv >> 1) & 1) ^ 1, sm, a.err)) return false;
-                if (lane == 0) mbar_expect_tx(&sm.vfull[vb], (uint32_t)(kSlices * n * LORA_MAX_RANK * 4));
+                if (lane == 0) mbar_expect_tx(&sm.vfull[vb], (uint32_t)(__popc(qmask) * n * LORA_MAX_RANK * 4));
                 __syncwarp();
-                if (lane < kSlices)
+                if (lane < kSlices && ((qmask >> lane) & 1u))
                     bulk_load(sm.vst[vb][lane], a.vpart + ((size_t)lane * a.T + q0) * LORA_MAX_RANK,
                               (uint32_t)(n * LORA_MAX_RANK * 4), &sm.vfull[vb]);
                 ++nv;
@@ -560,6 +573,7 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
     // ------------------------------ consumers ------------------------------
     const int li = lane & 7, lj = lane >> 3, g8 = lane >> 2, tig = lane & 3;
     const uint32_t vt_base = smem_u32(sm.vt);
+    const unsigned qmask = quarter_mask(a.d_in);
     int chunk = 0, nunit = 0;
     while (true) {
         const int st = chunk % kStages;
@@ -579,7 +593,8 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
                 const int o = t * LORA_MAX_RANK + k;
                 float v = 0.f;
 #pragma unroll
-                for (int q = 0; q < kSlices; ++q) v += sm.vst[vb][q][o];
+                for (int q = 0; q < kSlices; ++q)
+                    if ((qmask >> q) & 1u) v += sm.vst[vb][q][o];
                 const uint16_t hv = bf16_rn(v);
                 const uint16_t lv = bf16_rn(v - __uint_as_float((uint32_t)hv << 16));
                 const uint32_t so = swz(t, LORA_MAX_RANK * 2, k >> 3) + (k & 7) * 2;
