@@ -5,4 +5,5 @@ include/lora.h; this package only marshals torch tensors into those calls.
 """
 from . import _binding
 from ._binding import *  # noqa: F401,F403
-from .layer import AdapterCache, AdapterLayer, apply_multi  # noqa: F401
+from .layer import AdapterCache, AdapterLayer, AdapterPrefetcher, PrefetchTicket, apply_multi  # noqa: F401
+from . import tp  # noqa: F401

@@ -276,21 +276,19 @@ static GatherProj gather_proj(float *Y, int d_out, const int32_t *ranks, const f
     return g;
 }
 
-// The tensor-core launches of a plan with long runs: one per projection.
+// The tensor-core launch of a plan with long runs: one for all projections.
 static int run_tiles(const uint16_t *X, int T, int d_in, const lora_projection_t *pr, int nproj, const PlanOut &o,
                      int32_t *err_dev, cudaStream_t st) {
     if (!plan_uses_tiles(T)) return LORA_OK;
+    TileArgs ta = {};
+    ta.X = X; ta.T = T; ta.d_in = d_in; ta.nproj = nproj;
     for (int p = 0; p < nproj; ++p) {
-        TileArgs ta = {};
-        ta.X = X; ta.Y = pr[p].Y; ta.T = T; ta.d_in = d_in; ta.d_out = pr[p].d_out;
-        ta.ranks = pr[p].ranks; ta.scales = pr[p].scales; ta.pt = pr[p].page_table; ta.pa = pr[p].pa;
-        ta.pb = pr[p].pb; ta.tiles = o.tiles; ta.hdr = o.header; ta.err = err_dev;
-        ta.rowsA = (long long)pr[p].pa->num_pages * LORA_PAGE_ROWS;
-        ta.rowsB = (long long)pr[p].pb->num_pages * LORA_PAGE_ROWS;
-        ta.long_thresh = opt_long_segment();
-        if (int rc = launch_tiles(ta, st, true)) return rc;
+        TileProj &q = ta.proj[p];
+        q.Y = pr[p].Y; q.d_out = pr[p].d_out; q.ranks = pr[p].ranks; q.scales = pr[p].scales;
+        q.pt = pr[p].page_table; q.pa = pr[p].pa; q.pb = pr[p].pb;
     }
-    return LORA_OK;
+    ta.tiles = o.tiles; ta.hdr = o.header; ta.err = err_dev; ta.long_thresh = opt_long_segment();
+    return launch_tiles(ta, st, true);
 }
 
 // Which gather path a call takes (both give bit-identical results).

@@ -170,20 +170,25 @@ int launch_gather(GatherMode mode, const GatherArgs &a, lora_pool_s *const *pa, 
 // size in clusters when there is enough work).
 int gather_clusters(int *out);
 
-struct TileArgs {
-    const uint16_t *X;
-    float *Y;
-    int T, d_in, d_out;
+// One projection of a tile launch: its output, slot tables and pools.
+struct TileProj {
+    float *Y;            // [T][d_out] fp32, in place
+    int d_out;
     const int32_t *ranks;
     const float *scales;
     const int32_t *pt;
     const lora_pool_s *pa;
     const lora_pool_s *pb;
+};
+
+struct TileArgs {
+    const uint16_t *X;
+    int T, d_in;
+    int nproj;           // projections sharing X and the plan (1..LORA_MAX_PROJECTIONS)
+    TileProj proj[LORA_MAX_PROJECTIONS];
     const int4 *tiles;
     const PlanHeader *hdr;
     int32_t *err;
-    long long rowsA;     // rows in the A pool (pages * 16)
-    long long rowsB;     // rows in the B pool
     int long_thresh;     // long-segment threshold the plan used
 };
 int launch_tiles(const TileArgs &a, cudaStream_t st, bool pdl);

@@ -99,10 +99,10 @@ extern "C" int lora_apply_noalloc(const uint16_t *X, float *Y, int T, int d_in, 
     if (int rc = launch_gather(kApply, a, ppa, ppb, st, true)) return rc;
     if (use_tiles) {
         TileArgs ta = {};
-        ta.X = X; ta.Y = Y; ta.T = T; ta.d_in = d_in; ta.d_out = d_out;
-        ta.ranks = ranks; ta.scales = scales; ta.pt = page_table; ta.pa = pa; ta.pb = pb;
-        ta.tiles = o.tiles; ta.hdr = o.header; ta.err = err_dev;
-        ta.rowsA = a.proj[0].rowsA; ta.rowsB = a.proj[0].rowsB; ta.long_thresh = long_thresh;
+        ta.X = X; ta.T = T; ta.d_in = d_in; ta.nproj = 1;
+        ta.proj[0].Y = Y; ta.proj[0].d_out = d_out; ta.proj[0].ranks = ranks; ta.proj[0].scales = scales;
+        ta.proj[0].pt = page_table; ta.proj[0].pa = pa; ta.proj[0].pb = pb;
+        ta.tiles = o.tiles; ta.hdr = o.header; ta.err = err_dev; ta.long_thresh = long_thresh;
         if (int rc = launch_tiles(ta, st, true)) return rc;
     }
     return LORA_OK;

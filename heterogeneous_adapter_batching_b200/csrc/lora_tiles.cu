@@ -8,10 +8,12 @@
 // the tensor cores, then expand v B scaled by alpha/r into the base output.
 //
 // Work: a tile is up to 128 consecutive tokens of one run (from the plan
-// kernel); an item is one tile times one 64-column n-tile of d_out.  Every CTA
-// (one per SM) takes an equal contiguous share of the items in tile-major
-// order and works through it as units of one tile each, recomputing the small
-// shrink of a tile whose items it shares with a neighbour.  Warp-specialised:
+// kernel); an item is one tile times one projection (a launch may cover up to
+// 8 projections that read the same X) times one 64-column n-tile of that
+// projection's d_out.  Every CTA (one per SM) takes an equal contiguous share
+// of the items in (tile, projection, n-tile) order and works through it as
+// units of one (tile, projection) each, recomputing the small shrink of a
+// unit whose items it shares with a neighbour.  Warp-specialised:
 //   warp 0     TMA producer of the shrink operands: X tile [128 x 64] and the
 //              adapter's A^T pages [16 x 64] per page, 128-byte swizzled;
 //   warp 1     TMA producer of the expand operands: B pages [16 x 64] of the
@@ -160,27 +162,62 @@ __device__ __forceinline__ bool epi_all(bool ok) {
     return r != 0;
 }
 
+// One projection of a launch, as the kernel sees it.
+struct KTileProj {
+    float *Y;
+    int d_out;
+    const int32_t *ranks;
+    const float *scales;
+    const int32_t *pt;
+    long long rowsA;     // rows in the A pool (pages * 16)
+    long long rowsB;     // rows in the B pool
+};
+
+template <int NP>
+struct KTile {
+    const uint16_t *X;
+    int T, d_in;
+    int nproj;
+    KTileProj proj[NP];
+    int jpre[NP + 1];    // n-tiles of the projections before p, within one tile
+    const int4 *tiles;
+    const PlanHeader *hdr;
+    int32_t *err;
+};
+
+template <int NP>
+struct TileMaps {
+    CUtensorMap X;
+    CUtensorMap A[NP];
+    CUtensorMap B[NP];
+    CUtensorMap Y[NP];
+};
+
 struct UnitInfo {
     int slot, row0, ntok, r, n1, np, j0, j1;
+    int p;       // projection
     bool skip;
     bool bad;    // rank above 64 or a page outside its pool (LORA_DEV_ERR_BAD_PAGE); rank 0 is not bad
 };
 
-__device__ __forceinline__ UnitInfo unit_info(const TileArgs &a, int tile, int j0, int j1) {
+template <int NP>
+__device__ __forceinline__ UnitInfo unit_info(const KTile<NP> &a, int tile, int pj, int j0, int j1) {
     UnitInfo ui;
     const int4 t = a.tiles[tile];
+    const KTileProj &pr = a.proj[pj];
     ui.slot = t.x;
     ui.row0 = t.y;
     ui.ntok = t.z;
     ui.j0 = j0;
     ui.j1 = j1;
-    int r = a.ranks[ui.slot];
+    ui.p = pj;
+    int r = pr.ranks[ui.slot];
     bool bad = r > LORA_MAX_RANK;
     const int np = (bad || r <= 0) ? 0 : (r + 15) >> 4;
     for (int p = 0; p < np; ++p) {
-        const int pa = a.pt[ui.slot * 8 + p], pb = a.pt[ui.slot * 8 + 4 + p];
-        if (pa < 0 || (long long)(pa + 1) * LORA_PAGE_ROWS > a.rowsA) bad = true;
-        if (pb < 0 || (long long)(pb + 1) * LORA_PAGE_ROWS > a.rowsB) bad = true;
+        const int pa = pr.pt[ui.slot * 8 + p], pb = pr.pt[ui.slot * 8 + 4 + p];
+        if (pa < 0 || (long long)(pa + 1) * LORA_PAGE_ROWS > pr.rowsA) bad = true;
+        if (pb < 0 || (long long)(pb + 1) * LORA_PAGE_ROWS > pr.rowsB) bad = true;
     }
     ui.bad = bad;
     bad = bad || r <= 0;
@@ -191,49 +228,82 @@ __device__ __forceinline__ UnitInfo unit_info(const TileArgs &a, int tile, int j
     return ui;
 }
 
-// Every CTA takes an equal contiguous share of the (tile, n-tile) items in
-// tile-major order and walks it as units of one tile each; a CTA whose share
-// starts or ends inside a tile recomputes that tile's (small) shrink.
+// Items are (tile, projection, 64-column n-tile) in that order; every CTA
+// takes an equal contiguous share and walks it as units of one (tile,
+// projection) each, so a CTA's consecutive units read the same X tile (the
+// second and later projections find it in L2).  A CTA whose share starts or
+// ends inside a unit recomputes that unit's (small) shrink.  Even CTAs walk
+// their share forward and odd CTAs backward, so the two CTAs that share a
+// unit reach it at the same time (both first, or both last) and the second
+// reader of its X rows and adapter pages finds them in L2.
 struct UnitIter {
-    long long it, hi;
-    int nj;
+    long long lo, hi;   // items not yet walked
+    int nj;             // items per tile (all projections)
+    bool back;
 };
 
 __device__ __forceinline__ UnitIter unit_range(int n_tiles, int nj) {
     UnitIter u;
     const long long total = (long long)n_tiles * nj;
-    u.it = total * blockIdx.x / gridDim.x;
+    u.lo = total * blockIdx.x / gridDim.x;
     u.hi = total * (blockIdx.x + 1) / gridDim.x;
     u.nj = nj;
+    u.back = (blockIdx.x & 1) != 0;
     return u;
 }
 
-__device__ __forceinline__ bool next_unit(const TileArgs &a, UnitIter &u, UnitInfo &ui) {
-    if (u.it >= u.hi) return false;
-    const int tile = (int)(u.it / u.nj), j0 = (int)(u.it % u.nj);
-    const int j1 = (int)min((long long)u.nj, j0 + (u.hi - u.it));
-    ui = unit_info(a, tile, j0, j1);
-    u.it += j1 - j0;
+template <int NP>
+__device__ __forceinline__ int proj_of(const KTile<NP> &a, int off) {
+    int pj = 0;
+#pragma unroll
+    for (int q = 1; q < NP; ++q)
+        if (q < a.nproj && off >= a.jpre[q]) pj = q;
+    return pj;
+}
+
+template <int NP>
+__device__ __forceinline__ bool next_unit(const KTile<NP> &a, UnitIter &u, UnitInfo &ui) {
+    if (u.lo >= u.hi) return false;
+    int tile, pj, j0, j1;
+    if (!u.back) {
+        tile = (int)(u.lo / u.nj);
+        const int off = (int)(u.lo - (long long)tile * u.nj);
+        pj = proj_of(a, off);
+        j0 = off - a.jpre[pj];
+        j1 = (int)min((long long)(a.jpre[pj + 1] - a.jpre[pj]), j0 + (u.hi - u.lo));
+        u.lo += j1 - j0;
+    } else {
+        tile = (int)((u.hi - 1) / u.nj);
+        const long long ts = (long long)tile * u.nj;
+        const int off = (int)(u.hi - 1 - ts);
+        pj = proj_of(a, off);
+        const long long us = ts + a.jpre[pj];
+        const long long st = u.lo > us ? u.lo : us;
+        j0 = (int)(st - us);
+        j1 = off - a.jpre[pj] + 1;
+        u.hi = st;
+    }
+    ui = unit_info(a, tile, pj, j0, j1);
     return true;
 }
 
+template <int NP>
 __global__ void __launch_bounds__(kThreads, 1)
-tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmA,
-             const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmY, TileArgs a) {
+tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ KTile<NP> a) {
     extern __shared__ unsigned char smem_raw[];
     TileSmem &sm = *reinterpret_cast<TileSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     // Fetch this launch's parameters and tensor maps while the previous
     // kernel drains.
-    if (threadIdx.x == 0) {
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmX)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmY)) : "memory");
+    const int nproj = NP == 1 ? 1 : a.nproj;
+    if (threadIdx.x == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.X)) : "memory");
+    if (threadIdx.x >= 32 && threadIdx.x < 32 + 3 * nproj) {
+        const int i = threadIdx.x - 32, q = i / 3;
+        const CUtensorMap *m = (i % 3 == 0) ? &maps.A[q] : (i % 3 == 1) ? &maps.B[q] : &maps.Y[q];
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
     }
-    asm volatile("" ::"l"(a.X), "l"(a.Y), "r"(a.T), "r"(a.d_in), "r"(a.d_out), "l"(a.ranks), "l"(a.scales),
-                 "l"(a.pt), "l"(a.tiles), "l"(a.hdr), "l"(a.err), "l"(a.rowsA), "l"(a.rowsB), "r"(a.long_thresh));
+    asm volatile("" ::"l"(a.X), "r"(a.T), "r"(a.d_in), "l"(a.tiles), "l"(a.hdr), "l"(a.err));
     // The kernels before this one on the stream produce the plan.  A batch
     // without long runs has no tiles: leave before touching tensor memory.
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -265,7 +335,7 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    const int nj = (a.d_out + kNB - 1) / kNB;
+    const int nj = a.jpre[nproj];     // items per tile over all projections
     const int nkb = (a.d_in + kKB - 1) / kKB;
 
     if (warp == 0 && lane == 0) {
@@ -277,14 +347,16 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
             if (ui.bad && a.err) atomicOr(a.err, LORA_DEV_ERR_BAD_PAGE);
             if (ui.skip) continue;
             int pg[4];
-            for (int p = 0; p < 4; ++p) pg[p] = p < ui.np ? a.pt[ui.slot * 8 + p] : 0;
+            const int32_t *pt = a.proj[ui.p].pt;
+            for (int p = 0; p < 4; ++p) pg[p] = p < ui.np ? pt[ui.slot * 8 + p] : 0;
+            const CUtensorMap *tmA = &maps.A[ui.p];
             for (int kb = 0; kb < nkb; ++kb, ++it) {
                 const int s = it % kStages;
                 if (!mbar_wait(&sm.empty[s], ((it / kStages) & 1) ^ 1, sm, a.err)) break;
                 mbar_expect_tx(&sm.full[s], (uint32_t)(kM * kKB * 2 + ui.np * 16 * kKB * 2));
-                tma_load(sm.xs[s], &tmX, kb * kKB, ui.row0, &sm.full[s]);
+                tma_load(sm.xs[s], &maps.X, kb * kKB, ui.row0, &sm.full[s]);
                 for (int p = 0; p < ui.np; ++p)
-                    tma_load(&sm.as[s][p * 16 * kKB], &tmA, kb * kKB, pg[p] * LORA_PAGE_ROWS, &sm.full[s]);
+                    tma_load(&sm.as[s][p * 16 * kKB], tmA, kb * kKB, pg[p] * LORA_PAGE_ROWS, &sm.full[s]);
             }
         }
         // the loads this thread armed last on each stage have landed before exit
@@ -297,7 +369,9 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
         while (next_unit(a, ur, ui) && !aborted(sm)) {
             if (ui.skip) continue;
             int pg[4];
-            for (int p = 0; p < 4; ++p) pg[p] = p < ui.np ? a.pt[ui.slot * 8 + 4 + p] : 0;
+            const int32_t *pt = a.proj[ui.p].pt;
+            for (int p = 0; p < 4; ++p) pg[p] = p < ui.np ? pt[ui.slot * 8 + 4 + p] : 0;
+            const CUtensorMap *tmB = &maps.B[ui.p], *tmY = &maps.Y[ui.p];
             for (int j = ui.j0; j < ui.j1; ++j, ++it) {
                 const int b = it % kBuf;
                 const uint32_t par = ((it / kBuf) & 1) ^ 1;
@@ -305,10 +379,10 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
                 if (!mbar_wait(&sm.yempty[b], par, sm, a.err)) break;
                 mbar_expect_tx(&sm.bfull[b], (uint32_t)(ui.np * 16 * kNB * 2));
                 for (int p = 0; p < ui.np; ++p)
-                    tma_load(&sm.bs[b][p * 16 * kNB], &tmB, j * kNB, pg[p] * LORA_PAGE_ROWS, &sm.bfull[b]);
+                    tma_load(&sm.bs[b][p * 16 * kNB], tmB, j * kNB, pg[p] * LORA_PAGE_ROWS, &sm.bfull[b]);
                 mbar_expect_tx(&sm.yfull[b], (uint32_t)(kM * kNB * 4));
-                tma_load(&sm.ys[b][0], &tmY, j * kNB, ui.row0, &sm.yfull[b]);
-                tma_load(&sm.ys[b][kM * 32], &tmY, j * kNB + 32, ui.row0, &sm.yfull[b]);
+                tma_load(&sm.ys[b][0], tmY, j * kNB, ui.row0, &sm.yfull[b]);
+                tma_load(&sm.ys[b][kM * 32], tmY, j * kNB + 32, ui.row0, &sm.yfull[b]);
             }
         }
         for (int i = (it > kBuf ? it - kBuf : 0); i < it; ++i) {
@@ -381,7 +455,8 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
         while (next_unit(a, ur, ui)) {
             if (!epi_all(!aborted(sm))) break;   // same decision in all 128 epilogue threads
             if (ui.skip) continue;
-            const float sc = a.scales[ui.slot];
+            const KTileProj &pr = a.proj[ui.p];
+            const float sc = pr.scales[ui.slot];
             // v = D1 row m, rounded to bf16 into the swizzled V tile
             if (!epi_all(mbar_wait(&sm.shrink_done, itt & 1, sm, a.err))) break;
             tc_fence_after();
@@ -440,16 +515,16 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
                         *yp = y;
                     } else if (m < ui.ntok) {
                         const int col = j * kNB + c * 4;
-                        if (col < a.d_out)
-                            *reinterpret_cast<float4 *>(a.Y + (size_t)(ui.row0 + m) * a.d_out + col) = y;
+                        if (col < pr.d_out)
+                            *reinterpret_cast<float4 *>(pr.Y + (size_t)(ui.row0 + m) * pr.d_out + col) = y;
                     }
                 }
                 if (full_tile) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 epi_sync();
                 if (leader) {
                     if (full_tile) {
-                        tma_store(&tmY, j * kNB, ui.row0, &sm.ys[b][0]);
-                        tma_store(&tmY, j * kNB + 32, ui.row0, &sm.ys[b][kM * 32]);
+                        tma_store(&maps.Y[ui.p], j * kNB, ui.row0, &sm.ys[b][0]);
+                        tma_store(&maps.Y[ui.p], j * kNB + 32, ui.row0, &sm.ys[b][kM * 32]);
                         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                         // the previous store has finished reading its buffer once at
                         // most one group (this one) is still reading
@@ -489,30 +564,36 @@ tiles_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CU
 
 bool tiles_supported() { return tma_supported(); }
 
-int launch_tiles(const TileArgs &a, cudaStream_t st, bool pdl) {
-    static int num_sms[64] = {};
-    int dev = 0;
-    if (int rc = cuda_check(cudaGetDevice(&dev))) return rc;
-    if (dev < 0 || dev >= 64) return LORA_ERR_INVALID_ARG;
+namespace {
+
+template <int NP>
+int launch_np(const TileArgs &a, cudaStream_t st, bool pdl, int sms) {
     const size_t smem = sizeof(TileSmem) + 1024;
-    if (num_sms[dev] == 0) {
-        if (int rc = cuda_check(cudaFuncSetAttribute(tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+    TileMaps<NP> maps;
+    KTile<NP> k;
+    k.X = a.X; k.T = a.T; k.d_in = a.d_in; k.nproj = a.nproj;
+    k.tiles = a.tiles; k.hdr = a.hdr; k.err = a.err;
+    if (int rc = make_tensor_map(&maps.X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.X, (uint64_t)a.d_in, (uint64_t)a.T,
+                                 kKB, kM, true))
+        return rc;
+    k.jpre[0] = 0;
+    for (int p = 0; p < NP; ++p) {
+        const TileProj &q = a.proj[p < a.nproj ? p : 0];
+        k.proj[p].Y = q.Y; k.proj[p].d_out = q.d_out; k.proj[p].ranks = q.ranks; k.proj[p].scales = q.scales;
+        k.proj[p].pt = q.pt;
+        k.proj[p].rowsA = (long long)q.pa->num_pages * LORA_PAGE_ROWS;
+        k.proj[p].rowsB = (long long)q.pb->num_pages * LORA_PAGE_ROWS;
+        if (int rc = make_tensor_map(&maps.Y[p], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, q.Y, (uint64_t)q.d_out,
+                                     (uint64_t)a.T, 32, kM, true))
             return rc;
-        int n = 0;
-        if (int rc = cuda_check(cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev))) return rc;
-        num_sms[dev] = n > 0 ? n : 1;
+        if (int rc = pool_tensor_map(const_cast<lora_pool_s *>(q.pa), &maps.A[p])) return rc;
+        if (int rc = pool_tensor_map(const_cast<lora_pool_s *>(q.pb), &maps.B[p])) return rc;
+        k.jpre[p + 1] = k.jpre[p] + (p < a.nproj ? (q.d_out + kNB - 1) / kNB : 0);
     }
-    CUtensorMap mx, my, ma, mb;
-    if (int rc = make_tensor_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.X, (uint64_t)a.d_in, (uint64_t)a.T, kKB, kM, true))
-        return rc;
-    if (int rc = make_tensor_map(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.Y, (uint64_t)a.d_out, (uint64_t)a.T, 32, kM, true))
-        return rc;
-    if (int rc = pool_tensor_map(const_cast<lora_pool_s *>(a.pa), &ma)) return rc;
-    if (int rc = pool_tensor_map(const_cast<lora_pool_s *>(a.pb), &mb)) return rc;
-    // one CTA per SM (never more than there can be (tile, n-tile) items)
+    // one CTA per SM (never more than there can be items)
     const long long max_tiles = (a.T + kM - 1) / kM + (a.long_thresh > 0 ? a.T / a.long_thresh : 0);
-    long long grid = num_sms[dev];
-    if (grid > max_tiles * ((a.d_out + kNB - 1) / kNB)) grid = max_tiles * ((a.d_out + kNB - 1) / kNB);
+    long long grid = sms;
+    if (grid > max_tiles * k.jpre[NP]) grid = max_tiles * k.jpre[NP];
     if (grid < 1) grid = 1;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
@@ -524,9 +605,33 @@ int launch_tiles(const TileArgs &a, cudaStream_t st, bool pdl) {
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    if (int rc = cuda_check(cudaLaunchKernelEx(&cfg, tiles_kernel, mx, ma, mb, my, a))) return rc;
+    if (int rc = cuda_check(cudaLaunchKernelEx(&cfg, tiles_kernel<NP>, maps, k))) return rc;
     count_launch();
     return LORA_OK;
+}
+
+}  // namespace
+
+int launch_tiles(const TileArgs &a, cudaStream_t st, bool pdl) {
+    static int num_sms[64] = {};
+    int dev = 0;
+    if (a.nproj < 1 || a.nproj > LORA_MAX_PROJECTIONS) return LORA_ERR_INVALID_ARG;
+    if (int rc = cuda_check(cudaGetDevice(&dev))) return rc;
+    if (dev < 0 || dev >= 64) return LORA_ERR_INVALID_ARG;
+    const size_t smem = sizeof(TileSmem) + 1024;
+    if (num_sms[dev] == 0) {
+        if (int rc = cuda_check(cudaFuncSetAttribute(tiles_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     (int)smem)))
+            return rc;
+        if (int rc = cuda_check(cudaFuncSetAttribute(tiles_kernel<LORA_MAX_PROJECTIONS>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+            return rc;
+        int n = 0;
+        if (int rc = cuda_check(cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev))) return rc;
+        num_sms[dev] = n > 0 ? n : 1;
+    }
+    return a.nproj == 1 ? launch_np<1>(a, st, pdl, num_sms[dev])
+                        : launch_np<LORA_MAX_PROJECTIONS>(a, st, pdl, num_sms[dev]);
 }
 
 }  // namespace lora

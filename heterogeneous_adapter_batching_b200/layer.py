@@ -131,3 +131,90 @@ class AdapterCache:
     def release(self, pinned) -> None:
         for s in pinned:
             self.slots.unpin(s)
+
+
+class PrefetchTicket:
+    """A batch whose adapters are being brought in: its slot ids (host), the
+    slots it pins and the event that marks the end of its loads."""
+
+    def __init__(self, ids_host: torch.Tensor, pinned, ready: torch.cuda.Event, misses: int, bytes_loaded: int):
+        self.ids_host, self.pinned, self.ready = ids_host, pinned, ready
+        self.misses, self.bytes_loaded = misses, bytes_loaded
+
+
+class AdapterPrefetcher:
+    """Brings the adapters of upcoming batches into one AdapterLayer's pools on a
+    copy stream while the current batch computes.
+
+    Page "Multi-LoRA Serving in Production", section "Production Engineering
+    Guidelines", "Asynchronous Prefetching and Request Queuing": on a cache
+    miss the weights move from pinned host memory into the GPU pool with a
+    non-blocking cudaMemcpyAsync, and the request waits an iteration or two
+    until the transfer lands instead of stalling the batches already running.
+    Page "LoRA Adapters at Serve Time with vLLM Multi-LoRA", section "The
+    Inference Mechanism: A Worked Scenario", step "Eviction": the least
+    recently used adapter makes room (lora_slot_cache_*, which never picks a
+    slot pinned by a batch that has not been released).
+
+    Ordering, all on the device (the host never waits):
+      * a load into slot s first makes the copy stream wait for the event
+        recorded after the last batch that read s, so pages are not
+        overwritten under a batch still in flight; pages freed by an eviction
+        are reused only by later loads on the same copy stream;
+      * the compute stream waits for a ticket's `ready` event before the batch
+        that uses it.
+    `host` maps an adapter key to (a_t_bits [r, d_in], b_bits [r, d_out], alpha):
+    pinned host tensors give asynchronous transfers.
+    """
+
+    def __init__(self, layer: AdapterLayer, host, copy_stream: Optional[torch.cuda.Stream] = None):
+        self.layer = layer
+        self.host = host
+        self.slots = B.SlotCache(layer.S)
+        self.copy = copy_stream or torch.cuda.Stream(device=layer.device)
+        self.last_use = [None] * layer.S
+
+    def prefetch(self, keys) -> PrefetchTicket:
+        """Make every key of a coming batch resident (pinning its slot) and return
+        its ticket; the loads of the misses are queued on the copy stream."""
+        slot_of, pinned = {}, []
+        misses, nbytes = 0, 0
+        for k in keys:
+            k = int(k)
+            if k < 0 or k in slot_of:
+                continue
+            slot, hit, evicted = self.slots.acquire(k, pin=True)
+            pinned.append(slot)
+            if not hit:
+                ev = self.last_use[slot]
+                if ev is not None:
+                    self.copy.wait_event(ev)
+                if evicted >= 0:
+                    self.layer.evict(slot, stream=self.copy)
+                at, b, alpha = self.host[k]
+                self.layer.load(slot, at.shape[0], alpha, at, b, stream=self.copy)
+                misses += 1
+                nbytes += at.numel() * at.element_size() + b.numel() * b.element_size()
+            slot_of[k] = slot
+        ready = torch.cuda.Event()
+        ready.record(self.copy)
+        ids = torch.tensor([slot_of.get(int(k), -1) for k in keys], dtype=torch.int32)
+        return PrefetchTicket(ids, pinned, ready, misses, nbytes)
+
+    def begin(self, ticket: PrefetchTicket, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """Order `stream` (default: the current stream) after the ticket's loads and
+        return the batch's slot ids on the device."""
+        stream = stream or torch.cuda.current_stream(self.layer.device)
+        stream.wait_event(ticket.ready)
+        with torch.cuda.stream(stream):
+            return ticket.ids_host.to(self.layer.device, non_blocking=True)
+
+    def end(self, ticket: PrefetchTicket, stream: Optional[torch.cuda.Stream] = None) -> None:
+        """After the batch's kernels are queued on `stream`: record when they finish
+        reading its slots and release the pins."""
+        stream = stream or torch.cuda.current_stream(self.layer.device)
+        done = torch.cuda.Event()
+        done.record(stream)
+        for s in ticket.pinned:
+            self.last_use[s] = done
+            self.slots.unpin(s)

@@ -257,8 +257,9 @@ typedef struct {
  *   num_slots and one plan (made with projs[0].ranks: the error bits and the
  *   tokens dropped follow projection 0; a slot that is empty in another
  *   projection is skipped there).  Short segments of every projection are
- *   handled by one gather launch; long runs get one tile launch per
- *   projection.  ws as for lora_apply (lora_workspace_size(T, num_slots)).
+ *   handled by one gather launch (on the split gather path: a shrink and an
+ *   expand launch per projection); long runs by one tile launch for all
+ *   projections.  ws as for lora_apply (lora_workspace_size(T, num_slots)).
  * Each projection's result is bit-identical to lora_apply on that projection
  * alone.  Errors: as lora_apply, checked for every projection before any
  * work is enqueued; LORA_ERR_INVALID_ARG for num_projs out of range. */

@@ -26,7 +26,7 @@ def H():
 
 @pytest.fixture(autouse=True)
 def _restore_options(H):
-    old = {k: H.lora_get_option(k) for k in (H.OPT_LONG_SEGMENT, H.OPT_DECODE_JOB_TOKENS)}
+    old = {k: H.lora_get_option(k) for k in (H.OPT_LONG_SEGMENT, H.OPT_DECODE_JOB_TOKENS, H.OPT_GATHER_PATH)}
     yield
     for k, v in old.items():
         H.lora_set_option(k, v)
@@ -53,6 +53,7 @@ def _run(H, wls):
     Ys = [U.dev_inputs(w)[1] for w in wls]
     layers[0].err.zero_()
     H.apply_multi(layers, X, Ys, ids)
+    _run.launches = H.lora_last_launch_count()
     torch.cuda.synchronize()
     multi = [Y.cpu().numpy() for Y in Ys]
     err = int(layers[0].err.item())
@@ -86,11 +87,14 @@ def test_multi_matches_single_and_oracle(H, seed, T, d_in, d_outs, S):
 
 
 def test_multi_long_runs(H):
-    """Long runs take one tile launch per projection; short segments the shared gather launch."""
+    """Long runs of all projections take one tile launch; short segments the shared
+    gather launch (cluster path: plan + gather + tiles = 3 launches)."""
     H.lora_set_option(H.OPT_LONG_SEGMENT, 16)
+    H.lora_set_option(H.OPT_GATHER_PATH, H.GATHER_CLUSTER)
     base = W.segments(21, [5, 40, 300, 2, 129], 256, 512, 8, reuse=True)
     wls = _projections(base, [256, 1032], 21)
     multi, single, err = _run(H, wls)
+    assert _run.launches == 3
     assert err == 0
     for w, m, s in zip(wls, multi, single):
         assert np.array_equal(m, s), w.name
