@@ -56,6 +56,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-per-config", action="store_true")
+    p.add_argument("--no-prefetch", action="store_true")
     p.add_argument("--per-config", default=",".join(PER_CONFIG),
                    help="comma-separated workloads measured into the per_config object")
     return p.parse_args()
@@ -472,6 +473,61 @@ def measure_config(name: str, dev, stream, H, reps: int, peak_gbs: float, peak_t
     return out
 
 
+def measure_prefetch(dev, H, graph, stream, n_adapters: int = 32, d_in: int = 4096, d_out: int = 14336,
+                     rank: int = 64) -> dict:
+    """Asynchronous adapter loads into a paged pool (AdapterPrefetcher, pinned host
+    memory, a copy stream) alone and while the compute stream replays the
+    benchmark's step graph: H2D GB/s into the pool and the share of the loads'
+    time hidden under compute."""
+    import torch
+    g = torch.Generator()
+    g.manual_seed(99)
+    host = {}
+    for k in range(n_adapters):
+        at = (torch.randn((rank, d_in), generator=g) / math.sqrt(d_in)).to(torch.bfloat16).view(torch.int16)
+        b = (torch.randn((rank, d_out), generator=g) / math.sqrt(rank)).to(torch.bfloat16).view(torch.int16)
+        host[k] = (at.pin_memory(), b.pin_memory(), 2.0 * rank)
+    target = H.AdapterLayer(d_in, d_out, n_adapters, n_adapters * 4, n_adapters * 4, 16, device=dev)
+    pf = H.AdapterPrefetcher(target, host)
+    nbytes = sum(a.numel() * 2 + b.numel() * 2 for a, b, _ in host.values())
+
+    def load_all():
+        t = pf.prefetch(list(range(n_adapters)))
+        pf.end(t, pf.copy)
+        for k in range(n_adapters):              # the next round misses again
+            s = pf.slots.lookup(k)
+            target.evict(s, stream=pf.copy)
+            pf.slots.invalidate(s)
+
+    def compute():
+        with torch.cuda.stream(stream):
+            graph.replay()
+
+    def timed(fn):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        pf.copy.wait_event(e0)
+        fn()
+        stream.wait_stream(pf.copy)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    load_all()
+    compute()
+    t_l = min(timed(load_all) for _ in range(3))
+    t_c = min(timed(compute) for _ in range(3))
+    t_b = min(timed(lambda: (load_all(), compute())) for _ in range(3))
+    del target, pf
+    torch.cuda.empty_cache()
+    return {"adapters": n_adapters, "bytes": nbytes, "h2d_gbs": nbytes / (t_l * 1e-3) / 1e9,
+            "load_ms": t_l, "compute_ms": t_c, "both_ms": t_b,
+            "hidden": (t_l + t_c - t_b) / min(t_l, t_c),
+            "what": f"{n_adapters} rank-{rank} adapters ({d_in} -> {d_out}) from pinned host memory into the pool "
+                    f"on a copy stream, alone and during one replay of the step graph"}
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -584,6 +640,9 @@ def run_gpu(args):
                "d2h_bytes_per_step": int(Yout.numel() * 4), "ms_per_step": e2e_ms,
                "path": "pinned H2D of X, Y_base, ids -> lora_apply (plan + compute kernels) -> D2H of Y, one layer"}
 
+    prefetch = None
+    if world == 1 and not args.no_prefetch:
+        prefetch = measure_prefetch(dev, H, graph, stream)
     del graph
     ring_footprint = ring.footprint()
     del ring
@@ -619,6 +678,7 @@ def run_gpu(args):
                      "ring_bytes": ring_footprint, "parallelism": f"replicas x{world} (no collective)",
                      "projections_per_launch": P},
             "per_config": per_config,
+            "prefetch": prefetch,
         }
         print(json.dumps(line), flush=True)
     return 0
