@@ -41,6 +41,7 @@ MAX_PROJECTIONS = 8
 
 EXPORTS = [
     "lora_pool_create", "lora_pool_destroy", "lora_pool_free_pages", "lora_pool_num_pages",
+    "lora_pool_alloc_pages", "lora_pool_free_page_list", "lora_pool_usage",
     "lora_pool_load", "lora_pool_evict", "lora_pool_read_row", "lora_workspace_size",
     "lora_plan", "lora_shrink", "lora_expand_add", "lora_expand_add_strided", "lora_apply", "lora_apply_planned", "lora_apply_noalloc",
     "lora_apply_multi", "lora_apply_multi_planned",
@@ -83,6 +84,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lora_pool_destroy": (I, [V]),
         "lora_pool_free_pages": (I, [V]),
         "lora_pool_num_pages": (I, [V]),
+        "lora_pool_alloc_pages": (I, [V, I, V]),
+        "lora_pool_free_page_list": (I, [V, V, I]),
+        "lora_pool_usage": (I, [V, ctypes.POINTER(I), ctypes.POINTER(I)]),
         "lora_pool_load": (I, [V, V, I, I, I, F, V, V, V, V, V, V, V]),
         "lora_pool_evict": (I, [V, V, I, I, V, V, V, V]),
         "lora_pool_read_row": (I, [V, V, I, I, I, I, V, V]),
@@ -180,6 +184,27 @@ def lora_pool_free_pages(pool: Pool) -> int:
 
 def lora_pool_num_pages(pool: Pool) -> int:
     return load_library().lora_pool_num_pages(pool._h)
+
+
+def lora_pool_alloc_pages(pool: Pool, n: int) -> torch.Tensor:
+    """n free pages of the pool for another tenant (KV blocks); host int32 ids."""
+    ids = torch.empty(max(n, 0), dtype=torch.int32)
+    _check("lora_pool_alloc_pages", load_library().lora_pool_alloc_pages(pool._h, n, _p(ids) if n > 0 else None))
+    return ids
+
+
+def lora_pool_free_page_list(pool: Pool, ids: torch.Tensor) -> None:
+    ids = ids.to(torch.int32).contiguous()
+    assert ids.device.type == "cpu"
+    _check("lora_pool_free_page_list", load_library().lora_pool_free_page_list(
+        pool._h, _p(ids) if ids.numel() else None, ids.numel()))
+
+
+def lora_pool_usage(pool: Pool):
+    """(pages held by adapters, pages held through lora_pool_alloc_pages)."""
+    a, o = ctypes.c_int(), ctypes.c_int()
+    _check("lora_pool_usage", load_library().lora_pool_usage(pool._h, ctypes.byref(a), ctypes.byref(o)))
+    return a.value, o.value
 
 
 def lora_pool_load(pa: Pool, pb: Pool, slot: int, num_slots: int, rank: int, alpha: float,

@@ -84,7 +84,7 @@ static int take_pages(lora_pool_s *p, int n, const int32_t *want, std::vector<in
 
 static void give_pages(lora_pool_s *p, const std::vector<int> &pages) {
     for (int id : pages) {
-        if (id >= 0 && id < p->num_pages && p->used[id]) {
+        if (id >= 0 && id < p->num_pages && p->used[id] == 1) {
             p->used[id] = 0;
             p->free_stack.push_back(id);
         }
@@ -129,6 +129,48 @@ int lora_pool_free_pages(lora_pool_t pool) {
 }
 
 int lora_pool_num_pages(lora_pool_t pool) { return pool ? pool->num_pages : -1; }
+
+int lora_pool_alloc_pages(lora_pool_t pool, int n, int32_t *ids_out) {
+    if (!pool || n < 0 || (n > 0 && !ids_out)) return LORA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> g(pool->mu);
+    if ((int)pool->free_stack.size() < n) return LORA_ERR_POOL_OOM;
+    for (int i = 0; i < n; ++i) {
+        const int id = pool->free_stack.back();
+        pool->free_stack.pop_back();
+        pool->used[id] = 2;
+        ids_out[i] = id;
+    }
+    return LORA_OK;
+}
+
+int lora_pool_free_page_list(lora_pool_t pool, const int32_t *ids, int n) {
+    if (!pool || n < 0 || (n > 0 && !ids)) return LORA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> g(pool->mu);
+    for (int i = 0; i < n; ++i) {   // all or nothing
+        const int id = ids[i];
+        if (id < 0 || id >= pool->num_pages || pool->used[id] != 2) return LORA_ERR_BAD_SLOT;
+        for (int j = 0; j < i; ++j)
+            if (ids[j] == id) return LORA_ERR_BAD_SLOT;
+    }
+    for (int i = 0; i < n; ++i) {
+        pool->used[ids[i]] = 0;
+        pool->free_stack.push_back(ids[i]);
+    }
+    return LORA_OK;
+}
+
+int lora_pool_usage(lora_pool_t pool, int *adapter_pages, int *other_pages) {
+    if (!pool || !adapter_pages || !other_pages) return LORA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> g(pool->mu);
+    int a = 0, o = 0;
+    for (char u : pool->used) {
+        a += u == 1;
+        o += u == 2;
+    }
+    *adapter_pages = a;
+    *other_pages = o;
+    return LORA_OK;
+}
 
 int lora_pool_load(lora_pool_t pa, lora_pool_t pb, int slot, int num_slots, int rank, float alpha,
                    const uint16_t *a_t, const uint16_t *b, const int32_t *page_ids,

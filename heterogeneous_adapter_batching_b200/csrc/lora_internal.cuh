@@ -71,7 +71,7 @@ struct lora_pool_s {
     int page_rows = 0;
     int num_pages = 0;
     std::vector<int> free_stack;            // free page ids
-    std::vector<char> used;                 // per page
+    std::vector<char> used;                 // per page: 0 free, 1 an adapter's, 2 taken by lora_pool_alloc_pages
     // (page table identity, slot, matrix) -> pages owned
     std::map<std::tuple<const void *, int, int>, std::vector<int>> owners;
     std::mutex mu;

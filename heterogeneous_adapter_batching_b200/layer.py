@@ -49,6 +49,19 @@ class AdapterLayer:
         B.lora_pool_evict(self.pool_a, self.pool_b, slot, self.S, self.page_table, self.scales, self.ranks,
                           stream)
 
+    # Unified paging (shared_pool): KV-cache blocks and adapter pages from one free list.
+    def alloc_pages(self, n: int) -> torch.Tensor:
+        """n pages of pool_a for another tenant (KV blocks: 16 vectors of d_in values
+        each, rows [16 p, 16 p + 16) of buf_a); host int32 page ids."""
+        return B.lora_pool_alloc_pages(self.pool_a, n)
+
+    def free_pages(self, ids: torch.Tensor) -> None:
+        B.lora_pool_free_page_list(self.pool_a, ids)
+
+    def page_rows(self, page: int) -> torch.Tensor:
+        """The 16 rows of page `page` of pool_a (a view of buf_a)."""
+        return self.buf_a[page * B.PAGE_ROWS:(page + 1) * B.PAGE_ROWS]
+
     def apply(self, X: torch.Tensor, Y: torch.Tensor, ids: torch.Tensor, stream=None) -> None:
         T = X.shape[0]
         assert T <= self.max_tokens

@@ -107,6 +107,30 @@ int lora_pool_destroy(lora_pool_t pool);
 int lora_pool_free_pages(lora_pool_t pool);
 int lora_pool_num_pages(lora_pool_t pool);
 
+/* Unified paging: the pool's pages also serve a second tenant of the same
+ * memory, such as KV-cache blocks (16 token vectors of `width` values per
+ * page).  Page "Multi-LoRA Serving in Production", section "Unified Paging
+ * Architecture": all dynamic memory outside the base model is one pool of
+ * fixed-size physical pages that holds KV-cache tensors and adapter weights
+ * alike, so memory moves between the two as traffic changes with no external
+ * fragmentation; page "Multi-LoRA Serving Architecture ... (2026)", section
+ * "S-LoRA unified paging".  Adapter loads and these calls draw on one free
+ * list.
+ *
+ * lora_pool_alloc_pages takes n free pages and writes their ids to ids_out
+ * (host, n entries); LORA_ERR_POOL_OOM (nothing taken) when fewer are free.
+ * Page p is rows [16 p, 16 p + 16) of the pool, owned by the caller until it
+ * is returned; the library never reads or writes it. */
+int lora_pool_alloc_pages(lora_pool_t pool, int n, int32_t *ids_out);
+
+/* Return pages taken by lora_pool_alloc_pages (ids: host, n entries).  All or
+ * nothing: LORA_ERR_BAD_SLOT if an id is out of range, repeated, free, or
+ * held by an adapter. */
+int lora_pool_free_page_list(lora_pool_t pool, const int32_t *ids, int n);
+
+/* Pages held by adapters and by lora_pool_alloc_pages (host outputs). */
+int lora_pool_usage(lora_pool_t pool, int *adapter_pages, int *other_pages);
+
 /* Load adapter (A, B) of rank `rank` into slot `slot` of the page table
  * page_table_dev [num_slots][2][LORA_MAX_PAGES_PER_MATRIX] (int32; matrix 0 =
  * A, 1 = B; unused entries are written as -1).
