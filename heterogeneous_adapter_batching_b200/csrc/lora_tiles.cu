@@ -20,9 +20,11 @@
 //              current 64-column n-tile and the Y tile [128 x 64] fp32;
 //   warp 2     allocates tensor memory and issues tcgen05.mma:
 //                shrink  D1[128 x N1] = X[128 x d_in] A[d_in x N1]   (N1 = r rounded up to 16)
-//                expand  D2[128 x 64] = V[128 x N1] B[N1 x 64]        (B read MN-major)
-//   warps 4-7  epilogue: read D1 from tensor memory, round v to bf16 into a
-//              swizzled shared tile (the A operand of the expand), then per
+//                expand  D2[128 x 64] = Vhi[128 x N1] B[N1 x 64] + Vlo[128 x N1] B[N1 x 64]
+//                        (B read MN-major)
+//   warps 4-7  epilogue: read D1 from tensor memory, split v into a bf16 high
+//              part and a bf16 low part in two swizzled shared tiles (the A
+//              operands of the expand's two products), then per
 //              n-tile read D2, add s * D2 to the Y tile and write it back with
 //              a TMA store (or row stores for a tile with fewer than 128 tokens).
 // Pages hold 16 rank-rows; ranks that are not a multiple of 16 read the
@@ -49,7 +51,8 @@ constexpr long long kWaitLimit = 2000000000LL;
 struct TileSmem {
     __nv_bfloat16 xs[kStages][kM * kKB];      // 16 KB each, K-major SW128
     __nv_bfloat16 as[kStages][64 * kKB];      //  8 KB each, up to 4 pages x 16 rows
-    __nv_bfloat16 vs[kM * 64];                // 16 KB, V (expand A operand), K-major SW128
+    __nv_bfloat16 vs[kM * 64];                // 16 KB, v high part (expand A operand), K-major SW128
+    __nv_bfloat16 vl[kM * 64];                // 16 KB, v low part (v - high), same layout
     __nv_bfloat16 bs[kBuf][64 * kNB];         //  8 KB each, B n-tile, rank rows x 64 cols (MN-major SW128)
     float ys[kBuf][kM * kNB];                 // 32 KB each, two SW128 boxes of [128 rows x 32 cols]
     uint64_t full[kStages], empty[kStages];
@@ -58,6 +61,8 @@ struct TileSmem {
     uint32_t tmem_base;
     int abort;
 };
+
+static_assert(sizeof(TileSmem) + 1024 <= 227 * 1024, "tiles kernel: shared memory beyond the per-block limit");
 
 __device__ __forceinline__ uint32_t su32(const void *p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
@@ -420,6 +425,7 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
             if (!mbar_wait(&sm.v_ready, itt & 1, sm, a.err)) break;
             tc_fence_after();
             const uint64_t dv = sdesc(sm.vs, 16, 1024);
+            const uint64_t dvl = sdesc(sm.vl, 16, 1024);
             for (int j = ui.j0; j < ui.j1; ++j, ++ite) {
                 const int b = ite % kBuf;
                 const uint32_t par = (ite / kBuf) & 1;
@@ -430,6 +436,8 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
                 for (int k = 0; k < ui.np; ++k)
                     mma_bf16(tmem + 64 + 64 * b, dv + (uint64_t)(k * 2), dbb + (uint64_t)(k * (2048 >> 4)), idesc2,
                              k != 0);
+                for (int k = 0; k < ui.np; ++k)
+                    mma_bf16(tmem + 64 + 64 * b, dvl + (uint64_t)(k * 2), dbb + (uint64_t)(k * (2048 >> 4)), idesc2, 1);
                 mma_commit(&sm.bempty[b]);
                 mma_commit(&sm.accfull[b]);
             }
@@ -468,20 +476,24 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
             tc_fence_before();
             mbar_arrive(&sm.d1_empty);
             if (!epi_all(mbar_wait(&sm.v_empty, (itt & 1) ^ 1, sm, a.err))) break;
+            // v enters the expand as a bf16 high part and a bf16 low part
+            // (v - high), so the product keeps about 16 significant bits of v
             unsigned char *vrow = reinterpret_cast<unsigned char *>(sm.vs) + m * 128;
+            unsigned char *lrow = reinterpret_cast<unsigned char *>(sm.vl) + m * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 if (c < ui.np * 2) {
-                    uint4 pk;
-                    __nv_bfloat162 h0 = __floats2bfloat162_rn(d1[c * 8 + 0], d1[c * 8 + 1]);
-                    __nv_bfloat162 h1 = __floats2bfloat162_rn(d1[c * 8 + 2], d1[c * 8 + 3]);
-                    __nv_bfloat162 h2 = __floats2bfloat162_rn(d1[c * 8 + 4], d1[c * 8 + 5]);
-                    __nv_bfloat162 h3 = __floats2bfloat162_rn(d1[c * 8 + 6], d1[c * 8 + 7]);
-                    pk.x = *reinterpret_cast<uint32_t *>(&h0);
-                    pk.y = *reinterpret_cast<uint32_t *>(&h1);
-                    pk.z = *reinterpret_cast<uint32_t *>(&h2);
-                    pk.w = *reinterpret_cast<uint32_t *>(&h3);
-                    *reinterpret_cast<uint4 *>(vrow + ((c ^ (m & 7)) << 4)) = pk;
+                    uint32_t hw[4], lw[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float f0 = d1[c * 8 + 2 * e], f1 = d1[c * 8 + 2 * e + 1];
+                        const __nv_bfloat162 h = __floats2bfloat162_rn(f0, f1);
+                        const __nv_bfloat162 l = __floats2bfloat162_rn(f0 - __low2float(h), f1 - __high2float(h));
+                        hw[e] = *reinterpret_cast<const uint32_t *>(&h);
+                        lw[e] = *reinterpret_cast<const uint32_t *>(&l);
+                    }
+                    *reinterpret_cast<uint4 *>(vrow + ((c ^ (m & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4 *>(lrow + ((c ^ (m & 7)) << 4)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
                 }
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

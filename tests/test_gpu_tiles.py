@@ -5,7 +5,8 @@ the tile path, with ragged tails (tiles of fewer than 128 tokens), widths that
 are not multiples of the 64-column blocks, ranks that are not multiples of the
 16-row page, and a mix with short and non-contiguous segments (gather path).
 Tolerance: |err| <= 2e-3 + 1e-2 |ref| per element, and the adapter delta within
-8e-3 of its largest magnitude (v is rounded to bf16 between the two products).
+2e-4 of its largest magnitude (v enters the second product as a bf16 high part and a
+bf16 low part, about 16 significant bits).
 """
 import numpy as np
 import pytest
