@@ -162,7 +162,14 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
 
 // One slot's rank, pages and scale, validated against both pools (a unit is
 // skipped in both kernels when either matrix is out of range, so the expand
-// never reads a partial that the shrink did not write).
+// never reads a partial that the shrink did not write).  The loads (RawMeta)
+// are issued one unit ahead of their use, the checks (Meta) at the use.
+struct RawMeta {
+    int r;
+    int4 pga, pgb;
+    float scale;
+};
+
 struct Meta {
     int r, np;
     int4 pga, pgb;
@@ -170,21 +177,29 @@ struct Meta {
     bool bad;
 };
 
-__device__ __forceinline__ Meta slot_meta(const KSplit &a, const int4 *spt, const int *srk, const float *ssc,
-                                          bool staged, int slot) {
-    Meta m;
-    int r;
+__device__ __forceinline__ RawMeta raw_meta(const KSplit &a, const int4 *spt, const int *srk, const float *ssc,
+                                            bool staged, int slot) {
+    RawMeta m;
     if (staged) {
-        r = srk[slot];
+        m.r = srk[slot];
         m.pga = spt[2 * slot];
         m.pgb = spt[2 * slot + 1];
         m.scale = ssc ? ssc[slot] : 0.f;
     } else {
-        r = a.ranks[slot];
+        m.r = a.ranks[slot];
         m.pga = reinterpret_cast<const int4 *>(a.pt)[2 * slot];
         m.pgb = reinterpret_cast<const int4 *>(a.pt)[2 * slot + 1];
         m.scale = ssc ? a.scales[slot] : 0.f;
     }
+    return m;
+}
+
+__device__ __forceinline__ Meta check_meta(const KSplit &a, const RawMeta &raw) {
+    Meta m;
+    int r = raw.r;
+    m.pga = raw.pga;
+    m.pgb = raw.pgb;
+    m.scale = raw.scale;
     m.bad = r > LORA_MAX_RANK;
     if (r <= 0 || m.bad) r = 0;
     const int np = (r + LORA_PAGE_ROWS - 1) / LORA_PAGE_ROWS;
@@ -200,6 +215,10 @@ __device__ __forceinline__ Meta slot_meta(const KSplit &a, const int4 *spt, cons
     m.r = m.bad ? 0 : r;
     m.np = m.bad ? 0 : np;
     return m;
+}
+
+__device__ __forceinline__ int page_of(const int4 &pg, int p) {
+    return p == 0 ? pg.x : p == 1 ? pg.y : p == 2 ? pg.z : pg.w;
 }
 
 // Token t of a job: the first four are in the job record, the rest in the
@@ -258,14 +277,38 @@ shrink_part_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         const int n_jobs = a.hdr->n_jobs;
         const int n_units = n_jobs * kSlices;
         const unsigned Gi = (unsigned)a.d_in >> 3;
+        const int G = gridDim.x;
         int chunk = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-            const int ji = u / kSlices, s = u - ji * kSlices;
-            const int4 job = a.jobs[2 * ji];
-            const int4 tk = a.jobs[2 * ji + 1];
-            const int slot = job.x, n = min(job.y, LORA_MAX_JOB_TOKENS), q0 = job.z;
-            const Meta m = slot_meta(a, sm.pt, sm.ranks, nullptr, staged, slot);
+        // the job record two units ahead and the slot tables one unit ahead are
+        // in flight while the current unit streams
+        int4 jobA = make_int4(0, 0, 0, 0), tkA = jobA, jobB = jobA, tkB = jobA;
+        RawMeta rmA = {};
+        int tokA = -1;
+        const int u0 = blockIdx.x;
+        if (u0 < n_units) { jobA = a.jobs[2 * (u0 / kSlices)]; tkA = a.jobs[2 * (u0 / kSlices) + 1]; }
+        if (u0 + G < n_units) { jobB = a.jobs[2 * ((u0 + G) / kSlices)]; tkB = a.jobs[2 * ((u0 + G) / kSlices) + 1]; }
+        if (u0 < n_units) {
+            rmA = raw_meta(a, sm.pt, sm.ranks, nullptr, staged, jobA.x);
+            tokA = job_token(a, tkA, jobA.z, min(jobA.y, LORA_MAX_JOB_TOKENS), lane);
+        }
+        for (int u = u0; u < n_units && ok; u += G) {
+            const int s = u - (u / kSlices) * kSlices;
+            const int4 job = jobA;
+            const RawMeta rm = rmA;
+            const int mytok = tokA;
+            jobA = jobB;
+            tkA = tkB;
+            if (u + G < n_units) {
+                rmA = raw_meta(a, sm.pt, sm.ranks, nullptr, staged, jobA.x);
+                tokA = job_token(a, tkA, jobA.z, min(jobA.y, LORA_MAX_JOB_TOKENS), lane);
+            }
+            if (u + 2 * G < n_units) {
+                jobB = a.jobs[2 * ((u + 2 * G) / kSlices)];
+                tkB = a.jobs[2 * ((u + 2 * G) / kSlices) + 1];
+            }
+            const int n = min(job.y, LORA_MAX_JOB_TOKENS), q0 = job.z;
+            const Meta m = check_meta(a, rm);
             if (m.r == 0 || n <= 0) continue;
             const int nt = (n + kNTok - 1) / kNTok;
             const int in0 = 8 * (int)(Gi * s / kSlices), in1 = 8 * (int)(Gi * (s + 1) / kSlices);
@@ -273,8 +316,6 @@ shrink_part_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             const int nb = min(16 / m.np, nt > 1 ? 8 : 16);
             const int cw = nb * kBoxCols, px = cw * 2 + 16;
             const int nch = (in1 - in0 + cw - 1) / cw;
-            const int mytok = job_token(a, tk, q0, n, lane);
-            const int pa[4] = {m.pga.x, m.pga.y, m.pga.z, m.pga.w};
             for (int c = 0; c < nch; ++c) {
                 const int st = chunk % kStages;
                 if (!wait_w(&sm.empty[st], ((chunk / kStages) & 1) ^ 1, sm, a.err)) { ok = false; break; }
@@ -289,11 +330,13 @@ shrink_part_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                 }
                 __syncwarp();
                 unsigned char *sb = sm.stage[st];
-                if (lane == 0)
-                    for (int p = 0; p < m.np; ++p)
-                        for (int b = 0; b < boxes; ++b)
-                            tma_load_2d(sb + (p * nb + b) * kBoxBytes, &tmA, c0 + b * kBoxCols, pa[p] * LORA_PAGE_ROWS,
-                                        &sm.full[st]);
+                // lanes 16..31 issue the page boxes (at most 16), lanes 0..n-1 the X rows
+                const int bi = lane - 16;
+                if (bi >= 0 && bi < m.np * boxes) {
+                    const int p = bi / boxes, b = bi - p * boxes;
+                    tma_load_2d(sb + (p * nb + b) * kBoxBytes, &tmA, c0 + b * kBoxCols,
+                                page_of(m.pga, p) * LORA_PAGE_ROWS, &sm.full[st]);
+                }
                 if (lane < n)
                     bulk_load(sb + kBoxRegion + lane * px, a.X + (size_t)mytok * a.d_in + c0, (uint32_t)((c1 - c0) * 2),
                               &sm.full[st]);
@@ -489,12 +532,37 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
             asm volatile("griddepcontrol.launch_dependents;");
             waited = true;
         };
-        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const int G = gridDim.x;
+        int4 jobA = make_int4(0, 0, 0, 0), tkA = jobA, jobB = jobA, tkB = jobA;
+        RawMeta rmA = {};
+        int tokA = -1;
+        const int u0 = blockIdx.x;
+        if (u0 < n_units) { jobA = ld_cg_v4(a.jobs + 2 * (u0 / E)); tkA = ld_cg_v4(a.jobs + 2 * (u0 / E) + 1); }
+        if (u0 + G < n_units) {
+            jobB = ld_cg_v4(a.jobs + 2 * ((u0 + G) / E));
+            tkB = ld_cg_v4(a.jobs + 2 * ((u0 + G) / E) + 1);
+        }
+        if (u0 < n_units) {
+            rmA = raw_meta(a, sm.pt, sm.ranks, sm.scales, staged, jobA.x);
+            tokA = job_token(a, tkA, jobA.z, min(jobA.y, LORA_MAX_JOB_TOKENS), lane);
+        }
+        for (int u = u0; u < n_units && ok; u += G) {
             const int ji = u / E, e = u - ji * E;
-            const int4 job = ld_cg_v4(a.jobs + 2 * ji);
-            const int4 tk = ld_cg_v4(a.jobs + 2 * ji + 1);
-            const int slot = job.x, n = min(job.y, LORA_MAX_JOB_TOKENS), q0 = job.z;
-            const Meta m = slot_meta(a, sm.pt, sm.ranks, sm.scales, staged, slot);
+            const int4 job = jobA;
+            const RawMeta rm = rmA;
+            const int mytok = tokA;
+            jobA = jobB;
+            tkA = tkB;
+            if (u + G < n_units) {
+                rmA = raw_meta(a, sm.pt, sm.ranks, sm.scales, staged, jobA.x);
+                tokA = job_token(a, tkA, jobA.z, min(jobA.y, LORA_MAX_JOB_TOKENS), lane);
+            }
+            if (u + 2 * G < n_units) {
+                jobB = ld_cg_v4(a.jobs + 2 * ((u + 2 * G) / E));
+                tkB = ld_cg_v4(a.jobs + 2 * ((u + 2 * G) / E) + 1);
+            }
+            const int n = min(job.y, LORA_MAX_JOB_TOKENS), q0 = job.z;
+            const Meta m = check_meta(a, rm);
             if (m.bad && e == 0 && lane == 0 && a.err) atomicOr(a.err, LORA_DEV_ERR_BAD_PAGE);
             if (m.r == 0 || n <= 0) continue;
             const int out0 = 8 * (int)(Go * e / E), out1 = 8 * (int)(Go * (e + 1) / E);
@@ -504,8 +572,6 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
             const int nb = max(1, min(16 / m.np, ylim));
             const int cw = nb * kBoxCols, py = cw * 4 + 16;
             const int nch = (out1 - out0 + cw - 1) / cw;
-            const int mytok = job_token(a, tk, q0, n, lane);
-            const int pb[4] = {m.pgb.x, m.pgb.y, m.pgb.z, m.pgb.w};
             const int vb = nv & 1;
             auto issue_v = [&]() {
                 if (!wait_w(&sm.vempty[vb], ((nv >> 1) & 1) ^ 1, sm, a.err)) return false;
@@ -536,11 +602,13 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
                     mbar_expect_tx(&sm.full[st], (uint32_t)(m.np * boxes * kBoxBytes + n * (c1 - c0) * 4));
                 __syncwarp();
                 unsigned char *sb = sm.stage[st];
-                if (lane == 0)
-                    for (int p = 0; p < m.np; ++p)
-                        for (int b = 0; b < boxes; ++b)
-                            tma_load_2d(sb + (p * nb + b) * kBoxBytes, &tmB, c0 + b * kBoxCols, pb[p] * LORA_PAGE_ROWS,
-                                        &sm.full[st]);
+                // lanes 16..31 issue the page boxes (at most 16), lanes 0..n-1 the Y rows
+                const int bi = lane - 16;
+                if (bi >= 0 && bi < m.np * boxes) {
+                    const int p = bi / boxes, b = bi - p * boxes;
+                    tma_load_2d(sb + (p * nb + b) * kBoxBytes, &tmB, c0 + b * kBoxCols,
+                                page_of(m.pgb, p) * LORA_PAGE_ROWS, &sm.full[st]);
+                }
                 if (lane < n)
                     bulk_load(sb + kBoxRegion + lane * py, a.Y + (size_t)mytok * a.d_out + c0,
                               (uint32_t)((c1 - c0) * 4), &sm.full[st]);
