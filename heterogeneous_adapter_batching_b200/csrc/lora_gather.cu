@@ -44,6 +44,7 @@
 // LORA_DEV_ERR_TIMEOUT in the error word and the kernel runs to completion
 // without trapping.  No cluster multicast is used.
 #include "lora_internal.cuh"
+#include "lora_ptx.cuh"
 
 namespace lora {
 namespace {
@@ -112,6 +113,8 @@ template <int NP>
 struct GatherMaps {
     CUtensorMap A[NP];
     CUtensorMap B[NP];
+    CUtensorMap A4[NP];   // the pools seen in 3D (four 64-column blocks per box); a copy of A/B for widths below 256
+    CUtensorMap B4[NP];
 };
 
 template <int NP>
@@ -184,11 +187,6 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
-__device__ __forceinline__ void tma_load_box(void *dst, const CUtensorMap *m, int x, int y, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(smem_u32(bar)) : "memory");
-}
 
 __device__ __forceinline__ uint32_t map_peer(uint32_t addr, uint32_t rank) {
     uint32_t r;
@@ -381,8 +379,9 @@ gather_kernel(const __grid_constant__ GatherMaps<NP> maps, const __grid_constant
     // Every launch's parameters sit in memory this SM has not read yet: fetch
     // them and both tensor maps now, while the previous kernel drains, rather
     // than on first use.
-    if (warp == kConsumerWarps && lane < 2 * nproj) {
-        const CUtensorMap *m = (lane & 1) ? &maps.B[lane >> 1] : &maps.A[lane >> 1];
+    if (warp == kConsumerWarps && lane < 4 * nproj) {
+        const int q = lane >> 2, k = lane & 3;
+        const CUtensorMap *m = k == 0 ? &maps.A[q] : k == 1 ? &maps.B[q] : k == 2 ? &maps.A4[q] : &maps.B4[q];
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
     }
     asm volatile("" ::"l"(a.X), "l"(a.V), "r"(a.T), "r"(a.d_in), "r"(a.S), "r"(nproj), "l"(a.perm), "l"(a.jobs),
@@ -457,28 +456,31 @@ gather_kernel(const __grid_constant__ GatherMaps<NP> maps, const __grid_constant
             const SlotMeta m = slot_meta<MODE>(a, sm, staged, pj, job.x);
             const UnitGeom g = unit_geom<MODE>(a, sm, pj, m.np, e, crank);
             const CUtensorMap *tmA = &maps.A[pj], *tmB = &maps.B[pj];
+            const CUtensorMap *tmA4 = &maps.A4[pj], *tmB4 = &maps.B4[pj];
+            const int d_out = a.proj[pj].d_out;
             // Shrink chunks, then expand chunks, in the order the consumers use
             // them; the ring lets the loads run up to kStages chunks ahead,
-            // into the next unit.
-            const int pa[4] = {m.pga.x, m.pga.y, m.pga.z, m.pga.w};
-            const int pb[4] = {m.pgb.x, m.pgb.y, m.pgb.z, m.pgb.w};
+            // into the next unit.  Lane 0 arms the stage; lanes 0..15 each issue
+            // one page's group of four 64-column blocks (one 3D box, or 2D
+            // boxes at the row's end).
             const int cw = g.nb * kBoxCols;
-            auto issue = [&](int c) {
+            for (int c = 0; c < g.n_shrink + g.n_expand; ++c) {
                 const int s = chunk % kStages;
                 mbar_wait(&sm.empty[s], ((chunk / kStages) & 1) ^ 1, sm, a.err);
                 const bool shrink = c < g.n_shrink;
                 const int c0 = shrink ? g.in0 + c * cw : g.out0 + (c - g.n_shrink) * cw;
                 const int c1 = shrink ? g.in1 : g.out1;
                 const int boxes = min(g.nb, (c1 - c0 + kBoxCols - 1) / kBoxCols);
-                mbar_expect_tx(&sm.full[s], (uint32_t)(m.np * boxes * kBoxBytes));
-                for (int p = 0; p < m.np; ++p)
-                    for (int b = 0; b < boxes; ++b)
-                        tma_load_box(sm.stage[s] + (size_t)(p * g.nb + b) * kBoxBytes, shrink ? tmA : tmB,
-                                     c0 + b * kBoxCols, (shrink ? pa[p] : pb[p]) * LORA_PAGE_ROWS, &sm.full[s]);
+                if (lane == 0) mbar_expect_tx(&sm.full[s], (uint32_t)(m.np * boxes * kBoxBytes));
+                __syncwarp();
+                if (shrink)
+                    ptx::issue_page_boxes(lane, sm.stage[s], tmA, tmA4, a.d_in >= 256, a.d_in, m.np, g.nb, boxes, c0,
+                                          m.pga, &sm.full[s]);
+                else
+                    ptx::issue_page_boxes(lane, sm.stage[s], tmB, tmB4, d_out >= 256, d_out, m.np, g.nb, boxes, c0,
+                                          m.pgb, &sm.full[s]);
                 ++chunk;
-            };
-            if (lane == 0)
-                for (int c = 0; c < g.n_shrink + g.n_expand; ++c) issue(c);
+            }
             __syncwarp();
         }
         if (lane == 0) {
@@ -869,6 +871,14 @@ int launch_mode(const GatherArgs &ga, lora_pool_s *const *pa, lora_pool_s *const
         }
         if (MODE == kExpand) maps.A[p] = maps.B[p];
         if (MODE == kShrink) maps.B[p] = maps.A[p];
+        maps.A4[p] = maps.A[p];
+        maps.B4[p] = maps.B[p];
+        if (MODE != kExpand && pa[p]->width >= 256) {
+            if (int rc = pool_tensor_map4(pa[p], &maps.A4[p])) return rc;
+        }
+        if (MODE != kShrink && pb[p]->width >= 256) {
+            if (int rc = pool_tensor_map4(pb[p], &maps.B4[p])) return rc;
+        }
         // a d_out part keeps at least kCS x 8 column groups (8 per CTA)
         const int em = (a.proj[p].d_out >> 3) / (kCS * 8);
         e_max = min(e_max, em < 1 ? 1 : em);
@@ -876,6 +886,8 @@ int launch_mode(const GatherArgs &ga, lora_pool_s *const *pa, lora_pool_s *const
     for (int p = a.nproj; p < NP; ++p) {   // unused slots: valid copies, never read
         maps.A[p] = maps.A[0];
         maps.B[p] = maps.B[0];
+        maps.A4[p] = maps.A4[0];
+        maps.B4[p] = maps.B4[0];
     }
 
     cudaLaunchConfig_t cfg = {};

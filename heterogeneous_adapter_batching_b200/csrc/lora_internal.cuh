@@ -78,6 +78,8 @@ struct lora_pool_s {
     // TMA descriptors of the pool, built on first use (see pool_tensor_map)
     CUtensorMap tmap;
     bool tmap_ok = false;
+    CUtensorMap tmap4;       // 4 consecutive 64-column blocks per box (pool_tensor_map4)
+    bool tmap4_ok = false;
 };
 
 namespace lora {
@@ -88,6 +90,11 @@ int make_tensor_map(CUtensorMap *m, CUtensorMapDataType dt, int esize, const voi
                     uint64_t rows, uint32_t box_cols, uint32_t box_rows, bool swizzle128);
 // The pool's map: a box is 64 columns x 16 rows (one page high), 128-byte swizzle.
 int pool_tensor_map(lora_pool_s *pool, CUtensorMap *out);
+// The pool seen in 3D, (column, row, 64-column step): one box (64, 16, 4) lands
+// the same shared-memory bytes as four boxes of the 2D map at columns x, x+64,
+// x+128, x+192 (valid for x + 256 <= width), with one TMA operation instead of
+// four.  Only for widths of at least 256 (LORA_ERR_INVALID_ARG otherwise).
+int pool_tensor_map4(lora_pool_s *pool, CUtensorMap *out);
 
 // Process-wide options.
 int opt_long_segment();

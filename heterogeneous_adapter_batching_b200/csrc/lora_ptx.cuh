@@ -42,6 +42,35 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, int
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(smem_u32(bar)) : "memory");
 }
 
+// 3D tiled TMA load of one box into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, int x, int y, int z, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// The page boxes of one chunk: for page p (rows pg * 16 ...) the 64-column
+// blocks b = 0 .. boxes-1 starting at column c0, written at dst + (p * nb + b)
+// * 2 KB.  Lane i (< np * ceil(boxes / 4)) takes page i / ng, blocks 4 g ..
+// 4 g + 3 of it: one 3D box when all four lie inside the row (m4 valid and
+// c0 + 64 (4 g + 4) <= width), else one 2D box per block.
+__device__ __forceinline__ void issue_page_boxes(int i, unsigned char *dst, const CUtensorMap *m2,
+                                                 const CUtensorMap *m4, bool use4, int width, int np, int nb,
+                                                 int boxes, int c0, int4 pages, uint64_t *bar) {
+    const int ng = (boxes + 3) >> 2;
+    if (i >= np * ng) return;
+    const int p = i / ng, g = i - p * ng;
+    const int pg = p == 0 ? pages.x : p == 1 ? pages.y : p == 2 ? pages.z : pages.w;
+    const int b0 = 4 * g, b1 = b0 + 4 < boxes ? b0 + 4 : boxes;
+    unsigned char *d = dst + (p * nb + b0) * 2048;
+    if (use4 && b1 - b0 == 4 && c0 + 64 * b1 <= width) {
+        tma_load_3d(d, m4, c0 + 64 * b0, pg * 16, 0, bar);
+    } else {
+        for (int b = b0; b < b1; ++b) tma_load_2d(dst + (p * nb + b) * 2048, m2, c0 + 64 * b, pg * 16, bar);
+    }
+}
+
 // Contiguous bulk copy global -> shared (both 16-byte aligned, bytes a
 // multiple of 16), completing on `bar`.
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {

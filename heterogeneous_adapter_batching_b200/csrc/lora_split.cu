@@ -13,8 +13,8 @@
 // adapter pages back to back, with no exchange inside a unit of work:
 //
 //   shrink_part_kernel   units = (gather job, quarter s of d_in).  A producer
-//                        warp streams the quarter's A^T pages (2D TMA boxes of
-//                        16 rank rows x 64 columns, 128-byte swizzle) and the
+//                        warp streams the quarter's A^T pages (TMA boxes of 16
+//                        rank rows x 4 x 64 columns, 128-byte swizzle) and the
 //                        job's X rows (bulk copies) into a ring of stages; 15
 //                        consumer warps run warp-level bf16 MMAs and write the
 //                        quarter's fp32 partial v into the workspace.
@@ -125,6 +125,7 @@ struct KSplit {
     float *vpart;            // [kSlices][T][LORA_MAX_RANK] fp32
     int32_t *err;
     int e_max;               // most d_out parts (each keeps >= 64 columns)
+    bool wide_in, wide_out;  // the 3D page maps are valid (width >= 256)
 };
 
 // Bounded wait on an mbarrier phase; false when it ran out or the CTA aborted.
@@ -217,10 +218,6 @@ __device__ __forceinline__ Meta check_meta(const KSplit &a, const RawMeta &raw) 
     return m;
 }
 
-__device__ __forceinline__ int page_of(const int4 &pg, int p) {
-    return p == 0 ? pg.x : p == 1 ? pg.y : p == 2 ? pg.z : pg.w;
-}
-
 // Token t of a job: the first four are in the job record, the rest in the
 // plan's token list.  -1 past the job's end.
 __device__ __forceinline__ int job_token(const KSplit &a, const int4 &tk, int q0, int n, int t) {
@@ -249,7 +246,8 @@ __device__ __forceinline__ bool stage_tables(const KSplit &a, Sm &sm, float *sca
 // Shrink: partial v of one d_in quarter per unit.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, 1)
-shrink_part_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ KSplit a) {
+shrink_part_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA4,
+                   const __grid_constant__ KSplit a) {
     extern __shared__ unsigned char smem_raw[];
     ShrinkSmem &sm = *reinterpret_cast<ShrinkSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -264,6 +262,7 @@ shrink_part_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA4)) : "memory");
     }
     const bool staged = stage_tables(a, sm, (float *)nullptr);
     // The plan (job list) may come from the kernel just before this one: wait
@@ -330,13 +329,11 @@ shrink_part_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                 }
                 __syncwarp();
                 unsigned char *sb = sm.stage[st];
-                // lanes 16..31 issue the page boxes (at most 16), lanes 0..n-1 the X rows
-                const int bi = lane - 16;
-                if (bi >= 0 && bi < m.np * boxes) {
-                    const int p = bi / boxes, b = bi - p * boxes;
-                    tma_load_2d(sb + (p * nb + b) * kBoxBytes, &tmA, c0 + b * kBoxCols,
-                                page_of(m.pga, p) * LORA_PAGE_ROWS, &sm.full[st]);
-                }
+                // lanes 16..31 issue the page boxes (a group of four 64-column
+                // blocks per lane), lanes 0..n-1 the X rows
+                if (lane >= 16)
+                    issue_page_boxes(lane - 16, sb, &tmA, &tmA4, a.wide_in, a.d_in, m.np, nb, boxes, c0, m.pga,
+                                     &sm.full[st]);
                 if (lane < n)
                     bulk_load(sb + kBoxRegion + lane * px, a.X + (size_t)mytok * a.d_in + c0, (uint32_t)((c1 - c0) * 2),
                               &sm.full[st]);
@@ -492,7 +489,8 @@ __device__ __forceinline__ int choose_parts(int n_jobs, int grid, int e_max) {
 // Expand: Y += s * v B over one d_out part per unit.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, 1)
-expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ KSplit a) {
+expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB4,
+                   const __grid_constant__ KSplit a) {
     extern __shared__ unsigned char smem_raw[];
     ExpandSmem &sm = *reinterpret_cast<ExpandSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -511,6 +509,7 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB4)) : "memory");
     }
     // The shrink kernel ahead of this one waited for the plan before it let
     // this grid start, so the plan, the slot tables, the pages and Y may be
@@ -602,13 +601,11 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
                     mbar_expect_tx(&sm.full[st], (uint32_t)(m.np * boxes * kBoxBytes + n * (c1 - c0) * 4));
                 __syncwarp();
                 unsigned char *sb = sm.stage[st];
-                // lanes 16..31 issue the page boxes (at most 16), lanes 0..n-1 the Y rows
-                const int bi = lane - 16;
-                if (bi >= 0 && bi < m.np * boxes) {
-                    const int p = bi / boxes, b = bi - p * boxes;
-                    tma_load_2d(sb + (p * nb + b) * kBoxBytes, &tmB, c0 + b * kBoxCols,
-                                page_of(m.pgb, p) * LORA_PAGE_ROWS, &sm.full[st]);
-                }
+                // lanes 16..31 issue the page boxes (a group of four 64-column
+                // blocks per lane), lanes 0..n-1 the Y rows
+                if (lane >= 16)
+                    issue_page_boxes(lane - 16, sb, &tmB, &tmB4, a.wide_out, a.d_out, m.np, nb, boxes, c0, m.pgb,
+                                     &sm.full[st]);
                 if (lane < n)
                     bulk_load(sb + kBoxRegion + lane * py, a.Y + (size_t)mytok * a.d_out + c0,
                               (uint32_t)((c1 - c0) * 4), &sm.full[st]);
@@ -785,9 +782,20 @@ size_t split_vpart_bytes(int T) { return (size_t)kSlices * (size_t)(T > 0 ? T : 
 int launch_split(const SplitArgs &s, lora_pool_s *pa, lora_pool_s *pb, cudaStream_t st) {
     int grid = 1;
     if (int rc = split_grid(&grid)) return rc;
-    CUtensorMap tmA, tmB;
+    CUtensorMap tmA, tmB, tmA4, tmB4;
     if (int rc = pool_tensor_map(pa, &tmA)) return rc;
     if (int rc = pool_tensor_map(pb, &tmB)) return rc;
+    const bool wide_in = pa->width >= 256, wide_out = pb->width >= 256;
+    if (wide_in) {
+        if (int rc = pool_tensor_map4(pa, &tmA4)) return rc;
+    } else {
+        tmA4 = tmA;
+    }
+    if (wide_out) {
+        if (int rc = pool_tensor_map4(pb, &tmB4)) return rc;
+    } else {
+        tmB4 = tmB;
+    }
     KSplit k;
     k.X = s.X; k.Y = s.Y; k.T = s.T; k.d_in = s.d_in; k.d_out = s.d_out; k.S = s.S;
     k.ranks = s.ranks; k.scales = s.scales; k.pt = s.pt;
@@ -795,6 +803,8 @@ int launch_split(const SplitArgs &s, lora_pool_s *pa, lora_pool_s *pb, cudaStrea
     k.rowsB = (long long)pb->num_pages * LORA_PAGE_ROWS;
     k.perm = s.perm; k.jobs = s.jobs; k.hdr = s.hdr; k.vpart = s.vpart; k.err = s.err;
     k.e_max = max(1, (s.d_out >> 3) / 8);
+    k.wide_in = wide_in;
+    k.wide_out = wide_out;
 
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
@@ -807,11 +817,11 @@ int launch_split(const SplitArgs &s, lora_pool_s *pa, lora_pool_s *pb, cudaStrea
     const long long t = s.T > 0 ? s.T : 1;
     cfg.gridDim = dim3((unsigned)(t * kSlices < grid ? t * kSlices : grid));
     cfg.dynamicSmemBytes = kShrinkSmemBytes;
-    if (int rc = cuda_check(cudaLaunchKernelEx(&cfg, shrink_part_kernel, tmA, k))) return rc;
+    if (int rc = cuda_check(cudaLaunchKernelEx(&cfg, shrink_part_kernel, tmA, tmA4, k))) return rc;
     count_launch();
     cfg.gridDim = dim3((unsigned)(t * k.e_max < grid ? t * k.e_max : grid));
     cfg.dynamicSmemBytes = kExpandSmemBytes;
-    if (int rc = cuda_check(cudaLaunchKernelEx(&cfg, expand_part_kernel, tmB, k))) return rc;
+    if (int rc = cuda_check(cudaLaunchKernelEx(&cfg, expand_part_kernel, tmB, tmB4, k))) return rc;
     count_launch();
     return LORA_OK;
 }

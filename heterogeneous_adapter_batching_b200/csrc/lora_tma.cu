@@ -59,4 +59,27 @@ int pool_tensor_map(lora_pool_s *pool, CUtensorMap *out) {
     return LORA_OK;
 }
 
+int pool_tensor_map4(lora_pool_s *pool, CUtensorMap *out) {
+    if (!pool || pool->width < 256) return LORA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> g(pool->mu);
+    if (!pool->tmap4_ok) {
+        EncodeTiledFn enc = encode_fn();
+        if (!enc) return LORA_ERR_CUDA;
+        // element (x, y, z) at base + 2 x + 2 width y + 128 z; x < width - 192 keeps
+        // every element of a box (x + 64 z + 63 < width) inside its row
+        const cuuint64_t rows = (cuuint64_t)pool->num_pages * LORA_PAGE_ROWS;
+        cuuint64_t dims[3] = {(cuuint64_t)pool->width - 192, rows, 4};
+        cuuint64_t strides[2] = {(cuuint64_t)pool->width * 2, 128};
+        cuuint32_t box[3] = {64, LORA_PAGE_ROWS, 4};
+        cuuint32_t es[3] = {1, 1, 1};
+        CUresult r = enc(&pool->tmap4, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, pool->base, dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return LORA_ERR_CUDA;
+        pool->tmap4_ok = true;
+    }
+    *out = pool->tmap4;
+    return LORA_OK;
+}
+
 }  // namespace lora
