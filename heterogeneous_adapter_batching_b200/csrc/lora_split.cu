@@ -55,23 +55,25 @@ constexpr int kThreads = kConsumers + 32;       // + one producer warp
 constexpr int kNTok = 8;                        // tokens per MMA (the N side)
 constexpr int kMaxNT = LORA_MAX_JOB_TOKENS / kNTok;
 constexpr int kMaxPages = LORA_MAX_RANK / LORA_PAGE_ROWS;
-constexpr int kStages = 3;
+constexpr int kSlots = 8;                                  // chunks in flight at most (barrier and header ring)
 constexpr int kBoxCols = 64;
 constexpr int kBoxBytes = LORA_PAGE_ROWS * kBoxCols * 2;   // 2 KB
-constexpr int kBoxRegion = 16 * kBoxBytes;                 // 16 boxes per stage
-constexpr int kRowRegion = 16640;                          // X or Y rows of a stage: 16 rows x 1040 B
-constexpr int kStageBytes = 50176;                         // kBoxRegion + kRowRegion, rounded up to 1 KB
+constexpr int kRowRegion = 16640;                          // most bytes of X or Y rows in one chunk: 16 rows x 1040 B
+constexpr int kMaxChunk = 16 * kBoxBytes + kRowRegion;     // 16 page boxes + rows
+constexpr int kShrinkArena = 159 * 1024;                   // byte rings the chunks are packed into
+constexpr int kExpandArena = 180 * 1024;
 constexpr int kTableSlots = 128;                           // slot tables up to this size live in shared memory
 constexpr long long kWaitLimit = 2000000000LL;             // cycles (~1 s)
 constexpr int kVPartFloats = LORA_MAX_JOB_TOKENS * LORA_MAX_RANK;
 constexpr int kVTileBytes = LORA_MAX_JOB_TOKENS * LORA_MAX_RANK * 2;   // one bf16 part of v
 
-static_assert(kStageBytes >= kBoxRegion + kRowRegion && kStageBytes % 1024 == 0, "stage layout");
+static_assert(kShrinkArena >= 3 * kMaxChunk && kExpandArena >= 3 * kMaxChunk, "rings hold at least three chunks");
 static_assert(kMaxNT * kNTok == LORA_MAX_JOB_TOKENS, "job size must be a whole number of MMA tiles");
 
-// What the producer tells the consumers about one stage.
+// What the producer tells the consumers about one chunk.
 struct ChunkHdr {
     int unit;          // >= 0: a chunk of a unit; -1: no more work
+    int off;           // byte offset of the chunk in the ring (1 KB aligned): page boxes, then rows
     int first, last;   // first / last chunk of its unit
     int c0, cols;      // first column, valid columns (a multiple of 8)
     int nb;            // 64-column boxes per page
@@ -84,29 +86,33 @@ struct ChunkHdr {
 };
 
 struct __align__(1024) ShrinkSmem {
-    unsigned char stage[kStages][kStageBytes];
+    unsigned char ring[kShrinkArena];
     float red[kCW * kMaxPages * kMaxNT * 128];   // the warps' partial sums of a unit
-    ChunkHdr hdr[kStages];
+    ChunkHdr hdr[kSlots];
     int4 pt[kTableSlots * 2];
     int ranks[kTableSlots];
-    uint64_t full[kStages], empty[kStages];
+    int asz[kSlots];                             // producer: ring bytes each chunk in flight holds
+    uint64_t full[kSlots], empty[kSlots];
     uint64_t red_full, red_free;
     int abort;
 };
 
 struct __align__(1024) ExpandSmem {
-    unsigned char stage[kStages][kStageBytes];
+    unsigned char ring[kExpandArena];
     float vst[2][kSlices][kVPartFloats];          // the four partials of a unit, double-buffered
     unsigned char vt[2 * kVTileBytes];            // v: bf16 high part [t][k] (16-byte groups swizzled), then low part
-    ChunkHdr hdr[kStages];
+    ChunkHdr hdr[kSlots];
     int4 pt[kTableSlots * 2];
     int ranks[kTableSlots];
     float scales[kTableSlots];
-    uint64_t full[kStages], empty[kStages];
+    int asz[kSlots];
+    uint64_t full[kSlots], empty[kSlots];
     uint64_t vfull[2], vempty[2];
     uint64_t vt_full, vt_free;
     int abort;
 };
+
+
 
 static_assert(sizeof(ShrinkSmem) + 1024 <= 227 * 1024, "shrink kernel: shared memory beyond the per-block limit");
 static_assert(sizeof(ExpandSmem) + 1024 <= 227 * 1024, "expand kernel: shared memory beyond the per-block limit");
@@ -159,6 +165,50 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
     const long long t0 = clock64();
     while (!mbar_try(a, parity) && clock64() - t0 < kWaitLimit / 8) {
     }
+}
+
+// The producer's side of a ring of chunks: chunk i uses barrier and header
+// slot i mod kSlots and a 1 KB aligned byte range of the arena; ranges are
+// handed out in order and come back in order (the consumers release chunks in
+// the order they take them), so the producer waits for the oldest chunks'
+// release until the next range and slot are free.
+struct Ring {
+    long long produced;   // bytes handed out (a chunk that would cross the end skips to the start)
+    long long released;   // bytes returned
+    int chunk;            // chunks handed out
+    int popped;           // chunks whose release the producer has seen
+};
+
+// Free the oldest chunk: wait for its release (all consumer warps arrived).
+template <class Sm>
+__device__ __forceinline__ bool ring_pop(Ring &rg, Sm &sm, int32_t *err) {
+    const int ps = rg.popped % kSlots;
+    if (!wait_w(&sm.empty[ps], (uint32_t)((rg.popped / kSlots) & 1), sm, err)) return false;
+    rg.released += sm.asz[ps];
+    ++rg.popped;
+    return true;
+}
+
+// Hand out `bytes` (rounded up to 1 KB) and the next slot; `before_block` runs
+// once, before the first wait this call would make.  Returns the byte offset,
+// or -1 when a wait failed.
+template <int kArena, class Sm, class F>
+__device__ __forceinline__ int ring_alloc(Ring &rg, Sm &sm, int bytes, int32_t *err, F &&before_block) {
+    const int need = (bytes + 1023) & ~1023;
+    const int at = (int)(rg.produced % kArena);
+    const int pad = at + need > kArena ? kArena - at : 0;
+    bool called = false;
+    while (rg.produced + pad + need - rg.released > kArena || rg.chunk - rg.popped >= kSlots) {
+        if (!called) {
+            before_block();
+            called = true;
+        }
+        if (rg.popped == rg.chunk || !ring_pop(rg, sm, err)) return -1;
+    }
+    if (threadIdx.x % 32 == 0) sm.asz[rg.chunk % kSlots] = pad + need;
+    __syncwarp();
+    rg.produced += pad + need;
+    return pad ? 0 : at;
 }
 
 // One slot's rank, pages and scale, validated against both pools (a unit is
@@ -253,7 +303,7 @@ shrink_part_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kSlots; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], kCW);
         }
@@ -277,7 +327,7 @@ shrink_part_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         const int n_units = n_jobs * kSlices;
         const unsigned Gi = (unsigned)a.d_in >> 3;
         const int G = gridDim.x;
-        int chunk = 0;
+        Ring rg = {0, 0, 0, 0};
         bool ok = true;
         // the job record two units ahead and the slot tables one unit ahead are
         // in flight while the current unit streams
@@ -315,44 +365,44 @@ shrink_part_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             const int nb = min(16 / m.np, nt > 1 ? 8 : 16);
             const int cw = nb * kBoxCols, px = cw * 2 + 16;
             const int nch = (in1 - in0 + cw - 1) / cw;
+            const int box_bytes = m.np * nb * kBoxBytes;
             for (int c = 0; c < nch; ++c) {
-                const int st = chunk % kStages;
-                if (!wait_w(&sm.empty[st], ((chunk / kStages) & 1) ^ 1, sm, a.err)) { ok = false; break; }
+                const int off = ring_alloc<kShrinkArena>(rg, sm, box_bytes + nt * kNTok * px, a.err, [] {});
+                if (off < 0) { ok = false; break; }
+                const int st = rg.chunk % kSlots;
                 const int c0 = in0 + c * cw, c1 = min(c0 + cw, in1);
                 const int boxes = (c1 - c0 + kBoxCols - 1) / kBoxCols;
                 if (lane == 0) {
                     ChunkHdr &h = sm.hdr[st];
-                    h.unit = u; h.first = c == 0; h.last = c == nch - 1;
+                    h.unit = u; h.off = off; h.first = c == 0; h.last = c == nch - 1;
                     h.c0 = c0; h.cols = c1 - c0; h.nb = nb; h.np = m.np; h.r = m.r; h.n = n; h.nt = nt;
                     h.lo = in0; h.hi = in1; h.q0 = q0; h.slice = s; h.scale = 0.f;
                     mbar_expect_tx(&sm.full[st], (uint32_t)(m.np * boxes * kBoxBytes + n * (c1 - c0) * 2));
                 }
                 __syncwarp();
-                unsigned char *sb = sm.stage[st];
+                unsigned char *sb = sm.ring + off;
                 // lanes 16..31 issue the page boxes (a group of four 64-column
                 // blocks per lane), lanes 0..n-1 the X rows
                 if (lane >= 16)
                     issue_page_boxes(lane - 16, sb, &tmA, &tmA4, a.wide_in, a.d_in, m.np, nb, boxes, c0, m.pga,
                                      &sm.full[st]);
                 if (lane < n)
-                    bulk_load(sb + kBoxRegion + lane * px, a.X + (size_t)mytok * a.d_in + c0, (uint32_t)((c1 - c0) * 2),
+                    bulk_load(sb + box_bytes + lane * px, a.X + (size_t)mytok * a.d_in + c0, (uint32_t)((c1 - c0) * 2),
                               &sm.full[st]);
-                ++chunk;
+                ++rg.chunk;
             }
         }
-        if (ok) {   // end marker
-            const int st = chunk % kStages;
-            if (wait_w(&sm.empty[st], ((chunk / kStages) & 1) ^ 1, sm, a.err)) {
-                if (lane == 0) {
-                    sm.hdr[st].unit = -1;
-                    mbar_arrive(&sm.full[st]);
-                }
-                ++chunk;
+        if (ok && ring_alloc<kShrinkArena>(rg, sm, 0, a.err, [] {}) >= 0) {   // end marker
+            const int st = rg.chunk % kSlots;
+            if (lane == 0) {
+                sm.hdr[st].unit = -1;
+                mbar_arrive(&sm.full[st]);
             }
+            ++rg.chunk;
         }
         if (lane == 0)
-            for (int i = (chunk > kStages ? chunk - kStages : 0); i < chunk; ++i)
-                drain_wait(&sm.full[i % kStages], (i / kStages) & 1);
+            for (int i = max(rg.popped, rg.chunk - kSlots); i < rg.chunk; ++i)
+                drain_wait(&sm.full[i % kSlots], (i / kSlots) & 1);
         return;
     }
 
@@ -361,12 +411,12 @@ shrink_part_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     float acc[kMaxPages][kMaxNT][4];
     int chunk = 0, nred = 0;
     while (true) {
-        const int st = chunk % kStages;
-        if (!wait_w(&sm.full[st], (chunk / kStages) & 1, sm, a.err)) break;
+        const int st = chunk % kSlots;
+        if (!wait_w(&sm.full[st], (chunk / kSlots) & 1, sm, a.err)) break;
         const ChunkHdr &h = sm.hdr[st];
         if (h.unit < 0) break;
         const int first = h.first, last = h.last, c0 = h.c0, cols = h.cols, nb = h.nb, np = h.np, r = h.r;
-        const int n = h.n, nt = h.nt, lo = h.lo, hi = h.hi, q0 = h.q0, slice = h.slice;
+        const int n = h.n, nt = h.nt, lo = h.lo, hi = h.hi, q0 = h.q0, slice = h.slice, off = h.off;
         if (first) {
 #pragma unroll
             for (int p = 0; p < kMaxPages; ++p)
@@ -378,8 +428,8 @@ shrink_part_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         const int px = nb * kBoxCols * 2 + 16;
         const int nks = (cols + 15) >> 4;
         const int kbase = (c0 - lo) >> 4;
-        const uint32_t sb = smem_u32(sm.stage[st]);
-        const uint32_t xb = sb + kBoxRegion;
+        const uint32_t sb = smem_u32(sm.ring + off);
+        const uint32_t xb = sb + np * nb * kBoxBytes;
         const bool tok0 = g8 < n, tok1 = kNTok + g8 < n;
         int kk = warp - kbase % kCW;
         if (kk < 0) kk += kCW;
@@ -496,7 +546,7 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kSlots; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], kCW);
         }
@@ -524,7 +574,8 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
         const int n_units = n_jobs * E;
         const long long Go = a.d_out >> 3;
         const unsigned qmask = quarter_mask(a.d_in);
-        int chunk = 0, nv = 0;
+        Ring rg = {0, 0, 0, 0};
+        int nv = 0;
         bool ok = true, waited = false;
         auto wait_shrink = [&]() {
             asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -582,16 +633,31 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
                 ++nv;
                 return true;
             };
-            if (waited && !issue_v()) { ok = false; break; }
-            const int early = min(kStages, nch);   // chunks issued before the first unit's partials
-            for (int c = 0; c < nch; ++c) {
-                const int st = chunk % kStages;
-                if (!wait_w(&sm.empty[st], ((chunk / kStages) & 1) ^ 1, sm, a.err)) { ok = false; break; }
+            // The first unit's partials are fetched (after waiting for the
+            // shrink grid) just before the producer would first have to wait
+            // for ring space, or after its last chunk: until then its B pages and
+            // Y rows stream in while the shrink kernel still runs.
+            bool pending_v = true;
+            if (waited) {
+                if (!issue_v()) { ok = false; break; }
+                pending_v = false;
+            }
+            auto before_block = [&]() {
+                if (!pending_v) return;
+                if (!waited) wait_shrink();
+                if (!issue_v()) ok = false;
+                pending_v = false;
+            };
+            const int box_bytes = m.np * nb * kBoxBytes;
+            for (int c = 0; c < nch && ok; ++c) {
+                const int off = ring_alloc<kExpandArena>(rg, sm, box_bytes + n * py, a.err, before_block);
+                if (off < 0 || !ok) { ok = false; break; }
+                const int st = rg.chunk % kSlots;
                 const int c0 = out0 + c * cw, c1 = min(c0 + cw, out1);
                 const int boxes = (c1 - c0 + kBoxCols - 1) / kBoxCols;
                 if (lane == 0) {
                     ChunkHdr &h = sm.hdr[st];
-                    h.unit = u; h.first = c == 0; h.last = c == nch - 1;
+                    h.unit = u; h.off = off; h.first = c == 0; h.last = c == nch - 1;
                     h.c0 = c0; h.cols = c1 - c0; h.nb = nb; h.np = m.np; h.r = m.r; h.n = n; h.nt = nt;
                     h.lo = out0; h.hi = out1; h.q0 = q0; h.slice = vb; h.scale = m.scale;
                 }
@@ -600,36 +666,31 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
                 if (lane == 0)
                     mbar_expect_tx(&sm.full[st], (uint32_t)(m.np * boxes * kBoxBytes + n * (c1 - c0) * 4));
                 __syncwarp();
-                unsigned char *sb = sm.stage[st];
+                unsigned char *sb = sm.ring + off;
                 // lanes 16..31 issue the page boxes (a group of four 64-column
                 // blocks per lane), lanes 0..n-1 the Y rows
                 if (lane >= 16)
                     issue_page_boxes(lane - 16, sb, &tmB, &tmB4, a.wide_out, a.d_out, m.np, nb, boxes, c0, m.pgb,
                                      &sm.full[st]);
                 if (lane < n)
-                    bulk_load(sb + kBoxRegion + lane * py, a.Y + (size_t)mytok * a.d_out + c0,
+                    bulk_load(sb + box_bytes + lane * py, a.Y + (size_t)mytok * a.d_out + c0,
                               (uint32_t)((c1 - c0) * 4), &sm.full[st]);
-                ++chunk;
-                if (!waited && c == early - 1) {
-                    wait_shrink();
-                    if (!issue_v()) { ok = false; break; }
-                }
+                ++rg.chunk;
             }
+            if (ok) before_block();   // a unit whose chunks all fit without waiting
         }
         if (!waited) wait_shrink();
-        if (ok) {   // end marker
-            const int st = chunk % kStages;
-            if (wait_w(&sm.empty[st], ((chunk / kStages) & 1) ^ 1, sm, a.err)) {
-                if (lane == 0) {
-                    sm.hdr[st].unit = -1;
-                    mbar_arrive(&sm.full[st]);
-                }
-                ++chunk;
+        if (ok && ring_alloc<kExpandArena>(rg, sm, 0, a.err, [] {}) >= 0) {   // end marker
+            const int st = rg.chunk % kSlots;
+            if (lane == 0) {
+                sm.hdr[st].unit = -1;
+                mbar_arrive(&sm.full[st]);
             }
+            ++rg.chunk;
         }
         if (lane == 0) {
-            for (int i = (chunk > kStages ? chunk - kStages : 0); i < chunk; ++i)
-                drain_wait(&sm.full[i % kStages], (i / kStages) & 1);
+            for (int i = max(rg.popped, rg.chunk - kSlots); i < rg.chunk; ++i)
+                drain_wait(&sm.full[i % kSlots], (i / kSlots) & 1);
             for (int i = (nv > 2 ? nv - 2 : 0); i < nv; ++i) drain_wait(&sm.vfull[i & 1], (i >> 1) & 1);
         }
         return;
@@ -641,12 +702,12 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
     const unsigned qmask = quarter_mask(a.d_in);
     int chunk = 0, nunit = 0;
     while (true) {
-        const int st = chunk % kStages;
-        if (!wait_w(&sm.full[st], (chunk / kStages) & 1, sm, a.err)) break;
+        const int st = chunk % kSlots;
+        if (!wait_w(&sm.full[st], (chunk / kSlots) & 1, sm, a.err)) break;
         const ChunkHdr &h = sm.hdr[st];
         if (h.unit < 0) break;
         const int first = h.first, last = h.last, c0 = h.c0, cols = h.cols, nb = h.nb, np = h.np, r = h.r;
-        const int n = h.n, nt = h.nt, hi = h.hi, vb = h.slice;
+        const int n = h.n, nt = h.nt, hi = h.hi, vb = h.slice, off = h.off;
         const float sc = h.scale;
         if (first) {
             // v = the four quarters' partials added in quarter order, split into
@@ -688,8 +749,8 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
         // congruent to w mod 15; Y rows of the chunk sit in the stage
         const int cw = nb * kBoxCols, py4 = cw + 4;   // Y row pitch in floats
         const int nmt = (cols + 15) >> 4;
-        const uint32_t sb = smem_u32(sm.stage[st]);
-        float *ys = reinterpret_cast<float *>(sm.stage[st] + kBoxRegion);
+        const uint32_t sb = smem_u32(sm.ring + off);
+        float *ys = reinterpret_cast<float *>(sm.ring + off + np * nb * kBoxBytes);
         const uint32_t vbase = vt_base + ((lj >> 1) ? kVTileBytes : 0);
         const int krow = li + 8 * (lj >> 1);
         for (int mt = warp; mt < nmt; mt += kCW) {
