@@ -59,7 +59,9 @@ constexpr int kSlots = 8;                                  // chunks in flight a
 constexpr int kBoxCols = 64;
 constexpr int kBoxBytes = LORA_PAGE_ROWS * kBoxCols * 2;   // 2 KB
 constexpr int kRowRegion = 16640;                          // most bytes of X or Y rows in one chunk: 16 rows x 1040 B
-constexpr int kMaxChunk = 16 * kBoxBytes + kRowRegion;     // 16 page boxes + rows
+constexpr int kMaxBoxes = 32;                              // page boxes in one chunk at most (64 KB)
+constexpr int kMaxChunk = kMaxBoxes * kBoxBytes + kRowRegion;
+constexpr int kTilesPerWarp = 3;                           // expand: m-tiles a warp runs at once
 constexpr int kShrinkArena = 159 * 1024;                   // byte rings the chunks are packed into
 constexpr int kExpandArena = 180 * 1024;
 constexpr int kTableSlots = 128;                           // slot tables up to this size live in shared memory
@@ -67,7 +69,8 @@ constexpr long long kWaitLimit = 2000000000LL;             // cycles (~1 s)
 constexpr int kVPartFloats = LORA_MAX_JOB_TOKENS * LORA_MAX_RANK;
 constexpr int kVTileBytes = LORA_MAX_JOB_TOKENS * LORA_MAX_RANK * 2;   // one bf16 part of v
 
-static_assert(kShrinkArena >= 3 * kMaxChunk && kExpandArena >= 3 * kMaxChunk, "rings hold at least three chunks");
+static_assert(kShrinkArena >= 3 * (16 * kBoxBytes + kRowRegion) && kExpandArena >= 2 * kMaxChunk,
+              "the rings hold at least three shrink or two expand chunks");
 static_assert(kMaxNT * kNTok == LORA_MAX_JOB_TOKENS, "job size must be a whole number of MMA tiles");
 
 // What the producer tells the consumers about one chunk.
@@ -619,7 +622,7 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
             if (out1 <= out0) continue;
             const int nt = (n + kNTok - 1) / kNTok;
             const int ylim = ((kRowRegion / n) - 16) / 4 / kBoxCols;   // Y rows of a chunk fit the row region
-            const int nb = max(1, min(16 / m.np, ylim));
+            const int nb = max(1, min(min(kMaxBoxes / m.np, 16), ylim));
             const int cw = nb * kBoxCols, py = cw * 4 + 16;
             const int nch = (out1 - out0 + cw - 1) / cw;
             const int vb = nv & 1;
@@ -753,47 +756,73 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
         float *ys = reinterpret_cast<float *>(sm.ring + off + np * nb * kBoxBytes);
         const uint32_t vbase = vt_base + ((lj >> 1) ? kVTileBytes : 0);
         const int krow = li + 8 * (lj >> 1);
-        for (int mt = warp; mt < nmt; mt += kCW) {
-            float d[kMaxNT][4];
+        // A warp runs up to kTilesPerWarp of its m-tiles (mt, mt + 15, mt + 30)
+        // at once: their MMA chains are independent and interleave, while each
+        // accumulator still sees pages in order, high part before low part.
+        for (int mt0 = warp; mt0 < nmt; mt0 += kTilesPerWarp * kCW) {
+            float d[kTilesPerWarp][kMaxNT][4];
+            uint32_t offA[kTilesPerWarp];
+            bool has[kTilesPerWarp];
 #pragma unroll
-            for (int jj = 0; jj < kMaxNT; ++jj)
+            for (int q = 0; q < kTilesPerWarp; ++q) {
+                const int mt = mt0 + q * kCW;
+                has[q] = mt < nmt;
+                offA[q] = (uint32_t)((mt >> 2) * kBoxBytes + krow * 128 + (((2 * (mt & 3) + (lj & 1)) ^ li) << 4));
 #pragma unroll
-                for (int i = 0; i < 4; ++i) d[jj][i] = 0.f;
-            const uint32_t offA = (uint32_t)((mt >> 2) * kBoxBytes + krow * 128 + (((2 * (mt & 3) + (lj & 1)) ^ li) << 4));
+                for (int jj = 0; jj < kMaxNT; ++jj)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) d[q][jj][i] = 0.f;
+            }
 #pragma unroll 1
             for (int p = 0; p < np; ++p) {
-                uint32_t af[4];
-                ldsm_x4_t(sb + (uint32_t)(p * nb * kBoxBytes) + offA, af);
+                uint32_t af[kTilesPerWarp][4];
+#pragma unroll
+                for (int q = 0; q < kTilesPerWarp; ++q)
+                    if (has[q]) ldsm_x4_t(sb + (uint32_t)(p * nb * kBoxBytes) + offA[q], af[q]);
 #pragma unroll
                 for (int jj = 0; jj < kMaxNT; ++jj) {
                     if (jj < nt) {
                         uint32_t bv[4];
                         ldsm_x4(vbase + swz(jj * kNTok + li, LORA_MAX_RANK * 2, 2 * p + (lj & 1)), bv);
-                        mma_bf16(d[jj], af, bv[0], bv[1]);
-                        mma_bf16(d[jj], af, bv[2], bv[3]);
+#pragma unroll
+                        for (int q = 0; q < kTilesPerWarp; ++q)
+                            if (has[q]) mma_bf16(d[q][jj], af[q], bv[0], bv[1]);
+#pragma unroll
+                        for (int q = 0; q < kTilesPerWarp; ++q)
+                            if (has[q]) mma_bf16(d[q][jj], af[q], bv[2], bv[3]);
                     }
                 }
             }
             // fragment (column g8 / g8 + 8, tokens 2 tig, 2 tig + 1) into the Y rows
 #pragma unroll
-            for (int jj = 0; jj < kMaxNT; ++jj) {
-                if (jj < nt) {
+            for (int q = 0; q < kTilesPerWarp; ++q) {
+                if (!has[q]) continue;
+                const int mt = mt0 + q * kCW;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int t = jj * kNTok + 2 * tig + (i & 1), cc = mt * 16 + g8 + 8 * (i >> 1);
-                        if (t < n && c0 + cc < hi) {
-                            float *y = ys + t * py4 + cc;
-                            *y = fmaf(sc, d[jj][i], *y);
+                for (int jj = 0; jj < kMaxNT; ++jj) {
+                    if (jj < nt) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int t = jj * kNTok + 2 * tig + (i & 1), cc = mt * 16 + g8 + 8 * (i >> 1);
+                            if (t < n && c0 + cc < hi) {
+                                float *y = ys + t * py4 + cc;
+                                *y = fmaf(sc, d[q][jj][i], *y);
+                            }
                         }
                     }
                 }
             }
             __syncwarp();
-            for (int idx = lane; idx < n * 4; idx += 32) {
-                const int t = idx >> 2, col = mt * 16 + 4 * (idx & 3);
-                if (c0 + col < hi)
-                    *reinterpret_cast<float4 *>(a.Y + (size_t)h.tok[t] * a.d_out + c0 + col) =
-                        *reinterpret_cast<const float4 *>(ys + t * py4 + col);
+#pragma unroll
+            for (int q = 0; q < kTilesPerWarp; ++q) {
+                if (!has[q]) continue;
+                const int mt = mt0 + q * kCW;
+                for (int idx = lane; idx < n * 4; idx += 32) {
+                    const int t = idx >> 2, col = mt * 16 + 4 * (idx & 3);
+                    if (c0 + col < hi)
+                        *reinterpret_cast<float4 *>(a.Y + (size_t)h.tok[t] * a.d_out + c0 + col) =
+                            *reinterpret_cast<const float4 *>(ys + t * py4 + col);
+                }
             }
         }
         // the Y rows were written through the generic proxy; order that before
