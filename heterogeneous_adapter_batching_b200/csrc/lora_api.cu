@@ -334,11 +334,22 @@ static int run_tiles(const uint16_t *X, int T, int d_in, const lora_projection_t
 }
 
 // Which gather path a call takes (both give bit-identical results).
-static bool use_split(int nproj) {
+// LORA_GATHER_AUTO: the split path where many distinct adapters are likely
+// (a pool of at least kSplitMinSlots slots and at least kSplitMinTokens
+// tokens, one projection).  Measured on B200 at the 7B/8B shapes, the cluster
+// kernel is faster with few gather jobs (decode over a small pool, one shared
+// adapter, mixed-rank MLPs over 128 slots: 10-35 % ahead), the split pair with
+// many (64 and 512 distinct rank-64 adapters at d_out 14336: 23 % and 36 %
+// ahead).  The job count itself is known only on the device, so the host
+// decides from the pool size and the token count.
+constexpr int kSplitMinSlots = 256;
+constexpr int kSplitMinTokens = 64;
+
+static bool use_split(int nproj, int T, int num_slots) {
     const int p = opt_gather_path();
     if (p == LORA_GATHER_SPLIT) return true;
     if (p == LORA_GATHER_CLUSTER) return false;
-    return nproj == 1;
+    return nproj == 1 && num_slots >= kSplitMinSlots && T >= kSplitMinTokens;
 }
 
 // The apply kernels over a plan already in ws: the short segments of every
@@ -348,7 +359,7 @@ static bool use_split(int nproj) {
 static int run_planned(const uint16_t *X, int T, int d_in, int num_slots, const lora_projection_t *pr, int nproj,
                        void *ws, int32_t *err_dev, cudaStream_t st) {
     const PlanOut o = plan_out(ws, T, num_slots, nullptr, nullptr);
-    if (use_split(nproj)) {
+    if (use_split(nproj, T, num_slots)) {
         float *vpart = reinterpret_cast<float *>(static_cast<char *>(ws) + ws_layout(T, num_slots).vpart);
         for (int p = 0; p < nproj; ++p) {
             SplitArgs s = {};

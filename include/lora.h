@@ -388,7 +388,9 @@ int lora_slot_cache_stats(lora_slot_cache_t c, int64_t *hits, int64_t *misses, i
 #define LORA_OPT_GATHER_PATH    3   /* kernels for short segments in lora_apply, lora_apply_planned and the
                                         multi-projection calls: LORA_GATHER_AUTO (default), LORA_GATHER_CLUSTER
                                         or LORA_GATHER_SPLIT; every choice gives bit-identical results */
-#define LORA_GATHER_AUTO        0   /* the library picks by the call's shape */
+#define LORA_GATHER_AUTO        0   /* the library picks by the call's shape: the split pair for one projection
+                                        with num_slots >= 256 and T >= 64 (many distinct adapters likely),
+                                        the cluster kernel otherwise */
 #define LORA_GATHER_CLUSTER     1   /* one kernel: 4-CTA clusters exchange the shrink partials on chip */
 #define LORA_GATHER_SPLIT       2   /* a shrink kernel writes per-quarter partials to the workspace, an expand
                                         kernel adds them and updates Y; one pair per projection */
