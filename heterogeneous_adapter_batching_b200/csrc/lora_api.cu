@@ -320,7 +320,7 @@ static GatherProj gather_proj(float *Y, int d_out, const int32_t *ranks, const f
 
 // The tensor-core launch of a plan with long runs: one for all projections.
 static int run_tiles(const uint16_t *X, int T, int d_in, const lora_projection_t *pr, int nproj, const PlanOut &o,
-                     int32_t *err_dev, cudaStream_t st) {
+                     float *vpart, int32_t *err_dev, cudaStream_t st) {
     if (!plan_uses_tiles(T)) return LORA_OK;
     TileArgs ta = {};
     ta.X = X; ta.T = T; ta.d_in = d_in; ta.nproj = nproj;
@@ -330,6 +330,7 @@ static int run_tiles(const uint16_t *X, int T, int d_in, const lora_projection_t
         q.pt = pr[p].page_table; q.pa = pr[p].pa; q.pb = pr[p].pb;
     }
     ta.tiles = o.tiles; ta.hdr = o.header; ta.err = err_dev; ta.long_thresh = opt_long_segment();
+    ta.vpart = vpart;
     return launch_tiles(ta, st, true);
 }
 
@@ -359,8 +360,11 @@ static bool use_split(int nproj, int T, int num_slots) {
 static int run_planned(const uint16_t *X, int T, int d_in, int num_slots, const lora_projection_t *pr, int nproj,
                        void *ws, int32_t *err_dev, cudaStream_t st) {
     const PlanOut o = plan_out(ws, T, num_slots, nullptr, nullptr);
+    // per-quarter partials of v: the split gather pair's (by short-token
+    // position), then the tile shrink's (by token); the tile launches wait for
+    // the gather kernels before they write
+    float *vpart = reinterpret_cast<float *>(static_cast<char *>(ws) + ws_layout(T, num_slots).vpart);
     if (use_split(nproj, T, num_slots)) {
-        float *vpart = reinterpret_cast<float *>(static_cast<char *>(ws) + ws_layout(T, num_slots).vpart);
         for (int p = 0; p < nproj; ++p) {
             SplitArgs s = {};
             s.X = X; s.Y = pr[p].Y; s.T = T; s.d_in = d_in; s.d_out = pr[p].d_out; s.S = num_slots;
@@ -368,7 +372,7 @@ static int run_planned(const uint16_t *X, int T, int d_in, int num_slots, const 
             s.perm = o.perm_short; s.jobs = o.jobs; s.hdr = o.header; s.vpart = vpart; s.err = err_dev;
             if (int rc = launch_split(s, pr[p].pa, pr[p].pb, st)) return rc;
         }
-        return run_tiles(X, T, d_in, pr, nproj, o, err_dev, st);
+        return run_tiles(X, T, d_in, pr, nproj, o, vpart, err_dev, st);
     }
     GatherArgs a = {};
     a.X = X; a.T = T; a.d_in = d_in; a.S = num_slots; a.nproj = nproj;
@@ -380,7 +384,7 @@ static int run_planned(const uint16_t *X, int T, int d_in, int num_slots, const 
     }
     a.perm = o.perm_short; a.jobs = o.jobs; a.hdr = o.header; a.err = err_dev;
     if (int rc = launch_gather(kApply, a, pa, pb, st, true)) return rc;
-    return run_tiles(X, T, d_in, pr, nproj, o, err_dev, st);
+    return run_tiles(X, T, d_in, pr, nproj, o, vpart, err_dev, st);
 }
 
 static lora_projection_t one_proj(float *Y, int d_out, const int32_t *ranks, const float *scales,

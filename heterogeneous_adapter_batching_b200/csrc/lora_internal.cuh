@@ -197,6 +197,9 @@ struct TileArgs {
     const PlanHeader *hdr;
     int32_t *err;
     int long_thresh;     // long-segment threshold the plan used
+    float *vpart;        // workspace for v's per-quarter partials ([4][T][64] fp32), or null: with one
+                         // projection and vpart set, the shrink of every tile runs once in its own
+                         // launch and a second launch streams B and Y; else one fused launch
 };
 int launch_tiles(const TileArgs &a, cudaStream_t st, bool pdl);
 bool tiles_supported();

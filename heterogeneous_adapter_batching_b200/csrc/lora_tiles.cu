@@ -43,26 +43,53 @@ constexpr int kM = 128;              // tokens per tile (MMA M)
 constexpr int kKB = 64;              // shrink K block: one 128-byte swizzle row of bf16
 constexpr int kNB = 64;              // expand n-tile width (MMA N)
 constexpr int kStages = 3;           // shrink pipeline depth
-constexpr int kBuf = 3;              // expand pipeline depth (B tile, Y tile, accumulator)
 constexpr int kThreads = 256;
-constexpr uint32_t kTmemCols = 256;  // D1 [0,64), D2[b] [64 + 64b, 128 + 64b) for b < 3
 constexpr long long kWaitLimit = 2000000000LL;
 
-struct TileSmem {
-    __nv_bfloat16 xs[kStages][kM * kKB];      // 16 KB each, K-major SW128
-    __nv_bfloat16 as[kStages][64 * kKB];      //  8 KB each, up to 4 pages x 16 rows
+// Launch modes.  kFused: one kernel does a unit's shrink and its expand (any
+// number of projections).  kShrinkQ + kExpandV: the shrink of every (tile,
+// quarter of d_in) once, into fp32 partials in the workspace, then a kernel
+// that only streams B and Y and rebuilds v from the partials (one projection).
+constexpr int kFused = 0, kShrinkQ = 1, kExpandV = 2;
+constexpr int kSlicesQ = 4;          // d_in quarters of the shrink-only launch
+
+// Shared memory of a mode: STAGES shrink stages, BUF expand buffers (B
+// n-tile, its accumulator, the Y tile).  Every array is a whole number of KB,
+// so each starts 1024-byte aligned as the 128-byte swizzle needs.
+template <int STAGES, int BUF>
+struct TileSmemT {
+    static constexpr int kBufN = BUF;
+    static constexpr int kStageN = STAGES;
+    __nv_bfloat16 xs[STAGES][kM * kKB];       // 16 KB each, K-major SW128
+    __nv_bfloat16 as[STAGES][64 * kKB];       //  8 KB each, up to 4 pages x 16 rows
     __nv_bfloat16 vs[kM * 64];                // 16 KB, v high part (expand A operand), K-major SW128
     __nv_bfloat16 vl[kM * 64];                // 16 KB, v low part (v - high), same layout
-    __nv_bfloat16 bs[kBuf][64 * kNB];         //  8 KB each, B n-tile, rank rows x 64 cols (MN-major SW128)
-    float ys[kBuf][kM * kNB];                 // 32 KB each, two SW128 boxes of [128 rows x 32 cols]
-    uint64_t full[kStages], empty[kStages];
-    uint64_t bfull[kBuf], bempty[kBuf], yfull[kBuf], yempty[kBuf], accfull[kBuf], accempty[kBuf];
-    uint64_t shrink_done, d1_empty, v_ready, v_empty, mma_drain;
+    __nv_bfloat16 bs[BUF][64 * kNB];          //  8 KB each, B n-tile, rank rows x 64 cols (MN-major SW128)
+    float ys[BUF][kM * kNB];                  // 32 KB each, two SW128 boxes of [128 rows x 32 cols]
+    uint64_t full[STAGES], empty[STAGES];
+    uint64_t bfull[BUF], bempty[BUF], yfull[BUF], yempty[BUF], accfull[BUF], accempty[BUF];
+    uint64_t shrink_done, d1_empty, v_ready, v_full, v_empty, mma_drain;
     uint32_t tmem_base;
+    int reduce;   // kShrinkQ: this CTA finishes the current tile's v
     int abort;
 };
 
-static_assert(sizeof(TileSmem) + 1024 <= 227 * 1024, "tiles kernel: shared memory beyond the per-block limit");
+template <int MODE>
+struct SmemOf {
+    using type = TileSmemT<MODE == kExpandV ? 1 : (MODE == kShrinkQ ? 6 : kStages), MODE == kShrinkQ ? 1 : (MODE == kExpandV ? 4 : 3)>;
+};
+// Tensor-memory columns: the shrink's D1 of quarter q at [64 q, 64 q + 64)
+// (kShrinkQ: its one quarter at [0, 64)); expand accumulator b at
+// [kAccCol + 64 b, kAccCol + 64 b + 64).
+constexpr int kAccCol = 64 * kSlicesQ;
+template <int MODE>
+constexpr uint32_t tmem_cols() { return MODE == kShrinkQ ? 64u : 512u; }
+
+static_assert(sizeof(SmemOf<kFused>::type) + 1024 <= 227 * 1024, "tiles kernel: shared memory beyond the per-block limit");
+static_assert(sizeof(SmemOf<kShrinkQ>::type) + 1024 <= 227 * 1024, "tiles kernel: shared memory beyond the per-block limit");
+static_assert(sizeof(SmemOf<kExpandV>::type) + 1024 <= 227 * 1024, "tiles kernel: shared memory beyond the per-block limit");
+static_assert(kAccCol + 64 * SmemOf<kExpandV>::type::kBufN <= (int)tmem_cols<kExpandV>() &&
+              kAccCol + 64 * SmemOf<kFused>::type::kBufN <= (int)tmem_cols<kFused>(), "accumulators beyond the allocation");
 
 __device__ __forceinline__ uint32_t su32(const void *p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
@@ -78,7 +105,8 @@ __device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t par) {
 // Bounded wait: true when the phase completed.  On timeout it raises the
 // CTA's abort flag and records LORA_DEV_ERR_TIMEOUT; once the flag is up every
 // wait returns false at once and each role stops issuing work.
-__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t par, TileSmem &sm, int32_t *err) {
+template <class Sm>
+__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t par, Sm &sm, int32_t *err) {
     const uint32_t a = su32(b);
     if (mbar_try(a, par)) return true;
     const long long t0 = clock64();
@@ -100,7 +128,8 @@ __device__ __forceinline__ void drain_wait(uint64_t *b, uint32_t par) {
     while (!mbar_try(a, par) && clock64() - t0 < kWaitLimit / 8) {
     }
 }
-__device__ __forceinline__ bool aborted(const TileSmem &sm) { return *(volatile const int *)&sm.abort != 0; }
+template <class Sm>
+__device__ __forceinline__ bool aborted(const Sm &sm) { return *(volatile const int *)&sm.abort != 0; }
 __device__ __forceinline__ void mbar_arrive(uint64_t *b) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
 }
@@ -185,13 +214,16 @@ struct KTile {
     int nproj;
     KTileProj proj[NP];
     int jpre[NP + 1];    // n-tiles of the projections before p, within one tile
-    const int4 *tiles;
+    int4 *tiles;         // the plan's tiles; kShrinkQ counts a tile's finished quarters in .w (0 between launches)
     const PlanHeader *hdr;
     int32_t *err;
+    float *vpart;        // kShrinkQ / kExpandV: [kSlicesQ][T][LORA_MAX_RANK] fp32 partials of v; the finished
+                         // v of row t as bf16 high part, low part in the first 256 bytes of quarter 0's row t
 };
 
 template <int NP>
 struct TileMaps {
+    CUtensorMap V;       // kExpandV: quarter 0 of the partials seen as bf16 [T][128] (v high | v low), SW128 boxes
     CUtensorMap X;
     CUtensorMap A[NP];
     CUtensorMap B[NP];
@@ -199,6 +231,7 @@ struct TileMaps {
 };
 
 struct UnitInfo {
+    int tile;
     int slot, row0, ntok, r, n1, np, j0, j1;
     int p;       // projection
     bool skip;
@@ -210,6 +243,7 @@ __device__ __forceinline__ UnitInfo unit_info(const KTile<NP> &a, int tile, int 
     UnitInfo ui;
     const int4 t = a.tiles[tile];
     const KTileProj &pr = a.proj[pj];
+    ui.tile = tile;
     ui.slot = t.x;
     ui.row0 = t.y;
     ui.ntok = t.z;
@@ -292,31 +326,56 @@ __device__ __forceinline__ bool next_unit(const KTile<NP> &a, UnitIter &u, UnitI
     return true;
 }
 
+// Units of the shrink-only launch: (tile, quarter q of the K blocks), handed
+// out round robin.  Quarter q covers K blocks [nkb q / 4, nkb (q + 1) / 4);
+// with fewer than four K blocks some quarters are empty and hold no partial.
+__device__ __forceinline__ void quarter_blocks(int nkb, int q, int &kb0, int &kb1) {
+    kb0 = nkb * q / kSlicesQ;
+    kb1 = nkb * (q + 1) / kSlicesQ;
+}
+
 template <int NP>
+__device__ __forceinline__ bool next_qunit(const KTile<NP> &a, int n_tiles, int &u, UnitInfo &ui, int &q) {
+    if (u >= n_tiles * kSlicesQ) return false;
+    const int tile = u / kSlicesQ;
+    q = u - tile * kSlicesQ;
+    ui = unit_info(a, tile, 0, 0, 1);
+    u += gridDim.x;
+    return true;
+}
+
+template <int NP, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ KTile<NP> a) {
+    using Sm = typename SmemOf<MODE>::type;
+    constexpr int kBuf = Sm::kBufN;
+    constexpr int kSt = Sm::kStageN;
     extern __shared__ unsigned char smem_raw[];
-    TileSmem &sm = *reinterpret_cast<TileSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    Sm &sm = *reinterpret_cast<Sm *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     // Fetch this launch's parameters and tensor maps while the previous
     // kernel drains.
     const int nproj = NP == 1 ? 1 : a.nproj;
-    if (threadIdx.x == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.X)) : "memory");
+    if (threadIdx.x == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.X)) : "memory");
+        if (MODE == kExpandV) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.V)) : "memory");
+    }
     if (threadIdx.x >= 32 && threadIdx.x < 32 + 3 * nproj) {
         const int i = threadIdx.x - 32, q = i / 3;
         const CUtensorMap *m = (i % 3 == 0) ? &maps.A[q] : (i % 3 == 1) ? &maps.B[q] : &maps.Y[q];
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
     }
     asm volatile("" ::"l"(a.X), "r"(a.T), "r"(a.d_in), "l"(a.tiles), "l"(a.hdr), "l"(a.err));
-    // The kernels before this one on the stream produce the plan.  A batch
-    // without long runs has no tiles: leave before touching tensor memory.
+    // The kernels before this one on the stream produce the plan (and, for
+    // kExpandV, v).  A batch without long runs has no tiles: leave before
+    // touching tensor memory.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int n_tiles = a.hdr->n_tiles;
     if (n_tiles <= 0) return;   // uniform over the grid
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], 1); }
+        for (int s = 0; s < kSt; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], 1); }
         for (int b = 0; b < kBuf; ++b) {
             mbar_init(&sm.bfull[b], 1); mbar_init(&sm.bempty[b], 1);
             mbar_init(&sm.yfull[b], 1); mbar_init(&sm.yempty[b], 1);
@@ -325,6 +384,7 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
         mbar_init(&sm.shrink_done, 1);
         mbar_init(&sm.d1_empty, 128);
         mbar_init(&sm.v_ready, 128);
+        mbar_init(&sm.v_full, 1);
         mbar_init(&sm.v_empty, 1);
         mbar_init(&sm.mma_drain, 1);
         sm.abort = 0;
@@ -332,7 +392,7 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
     }
     if (warp == 2) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&sm.tmem_base)),
-                     "r"(kTmemCols));
+                     "r"(tmem_cols<MODE>()));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     tc_fence_before();
@@ -342,108 +402,170 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
 
     const int nj = a.jpre[nproj];     // items per tile over all projections
     const int nkb = (a.d_in + kKB - 1) / kKB;
+    int nq = 0;                       // quarters of d_in that hold K blocks
+    for (int q = 0; q < kSlicesQ; ++q) {
+        int kb0, kb1;
+        quarter_blocks(nkb, q, kb0, kb1);
+        nq += kb1 > kb0;
+    }
 
     if (warp == 0 && lane == 0) {
         // ---------------- shrink operand producer ----------------
         int it = 0;
-        UnitIter ur = unit_range(n_tiles, nj);
-        UnitInfo ui;
-        while (next_unit(a, ur, ui) && !aborted(sm)) {
-            if (ui.bad && a.err) atomicOr(a.err, LORA_DEV_ERR_BAD_PAGE);
-            if (ui.skip) continue;
+        auto load_kblocks = [&](const UnitInfo &ui, int kb0, int kb1) {
             int pg[4];
             const int32_t *pt = a.proj[ui.p].pt;
             for (int p = 0; p < 4; ++p) pg[p] = p < ui.np ? pt[ui.slot * 8 + p] : 0;
             const CUtensorMap *tmA = &maps.A[ui.p];
-            for (int kb = 0; kb < nkb; ++kb, ++it) {
-                const int s = it % kStages;
-                if (!mbar_wait(&sm.empty[s], ((it / kStages) & 1) ^ 1, sm, a.err)) break;
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                const int s = it % kSt;
+                if (!mbar_wait(&sm.empty[s], ((it / kSt) & 1) ^ 1, sm, a.err)) return false;
                 mbar_expect_tx(&sm.full[s], (uint32_t)(kM * kKB * 2 + ui.np * 16 * kKB * 2));
                 tma_load(sm.xs[s], &maps.X, kb * kKB, ui.row0, &sm.full[s]);
                 for (int p = 0; p < ui.np; ++p)
                     tma_load(&sm.as[s][p * 16 * kKB], tmA, kb * kKB, pg[p] * LORA_PAGE_ROWS, &sm.full[s]);
             }
-        }
-        // the loads this thread armed last on each stage have landed before exit
-        for (int i = (it > kStages ? it - kStages : 0); i < it; ++i) drain_wait(&sm.full[i % kStages], (i / kStages) & 1);
-    } else if (warp == 1 && lane == 0) {
-        // ---------------- expand operand producer ----------------
-        int it = 0;
-        UnitIter ur = unit_range(n_tiles, nj);
-        UnitInfo ui;
-        while (next_unit(a, ur, ui) && !aborted(sm)) {
-            if (ui.skip) continue;
-            int pg[4];
-            const int32_t *pt = a.proj[ui.p].pt;
-            for (int p = 0; p < 4; ++p) pg[p] = p < ui.np ? pt[ui.slot * 8 + 4 + p] : 0;
-            const CUtensorMap *tmB = &maps.B[ui.p], *tmY = &maps.Y[ui.p];
-            for (int j = ui.j0; j < ui.j1; ++j, ++it) {
-                const int b = it % kBuf;
-                const uint32_t par = ((it / kBuf) & 1) ^ 1;
-                if (!mbar_wait(&sm.bempty[b], par, sm, a.err)) break;
-                if (!mbar_wait(&sm.yempty[b], par, sm, a.err)) break;
-                mbar_expect_tx(&sm.bfull[b], (uint32_t)(ui.np * 16 * kNB * 2));
-                for (int p = 0; p < ui.np; ++p)
-                    tma_load(&sm.bs[b][p * 16 * kNB], tmB, j * kNB, pg[p] * LORA_PAGE_ROWS, &sm.bfull[b]);
-                mbar_expect_tx(&sm.yfull[b], (uint32_t)(kM * kNB * 4));
-                tma_load(&sm.ys[b][0], tmY, j * kNB, ui.row0, &sm.yfull[b]);
-                tma_load(&sm.ys[b][kM * 32], tmY, j * kNB + 32, ui.row0, &sm.yfull[b]);
+            return true;
+        };
+        if constexpr (MODE == kFused) {
+            UnitIter ur = unit_range(n_tiles, nj);
+            UnitInfo ui;
+            while (next_unit(a, ur, ui) && !aborted(sm)) {
+                if (ui.bad && a.err) atomicOr(a.err, LORA_DEV_ERR_BAD_PAGE);
+                if (ui.skip) continue;
+                if (!load_kblocks(ui, 0, nkb)) break;
+            }
+        } else if constexpr (MODE == kShrinkQ) {
+            int u = blockIdx.x, q = 0, kb0, kb1;
+            UnitInfo ui;
+            while (next_qunit(a, n_tiles, u, ui, q) && !aborted(sm)) {
+                if (ui.bad && q == 0 && a.err) atomicOr(a.err, LORA_DEV_ERR_BAD_PAGE);
+                quarter_blocks(nkb, q, kb0, kb1);
+                if (ui.skip || kb1 <= kb0) continue;
+                if (!load_kblocks(ui, kb0, kb1)) break;
             }
         }
-        for (int i = (it > kBuf ? it - kBuf : 0); i < it; ++i) {
-            drain_wait(&sm.bfull[i % kBuf], (i / kBuf) & 1);
-            drain_wait(&sm.yfull[i % kBuf], (i / kBuf) & 1);
+        // the loads this thread armed last on each stage have landed before exit
+        for (int i = (it > kSt ? it - kSt : 0); i < it; ++i) drain_wait(&sm.full[i % kSt], (i / kSt) & 1);
+    } else if (warp == 1 && lane == 0) {
+        // ---------------- expand operand producer: v (kExpandV), B and Y ----------------
+        if constexpr (MODE != kShrinkQ) {
+            int it = 0, itv = 0;
+            UnitIter ur = unit_range(n_tiles, nj);
+            UnitInfo ui;
+            while (next_unit(a, ur, ui) && !aborted(sm)) {
+                if constexpr (MODE == kExpandV)
+                    if (ui.bad && a.err) atomicOr(a.err, LORA_DEV_ERR_BAD_PAGE);
+                if (ui.skip) continue;
+                if constexpr (MODE == kExpandV) {
+                    // the unit's v, high and low part, straight into the MMA's operand tiles
+                    if (!mbar_wait(&sm.v_empty, (itv & 1) ^ 1, sm, a.err)) break;
+                    mbar_expect_tx(&sm.v_full, (uint32_t)(2 * kM * 64 * 2));
+                    tma_load(sm.vs, &maps.V, 0, ui.row0, &sm.v_full);
+                    tma_load(sm.vl, &maps.V, 64, ui.row0, &sm.v_full);
+                    ++itv;
+                }
+                int pg[4];
+                const int32_t *pt = a.proj[ui.p].pt;
+                for (int p = 0; p < 4; ++p) pg[p] = p < ui.np ? pt[ui.slot * 8 + 4 + p] : 0;
+                const CUtensorMap *tmB = &maps.B[ui.p], *tmY = &maps.Y[ui.p];
+                for (int j = ui.j0; j < ui.j1; ++j, ++it) {
+                    const int b = it % kBuf;
+                    const uint32_t par = ((it / kBuf) & 1) ^ 1;
+                    if (!mbar_wait(&sm.bempty[b], par, sm, a.err)) break;
+                    mbar_expect_tx(&sm.bfull[b], (uint32_t)(ui.np * 16 * kNB * 2));
+                    for (int p = 0; p < ui.np; ++p)
+                        tma_load(&sm.bs[b][p * 16 * kNB], tmB, j * kNB, pg[p] * LORA_PAGE_ROWS, &sm.bfull[b]);
+                    if (!mbar_wait(&sm.yempty[b], par, sm, a.err)) break;
+                    mbar_expect_tx(&sm.yfull[b], (uint32_t)(kM * kNB * 4));
+                    tma_load(&sm.ys[b][0], tmY, j * kNB, ui.row0, &sm.yfull[b]);
+                    tma_load(&sm.ys[b][kM * 32], tmY, j * kNB + 32, ui.row0, &sm.yfull[b]);
+                }
+            }
+            for (int i = (it > kBuf ? it - kBuf : 0); i < it; ++i) {
+                drain_wait(&sm.bfull[i % kBuf], (i / kBuf) & 1);
+                drain_wait(&sm.yfull[i % kBuf], (i / kBuf) & 1);
+            }
+            if (itv > 0) drain_wait(&sm.v_full, (itv - 1) & 1);
         }
     } else if (warp == 2 && lane == 0) {
         // ---------------- MMA issuer ----------------
         int it = 0, ite = 0, itt = 0;
         bool issued = false;
         const uint32_t idesc2 = idesc_bf16(kM, kNB, 0, 1);
-        UnitIter ur = unit_range(n_tiles, nj);
-        UnitInfo ui;
-        while (next_unit(a, ur, ui) && !aborted(sm)) {
-            if (ui.skip) continue;
+        // shrink: for each quarter q in [q0, q1), D1_q = X A over its K blocks,
+        // into columns 64 q (spread) or 0
+        auto shrink = [&](const UnitInfo &ui, int q0, int q1, bool spread) {
             const uint32_t idesc1 = idesc_bf16(kM, ui.n1, 0, 0);
-            // shrink: D1 = X A over all K blocks
-            if (!mbar_wait(&sm.d1_empty, (itt & 1) ^ 1, sm, a.err)) break;
+            if (!mbar_wait(&sm.d1_empty, (itt & 1) ^ 1, sm, a.err)) return false;
             tc_fence_after();
-            for (int kb = 0; kb < nkb; ++kb, ++it) {
-                const int s = it % kStages;
-                if (!mbar_wait(&sm.full[s], (it / kStages) & 1, sm, a.err)) break;
-                tc_fence_after();
-                issued = true;
-                const uint64_t da = sdesc(sm.xs[s], 16, 1024);
-                const uint64_t db = sdesc(sm.as[s], 16, 1024);
+            for (int q = q0; q < q1; ++q) {
+                int kb0, kb1;
+                quarter_blocks(nkb, q, kb0, kb1);
+                const uint32_t d1 = tmem + (spread ? 64u * (uint32_t)q : 0u);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int s = it % kSt;
+                    if (!mbar_wait(&sm.full[s], (it / kSt) & 1, sm, a.err)) return false;
+                    tc_fence_after();
+                    issued = true;
+                    const uint64_t da = sdesc(sm.xs[s], 16, 1024);
+                    const uint64_t db = sdesc(sm.as[s], 16, 1024);
 #pragma unroll
-                for (int k = 0; k < kKB / 16; ++k)
-                    mma_bf16(tmem, da + (uint64_t)(k * 2), db + (uint64_t)(k * 2), idesc1, (kb | k) != 0);
-                mma_commit(&sm.empty[s]);
+                    for (int k = 0; k < kKB / 16; ++k)
+                        mma_bf16(d1, da + (uint64_t)(k * 2), db + (uint64_t)(k * 2), idesc1, (kb != kb0) || (k != 0));
+                    mma_commit(&sm.empty[s]);
+                }
             }
-            if (aborted(sm)) break;
+            if (aborted(sm)) return false;
             mma_commit(&sm.shrink_done);
-            // expand: one 64-column n-tile at a time into a buffered accumulator
-            if (!mbar_wait(&sm.v_ready, itt & 1, sm, a.err)) break;
+            return true;
+        };
+        // expand: one 64-column n-tile at a time into a buffered accumulator
+        auto expand = [&](const UnitInfo &ui) {
+            if (!mbar_wait(MODE == kExpandV ? &sm.v_full : &sm.v_ready, itt & 1, sm, a.err)) return false;
             tc_fence_after();
             const uint64_t dv = sdesc(sm.vs, 16, 1024);
             const uint64_t dvl = sdesc(sm.vl, 16, 1024);
             for (int j = ui.j0; j < ui.j1; ++j, ++ite) {
                 const int b = ite % kBuf;
                 const uint32_t par = (ite / kBuf) & 1;
-                if (!mbar_wait(&sm.accempty[b], par ^ 1, sm, a.err)) break;
-                if (!mbar_wait(&sm.bfull[b], par, sm, a.err)) break;
+                if (!mbar_wait(&sm.accempty[b], par ^ 1, sm, a.err)) return false;
+                if (!mbar_wait(&sm.bfull[b], par, sm, a.err)) return false;
                 tc_fence_after();
+                issued = true;
                 const uint64_t dbb = sdesc(sm.bs[b], (uint32_t)(ui.n1 * 128), 1024);
                 for (int k = 0; k < ui.np; ++k)
-                    mma_bf16(tmem + 64 + 64 * b, dv + (uint64_t)(k * 2), dbb + (uint64_t)(k * (2048 >> 4)), idesc2,
-                             k != 0);
+                    mma_bf16(tmem + kAccCol + 64 * b, dv + (uint64_t)(k * 2), dbb + (uint64_t)(k * (2048 >> 4)),
+                             idesc2, k != 0);
                 for (int k = 0; k < ui.np; ++k)
-                    mma_bf16(tmem + 64 + 64 * b, dvl + (uint64_t)(k * 2), dbb + (uint64_t)(k * (2048 >> 4)), idesc2, 1);
+                    mma_bf16(tmem + kAccCol + 64 * b, dvl + (uint64_t)(k * 2), dbb + (uint64_t)(k * (2048 >> 4)),
+                             idesc2, 1);
                 mma_commit(&sm.bempty[b]);
                 mma_commit(&sm.accfull[b]);
             }
-            if (aborted(sm)) break;
+            if (aborted(sm)) return false;
             mma_commit(&sm.v_empty);
-            ++itt;
+            return true;
+        };
+        if constexpr (MODE == kShrinkQ) {
+            int u = blockIdx.x, q = 0, kb0, kb1;
+            UnitInfo ui;
+            while (next_qunit(a, n_tiles, u, ui, q) && !aborted(sm)) {
+                quarter_blocks(nkb, q, kb0, kb1);
+                if (ui.skip || kb1 <= kb0) continue;
+                if (!shrink(ui, q, q + 1, false)) break;
+                ++itt;
+            }
+        } else {
+            UnitIter ur = unit_range(n_tiles, nj);
+            UnitInfo ui;
+            while (next_unit(a, ur, ui) && !aborted(sm)) {
+                if (ui.skip) continue;
+                if constexpr (MODE == kFused)
+                    if (!shrink(ui, 0, kSlicesQ, true)) break;
+                if (!expand(ui)) break;
+                ++itt;
+            }
         }
         // every MMA this thread issued has completed before tensor memory is freed
         if (issued) {
@@ -456,117 +578,196 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
         const int m = q * 32 + lane;         // tile row = accumulator lane
         const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
         const bool leader = (warp == 4 && lane == 0);
-        int pending = -1;   // buffer whose TMA store may still be reading it
         int ite = 0, itt = 0;
-        UnitIter ur = unit_range(n_tiles, nj);
-        UnitInfo ui;
-        while (next_unit(a, ur, ui)) {
-            if (!epi_all(!aborted(sm))) break;   // same decision in all 128 epilogue threads
-            if (ui.skip) continue;
-            const KTileProj &pr = a.proj[ui.p];
-            const float sc = pr.scales[ui.slot];
-            // v = D1 row m, rounded to bf16 into the swizzled V tile
-            if (!epi_all(mbar_wait(&sm.shrink_done, itt & 1, sm, a.err))) break;
-            tc_fence_after();
-            float d1[64];
+        // v (fp32, row m) -> bf16 high part and low part (v - high), the two
+        // 16-significant-bit halves the expand multiplies by B
+        auto split_v = [&](const float (&v)[64], int np, uint32_t (&hw)[32], uint32_t (&lw)[32]) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-                if (c < ui.np) TMEM_LD16(trow + c * 16, (&d1[c * 16]));
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&sm.d1_empty);
-            if (!epi_all(mbar_wait(&sm.v_empty, (itt & 1) ^ 1, sm, a.err))) break;
-            // v enters the expand as a bf16 high part and a bf16 low part
-            // (v - high), so the product keeps about 16 significant bits of v
-            unsigned char *vrow = reinterpret_cast<unsigned char *>(sm.vs) + m * 128;
-            unsigned char *lrow = reinterpret_cast<unsigned char *>(sm.vl) + m * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                if (c < ui.np * 2) {
-                    uint32_t hw[4], lw[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float f0 = d1[c * 8 + 2 * e], f1 = d1[c * 8 + 2 * e + 1];
-                        const __nv_bfloat162 h = __floats2bfloat162_rn(f0, f1);
-                        const __nv_bfloat162 l = __floats2bfloat162_rn(f0 - __low2float(h), f1 - __high2float(h));
-                        hw[e] = *reinterpret_cast<const uint32_t *>(&h);
-                        lw[e] = *reinterpret_cast<const uint32_t *>(&l);
-                    }
-                    *reinterpret_cast<uint4 *>(vrow + ((c ^ (m & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                    *reinterpret_cast<uint4 *>(lrow + ((c ^ (m & 7)) << 4)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            for (int e = 0; e < 32; ++e) {
+                if (e < np * 8) {
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+                    const __nv_bfloat162 l = __floats2bfloat162_rn(v[2 * e] - __low2float(h), v[2 * e + 1] - __high2float(h));
+                    hw[e] = *reinterpret_cast<const uint32_t *>(&h);
+                    lw[e] = *reinterpret_cast<const uint32_t *>(&l);
                 }
             }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_arrive(&sm.v_ready);
-            // n-tiles
-            for (int j = ui.j0; j < ui.j1; ++j, ++ite) {
-                const int b = ite % kBuf;
-                const uint32_t par = (ite / kBuf) & 1;
-                bool ok = mbar_wait(&sm.accfull[b], par, sm, a.err);
-                ok = mbar_wait(&sm.yfull[b], par, sm, a.err) && ok;
-                if (!epi_all(ok)) break;
+        };
+        if constexpr (MODE == kShrinkQ) {
+            // D1 rows of the tile's tokens -> the quarter's fp32 partials; the
+            // CTA that finishes a tile's last quarter adds the quarters in
+            // order and leaves v (bf16 high, low) in quarter 0's rows
+            int u = blockIdx.x, qq = 0, kb0, kb1;
+            UnitInfo ui;
+            while (next_qunit(a, n_tiles, u, ui, qq)) {
+                if (!epi_all(!aborted(sm))) break;
+                quarter_blocks(nkb, qq, kb0, kb1);
+                if (ui.skip || kb1 <= kb0) continue;
+                if (!epi_all(mbar_wait(&sm.shrink_done, itt & 1, sm, a.err))) break;
                 tc_fence_after();
-                float acc[64];
+                float d1[64];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) TMEM_LD16(trow + 64 + 64 * b + c * 16, (&acc[c * 16]));
+                for (int c = 0; c < 4; ++c)
+                    if (c < ui.np) TMEM_LD16(trow + c * 16, (&d1[c * 16]));
                 tmem_wait_ld();
                 tc_fence_before();
-                mbar_arrive(&sm.accempty[b]);
-                const bool full_tile = ui.ntok == kM;
+                mbar_arrive(&sm.d1_empty);
+                if (m < ui.ntok) {
+                    float4 *dst = reinterpret_cast<float4 *>(a.vpart + ((size_t)qq * a.T + ui.row0 + m) * LORA_MAX_RANK);
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const int h = c >> 3, cc = c & 7;
-                    float4 *yp = reinterpret_cast<float4 *>(reinterpret_cast<unsigned char *>(&sm.ys[b][h * kM * 32]) +
-                                                            m * 128 + ((cc ^ (m & 7)) << 4));
-                    float4 y = *yp;
-                    y.x = fmaf(sc, acc[c * 4 + 0], y.x);
-                    y.y = fmaf(sc, acc[c * 4 + 1], y.y);
-                    y.z = fmaf(sc, acc[c * 4 + 2], y.z);
-                    y.w = fmaf(sc, acc[c * 4 + 3], y.w);
-                    if (full_tile) {
-                        *yp = y;
-                    } else if (m < ui.ntok) {
-                        const int col = j * kNB + c * 4;
-                        if (col < pr.d_out)
-                            *reinterpret_cast<float4 *>(pr.Y + (size_t)(ui.row0 + m) * pr.d_out + col) = y;
-                    }
+                    for (int c = 0; c < 16; ++c)
+                        if (c < ui.np * 4)
+                            dst[c] = make_float4(d1[4 * c], d1[4 * c + 1], d1[4 * c + 2], d1[4 * c + 3]);
                 }
-                if (full_tile) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __threadfence();   // this quarter's rows are visible before it is counted
                 epi_sync();
-                if (leader) {
-                    if (full_tile) {
-                        tma_store(&maps.Y[ui.p], j * kNB, ui.row0, &sm.ys[b][0]);
-                        tma_store(&maps.Y[ui.p], j * kNB + 32, ui.row0, &sm.ys[b][kM * 32]);
-                        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-                        // the previous store has finished reading its buffer once at
-                        // most one group (this one) is still reading
-                        asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-                        if (pending >= 0) mbar_arrive(&sm.yempty[pending]);
-                        pending = b;
-                    } else {
-                        // a buffer whose store is still pending would otherwise wait for
-                        // the next full tile, which may never come on this CTA
-                        if (pending >= 0) {
-                            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-                            mbar_arrive(&sm.yempty[pending]);
-                            pending = -1;
+                if (leader) sm.reduce = atomicAdd(&a.tiles[ui.tile].w, 1) == nq - 1;
+                epi_sync();
+                if (sm.reduce) {
+                    __threadfence();
+                    if (m < ui.ntok) {
+                        float v[64];
+#pragma unroll
+                        for (int c = 0; c < 64; ++c) v[c] = 0.f;
+                        for (int q2 = 0; q2 < kSlicesQ; ++q2) {
+                            int b0, b1;
+                            quarter_blocks(nkb, q2, b0, b1);
+                            if (b1 <= b0) continue;
+                            const float4 *src =
+                                reinterpret_cast<const float4 *>(a.vpart + ((size_t)q2 * a.T + ui.row0 + m) * LORA_MAX_RANK);
+#pragma unroll
+                            for (int c = 0; c < 16; ++c) {
+                                if (c < ui.np * 4) {
+                                    const float4 w = __ldcg(src + c);
+                                    v[4 * c] += w.x;
+                                    v[4 * c + 1] += w.y;
+                                    v[4 * c + 2] += w.z;
+                                    v[4 * c + 3] += w.w;
+                                }
+                            }
                         }
-                        mbar_arrive(&sm.yempty[b]);
+                        uint32_t hw[32], lw[32];
+                        split_v(v, ui.np, hw, lw);
+                        uint4 *dst = reinterpret_cast<uint4 *>(a.vpart + ((size_t)ui.row0 + m) * LORA_MAX_RANK);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            if (c < ui.np * 2) {
+                                dst[c] = make_uint4(hw[4 * c], hw[4 * c + 1], hw[4 * c + 2], hw[4 * c + 3]);
+                                dst[8 + c] = make_uint4(lw[4 * c], lw[4 * c + 1], lw[4 * c + 2], lw[4 * c + 3]);
+                            }
+                        }
                     }
+                    if (leader) a.tiles[ui.tile].w = 0;   // ready for the next launch over this plan
                 }
+                ++itt;
             }
-            ++itt;
-        }
-        if (leader) {
-            asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-            if (pending >= 0) mbar_arrive(&sm.yempty[pending]);
+        } else {
+            UnitIter ur = unit_range(n_tiles, nj);
+            UnitInfo ui;
+            while (next_unit(a, ur, ui)) {
+                if (!epi_all(!aborted(sm))) break;   // same decision in all 128 epilogue threads
+                if (ui.skip) continue;
+                const KTileProj &pr = a.proj[ui.p];
+                const float sc = pr.scales[ui.slot];
+                if constexpr (MODE == kFused) {
+                    // v = row m of the quarters' D1 added in quarter order: the
+                    // same fp32 sums, and the same bf16 parts, as the two-launch form
+                    if (!epi_all(mbar_wait(&sm.shrink_done, itt & 1, sm, a.err))) break;
+                    tc_fence_after();
+                    float d1[64];
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) d1[c] = 0.f;
+                    for (int qq = 0; qq < kSlicesQ; ++qq) {
+                        int kb0, kb1;
+                        quarter_blocks(nkb, qq, kb0, kb1);
+                        if (kb1 <= kb0) continue;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            if (c < ui.np) {
+                                float t16[16];
+                                TMEM_LD16(trow + 64 * qq + c * 16, t16);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) d1[c * 16 + i] += t16[i];
+                            }
+                        }
+                    }
+                    tc_fence_before();
+                    mbar_arrive(&sm.d1_empty);
+                    uint32_t hw[32], lw[32];
+                    split_v(d1, ui.np, hw, lw);
+                    if (!epi_all(mbar_wait(&sm.v_empty, (itt & 1) ^ 1, sm, a.err))) break;
+                    unsigned char *vrow = reinterpret_cast<unsigned char *>(sm.vs) + m * 128;
+                    unsigned char *lrow = reinterpret_cast<unsigned char *>(sm.vl) + m * 128;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        if (c < ui.np * 2) {
+                            *reinterpret_cast<uint4 *>(vrow + ((c ^ (m & 7)) << 4)) =
+                                make_uint4(hw[4 * c], hw[4 * c + 1], hw[4 * c + 2], hw[4 * c + 3]);
+                            *reinterpret_cast<uint4 *>(lrow + ((c ^ (m & 7)) << 4)) =
+                                make_uint4(lw[4 * c], lw[4 * c + 1], lw[4 * c + 2], lw[4 * c + 3]);
+                        }
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    mbar_arrive(&sm.v_ready);
+                }
+                // n-tiles: y = s * D2 + y on the Y tile in shared memory (row m
+                // per thread), then the rows of the unit's tokens go back with
+                // coalesced stores from all 128 threads
+                for (int j = ui.j0; j < ui.j1; ++j, ++ite) {
+                    const int b = ite % kBuf;
+                    const uint32_t par = (ite / kBuf) & 1;
+                    bool ok = mbar_wait(&sm.accfull[b], par, sm, a.err);
+                    ok = mbar_wait(&sm.yfull[b], par, sm, a.err) && ok;
+                    if (!epi_all(ok)) break;
+                    tc_fence_after();
+                    float acc[64];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) TMEM_LD16(trow + kAccCol + 64 * b + c * 16, (&acc[c * 16]));
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    mbar_arrive(&sm.accempty[b]);
+                    unsigned char *yt = reinterpret_cast<unsigned char *>(&sm.ys[b][0]);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const int h = c >> 3, cc = c & 7;
+                        float4 *yp = reinterpret_cast<float4 *>(yt + h * kM * 128 + m * 128 + ((cc ^ (m & 7)) << 4));
+                        float4 y = *yp;
+                        y.x = fmaf(sc, acc[c * 4 + 0], y.x);
+                        y.y = fmaf(sc, acc[c * 4 + 1], y.y);
+                        y.z = fmaf(sc, acc[c * 4 + 2], y.z);
+                        y.w = fmaf(sc, acc[c * 4 + 3], y.w);
+                        *yp = y;
+                    }
+                    epi_sync();
+                    // 16 threads per row, one 16-byte group each: row r, group g
+                    const int tid = threadIdx.x - 128;
+#pragma unroll 4
+                    for (int i = 0; i < 16; ++i) {
+                        const int idx = tid + 128 * i, r = idx >> 4, g = idx & 15;
+                        const int col = j * kNB + 4 * g;
+                        if (r < ui.ntok && col < pr.d_out) {
+                            const int h = g >> 3, cc = g & 7;
+                            const float4 y =
+                                *reinterpret_cast<const float4 *>(yt + h * kM * 128 + r * 128 + ((cc ^ (r & 7)) << 4));
+                            *reinterpret_cast<float4 *>(pr.Y + (size_t)(ui.row0 + r) * pr.d_out + col) = y;
+                        }
+                    }
+                    // the tile was read and written through the generic proxy; order
+                    // that before the producer's next TMA load into it
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    epi_sync();
+                    if (leader) mbar_arrive(&sm.yempty[b]);
+                }
+                ++itt;
+            }
         }
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 2) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+    if (warp == 2)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tmem_cols<MODE>()));
 }
 
 // ---------------------------------------------------------------------------
@@ -578,16 +779,23 @@ bool tiles_supported() { return tma_supported(); }
 
 namespace {
 
-template <int NP>
+template <int NP, int MODE>
 int launch_np(const TileArgs &a, cudaStream_t st, bool pdl, int sms) {
-    const size_t smem = sizeof(TileSmem) + 1024;
+    const size_t smem = sizeof(typename SmemOf<MODE>::type) + 1024;
     TileMaps<NP> maps;
     KTile<NP> k;
     k.X = a.X; k.T = a.T; k.d_in = a.d_in; k.nproj = a.nproj;
-    k.tiles = a.tiles; k.hdr = a.hdr; k.err = a.err;
+    k.tiles = const_cast<int4 *>(a.tiles); k.hdr = a.hdr; k.err = a.err; k.vpart = a.vpart;
     if (int rc = make_tensor_map(&maps.X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.X, (uint64_t)a.d_in, (uint64_t)a.T,
                                  kKB, kM, true))
         return rc;
+    maps.V = maps.X;
+    if (MODE == kExpandV) {
+        // quarter 0 of the partials, row t = 256 bytes = v high [64] | v low [64] in bf16
+        if (int rc = make_tensor_map(&maps.V, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.vpart, 2 * LORA_MAX_RANK,
+                                     (uint64_t)a.T, 64, kM, true))
+            return rc;
+    }
     k.jpre[0] = 0;
     for (int p = 0; p < NP; ++p) {
         const TileProj &q = a.proj[p < a.nproj ? p : 0];
@@ -602,10 +810,11 @@ int launch_np(const TileArgs &a, cudaStream_t st, bool pdl, int sms) {
         if (int rc = pool_tensor_map(const_cast<lora_pool_s *>(q.pb), &maps.B[p])) return rc;
         k.jpre[p + 1] = k.jpre[p] + (p < a.nproj ? (q.d_out + kNB - 1) / kNB : 0);
     }
-    // one CTA per SM (never more than there can be items)
+    // one CTA per SM (never more than there can be units)
     const long long max_tiles = (a.T + kM - 1) / kM + (a.long_thresh > 0 ? a.T / a.long_thresh : 0);
     long long grid = sms;
-    if (grid > max_tiles * k.jpre[NP]) grid = max_tiles * k.jpre[NP];
+    const long long units = MODE == kShrinkQ ? max_tiles * kSlicesQ : max_tiles * k.jpre[NP];
+    if (grid > units) grid = units;
     if (grid < 1) grid = 1;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
@@ -617,9 +826,15 @@ int launch_np(const TileArgs &a, cudaStream_t st, bool pdl, int sms) {
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    if (int rc = cuda_check(cudaLaunchKernelEx(&cfg, tiles_kernel<NP>, maps, k))) return rc;
+    if (int rc = cuda_check(cudaLaunchKernelEx(&cfg, tiles_kernel<NP, MODE>, maps, k))) return rc;
     count_launch();
     return LORA_OK;
+}
+
+template <int NP, int MODE>
+int set_smem_attr() {
+    return cuda_check(cudaFuncSetAttribute(tiles_kernel<NP, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)(sizeof(typename SmemOf<MODE>::type) + 1024)));
 }
 
 }  // namespace
@@ -630,20 +845,22 @@ int launch_tiles(const TileArgs &a, cudaStream_t st, bool pdl) {
     if (a.nproj < 1 || a.nproj > LORA_MAX_PROJECTIONS) return LORA_ERR_INVALID_ARG;
     if (int rc = cuda_check(cudaGetDevice(&dev))) return rc;
     if (dev < 0 || dev >= 64) return LORA_ERR_INVALID_ARG;
-    const size_t smem = sizeof(TileSmem) + 1024;
     if (num_sms[dev] == 0) {
-        if (int rc = cuda_check(cudaFuncSetAttribute(tiles_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                     (int)smem)))
-            return rc;
-        if (int rc = cuda_check(cudaFuncSetAttribute(tiles_kernel<LORA_MAX_PROJECTIONS>,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
-            return rc;
+        if (int rc = set_smem_attr<1, kFused>()) return rc;
+        if (int rc = set_smem_attr<LORA_MAX_PROJECTIONS, kFused>()) return rc;
+        if (int rc = set_smem_attr<1, kShrinkQ>()) return rc;
+        if (int rc = set_smem_attr<1, kExpandV>()) return rc;
         int n = 0;
         if (int rc = cuda_check(cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev))) return rc;
         num_sms[dev] = n > 0 ? n : 1;
     }
-    return a.nproj == 1 ? launch_np<1>(a, st, pdl, num_sms[dev])
-                        : launch_np<LORA_MAX_PROJECTIONS>(a, st, pdl, num_sms[dev]);
+    const int sms = num_sms[dev];
+    if (a.nproj == 1 && a.vpart) {
+        if (int rc = launch_np<1, kShrinkQ>(a, st, pdl, sms)) return rc;
+        return launch_np<1, kExpandV>(a, st, true, sms);
+    }
+    return a.nproj == 1 ? launch_np<1, kFused>(a, st, pdl, sms)
+                        : launch_np<LORA_MAX_PROJECTIONS, kFused>(a, st, pdl, sms);
 }
 
 }  // namespace lora
