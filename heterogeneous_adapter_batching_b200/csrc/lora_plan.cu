@@ -117,7 +117,7 @@ __device__ __forceinline__ bool is_break(const int32_t *ids, int t, int id, bool
 
 // Dynamic shared memory of the kernel (ints).
 __host__ __device__ constexpr size_t plan_smem_ints(int T, int S, int W, bool in_smem) {
-    return (size_t)S * W + (size_t)S + (in_smem ? (size_t)5 * T + 2 * (size_t)S + 1 : 0);
+    return (((size_t)S * W + 3) & ~(size_t)3) + (size_t)S + (in_smem ? (size_t)5 * T + 2 * (size_t)S + 1 : 0);
 }
 
 template <bool SMEM>
@@ -129,8 +129,8 @@ plan_kernel(const int32_t *__restrict__ ids_g, int T, const int32_t *__restrict_
     asm volatile("griddepcontrol.launch_dependents;");
 
     extern __shared__ int smem[];
-    int *cnt = smem;                       // [S][W] per-warp counts, then scan offsets
-    int *scnt = cnt + (size_t)S * W;       // [S] short tokens per slot
+    int *cnt = smem;                       // [S][W] per-warp counts, then scan offsets (padded to 4 entries)
+    int *scnt = cnt + (((size_t)S * W + 3) & ~(size_t)3);   // [S] short tokens per slot
     int *ids_s = scnt + S;                 // SMEM only: [T] ids, [S] ranks, [T] perm, [T] perm_short,
     int *ranks_s = ids_s + T;              //   [T] run starts, [T] run ends, [S + 1] seg_start
     int *perm_s = ranks_s + S;
@@ -158,7 +158,7 @@ plan_kernel(const int32_t *__restrict__ ids_g, int T, const int32_t *__restrict_
         for (int t = tid; t < T; t += nthr) ids_s[t] = ids_g[t];
         for (int k = tid; k < S; k += nthr) ranks_s[k] = ranks_g[k];
     }
-    for (int e = tid; e < n_entries; e += nthr) cnt[e] = 0;
+    for (int e = tid; e < ((n_entries + 3) & ~3); e += nthr) cnt[e] = 0;
     for (int k = tid; k < S; k += nthr) scnt[k] = 0;
     __syncthreads();
 
@@ -202,12 +202,27 @@ plan_kernel(const int32_t *__restrict__ ids_g, int T, const int32_t *__restrict_
 
     // Phase 2: exclusive scan of cnt in slot-major order; carries of the run scans.
     {
-        const int per = (n_entries + nthr - 1) / nthr;
-        const int e0 = tid * per, e1 = min(n_entries, e0 + per);
+        // each thread a contiguous run of 4-entry groups (the table is padded
+        // to a multiple of 4 entries with zeros)
+        const int n4 = (n_entries + 3) >> 2;
+        const int per = (n4 + nthr - 1) / nthr;
+        const int g0 = tid * per, g1 = min(n4, g0 + per);
+        int4 *cnt4 = reinterpret_cast<int4 *>(cnt);
         int local = 0;
-        for (int e = e0; e < e1; ++e) local += cnt[e];
+        for (int g = g0; g < g1; ++g) {
+            const int4 c = cnt4[g];
+            local += c.x + c.y + c.z + c.w;
+        }
         int run = block_exclusive_scan(local, wsum, &s_total[0]);
-        for (int e = e0; e < e1; ++e) { int c = cnt[e]; cnt[e] = run; run += c; }
+        for (int g = g0; g < g1; ++g) {
+            const int4 c = cnt4[g];
+            int4 o;
+            o.x = run; run += c.x;
+            o.y = run; run += c.y;
+            o.z = run; run += c.z;
+            o.w = run; run += c.w;
+            cnt4[g] = o;
+        }
         if (tid < W) {
             int cl = -1, cr = T;
             for (int w = 0; w < tid; ++w) cl = max(cl, wlast[w]);
@@ -442,7 +457,10 @@ int launch_plan(const int32_t *ids, int T, const int32_t *ranks, int S, int long
                 const PlanOut &out, int32_t *err_dev, cudaStream_t st, int units_per_job) {
     const bool in_smem = T <= kSmemTokens;
     const int threads = T <= 1024 ? 256 : (in_smem ? 512 : kPlanMaxThreads);
+    // warps that own tokens: no more than there are 32-token groups (the
+    // [slot][warp] table and its scan shrink with them)
     int W = threads / 32;
+    if (W > (T + 31) / 32) W = (T + 31) / 32 > 0 ? (T + 31) / 32 : 1;
     while (W > 1 && W * S > kTableEntries) W >>= 1;
     const size_t smem = sizeof(int) * plan_smem_ints(T, S, W, in_smem);
     static bool attr_set[64] = {};
