@@ -34,6 +34,8 @@ OPT_LONG_SEGMENT = 1
 OPT_DECODE_JOB_TOKENS = 2
 OPT_GATHER_PATH = 3
 GATHER_AUTO, GATHER_CLUSTER, GATHER_SPLIT = 0, 1, 2
+OPT_PLAN_KERNEL = 4
+PLAN_AUTO, PLAN_GENERAL = 0, 1
 NOALLOC_MAX_TOKENS = 32768
 NOALLOC_SCRATCH_BYTES = 2162688
 MAX_JOB_TOKENS = 16

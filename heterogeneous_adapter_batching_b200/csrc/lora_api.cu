@@ -12,6 +12,7 @@ namespace {
 std::atomic<int> g_long_segment{128};
 std::atomic<int> g_job_tokens{LORA_MAX_JOB_TOKENS};
 std::atomic<int> g_gather_path{LORA_GATHER_AUTO};
+std::atomic<int> g_plan_kernel{LORA_PLAN_AUTO};
 thread_local int t_launches = 0;
 thread_local const char *t_last_cuda_error = "no error";
 
@@ -41,6 +42,7 @@ __global__ void read_row_kernel(const uint16_t *pool, int width, const int32_t *
 int opt_long_segment() { return g_long_segment.load(); }
 int opt_job_tokens() { return g_job_tokens.load(); }
 int opt_gather_path() { return g_gather_path.load(); }
+int opt_plan_kernel() { return g_plan_kernel.load(); }
 
 int cuda_check(cudaError_t e) {
     if (e == cudaSuccess) return LORA_OK;
@@ -542,6 +544,10 @@ int lora_set_option(int key, int value) {
             if (value < LORA_GATHER_AUTO || value > LORA_GATHER_SPLIT) return LORA_ERR_INVALID_ARG;
             g_gather_path.store(value);
             return LORA_OK;
+        case LORA_OPT_PLAN_KERNEL:
+            if (value < LORA_PLAN_AUTO || value > LORA_PLAN_GENERAL) return LORA_ERR_INVALID_ARG;
+            g_plan_kernel.store(value);
+            return LORA_OK;
     }
     return LORA_ERR_INVALID_ARG;
 }
@@ -551,6 +557,7 @@ int lora_get_option(int key) {
         case LORA_OPT_LONG_SEGMENT: return g_long_segment.load();
         case LORA_OPT_DECODE_JOB_TOKENS: return g_job_tokens.load();
         case LORA_OPT_GATHER_PATH: return g_gather_path.load();
+        case LORA_OPT_PLAN_KERNEL: return g_plan_kernel.load();
     }
     return LORA_ERR_INVALID_ARG;
 }

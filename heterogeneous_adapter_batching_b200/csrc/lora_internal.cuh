@@ -100,6 +100,7 @@ int pool_tensor_map4(lora_pool_s *pool, CUtensorMap *out);
 int opt_long_segment();
 int opt_job_tokens();
 int opt_gather_path();
+int opt_plan_kernel();
 
 // Record a CUDA error and return LORA_ERR_CUDA, or LORA_OK.
 int cuda_check(cudaError_t e);

@@ -451,6 +451,192 @@ plan_kernel(const int32_t *__restrict__ ids_g, int T, const int32_t *__restrict_
     }
 }
 
+// Small batches without long runs (T <= kSmallTokens, S <= kSmallSlots): the
+// same outputs as plan_kernel<true>, bit for bit, from one warp.  The
+// block-wide scans and barriers of the general kernel cost more than the
+// work at these sizes; here every step is a warp scan over shared tables,
+// with two passes over the tokens (counts, then the stable scatter) and two
+// over the slots (offsets and job-size counts, then the jobs).
+constexpr int kSmallTokens = 256;
+constexpr int kSmallSlots = 128;   // with more slots the warp's two slot passes cost more than the block's scans
+
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += y;
+    }
+    return v;
+}
+
+__global__ void __launch_bounds__(32, 1)
+plan_small_kernel(const int32_t *__restrict__ ids_g, int T, const int32_t *__restrict__ ranks_g, int S,
+                  int long_thresh, int job_tokens, int clusters, PlanOut out, int32_t *err_dev) {
+    asm volatile("griddepcontrol.launch_dependents;");
+    __shared__ int ids_s[kSmallTokens];
+    __shared__ int perm_s[kSmallTokens];    // perm (the workspace copy is not written, as in plan_kernel<true>)
+    __shared__ int rk[kSmallSlots];
+    __shared__ int pos[kSmallSlots];      // tokens per slot, then the next output position of each slot
+    __shared__ int seg[kSmallSlots + 1];
+    const int lane = threadIdx.x;
+    const unsigned lt_mask = (1u << lane) - 1u;
+
+    for (int k = lane; k < S; k += 32) {
+        rk[k] = ranks_g[k];
+        pos[k] = 0;
+    }
+    for (int t = lane; t < T; t += 32) ids_s[t] = ids_g[t];
+    __syncwarp();
+
+    // tokens per slot, and the error bits
+    int err = 0;
+    for (int base = 0; base < T; base += 32) {
+        const int t = base + lane;
+        int id = -1;
+        bool ok = false;
+        if (t < T) {
+            id = ids_s[t];
+            if (id < -1 || id >= S) err |= LORA_DEV_ERR_BAD_ID;
+            else if (id >= 0) {
+                if (rk[id] > 0) ok = true;
+                else err |= LORA_DEV_ERR_EMPTY_SLOT;
+            }
+        }
+        const unsigned act = __ballot_sync(0xffffffffu, ok);
+        if (ok) {
+            const unsigned m = __match_any_sync(act, id);
+            if (lane == __ffs(m) - 1) pos[id] += __popc(m);
+        }
+        __syncwarp();
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) err |= __shfl_xor_sync(0xffffffffu, err, o);
+    if (lane == 0 && err && err_dev) atomicOr(err_dev, err);
+
+    // slot offsets; the job counts of the three candidate sizes; the jobs of
+    // each rank class under each candidate
+    const int cand[3] = {min(4, job_tokens), min(8, job_tokens), job_tokens};
+    int run = 0, n_seg = 0;
+    int njc[3] = {0, 0, 0};
+    int ncls[3][kPlanRankClasses] = {};
+    for (int base = 0; base < S; base += 32) {
+        const int k = base + lane;
+        const int c = k < S ? pos[k] : 0;
+        const int inc = warp_incl_scan(c, lane);
+        if (k < S) {
+            const int st = run + inc - c;
+            seg[k] = st;
+            pos[k] = st;
+            out.seg_start[k] = st;
+            if (out.seg_start_copy) out.seg_start_copy[k] = st;
+            if (c > 0) {
+                const int cl = rank_class(rk[k]);
+#pragma unroll
+                for (int i = 0; i < 3; ++i) {
+                    const int nj = (c + cand[i] - 1) / cand[i];
+                    njc[i] += nj;
+#pragma unroll
+                    for (int q = 0; q < kPlanRankClasses; ++q) ncls[i][q] += cl == q ? nj : 0;
+                }
+            }
+        }
+        n_seg += __popc(__ballot_sync(0xffffffffu, k < S && c > 0));
+        run += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    const int n_valid = run;
+    if (lane == 0) {
+        seg[S] = n_valid;
+        out.seg_start[S] = n_valid;
+        if (out.seg_start_copy) out.seg_start_copy[S] = n_valid;
+    }
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) njc[i] += __shfl_xor_sync(0xffffffffu, njc[i], o);
+#pragma unroll
+        for (int q = 0; q < kPlanRankClasses; ++q)
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ncls[i][q] += __shfl_xor_sync(0xffffffffu, ncls[i][q], o);
+    }
+    __syncwarp();
+
+    // stable scatter: perm = perm_short (no long runs)
+    for (int base = 0; base < T; base += 32) {
+        const int t = base + lane;
+        int id = -1;
+        bool ok = false;
+        if (t < T) {
+            id = ids_s[t];
+            ok = valid_id(id, S, rk);
+        }
+        const unsigned act = __ballot_sync(0xffffffffu, ok);
+        unsigned m = 0;
+        if (ok) {
+            m = __match_any_sync(act, id);
+            const int p = pos[id] + __popc(m & lt_mask);
+            perm_s[p] = t;
+            out.perm_short[p] = t;
+            if (out.perm_copy) out.perm_copy[p] = t;
+        }
+        __syncwarp();
+        if (ok && lane == __ffs(m) - 1) pos[id] += __popc(m);
+        __syncwarp();
+    }
+
+    // job size: the largest candidate that still gives min(jobs at the
+    // smallest size, clusters) jobs (the general kernel's rule)
+    const int want = min(njc[0], clusters);
+    int ci = 0;
+#pragma unroll
+    for (int i = 1; i < 3; ++i)
+        if (cand[i] <= job_tokens && njc[i] >= want) ci = i;
+    const int jt = cand[ci];
+    int cls_base[kPlanRankClasses], n_jobs = 0;
+#pragma unroll
+    for (int q = 0; q < kPlanRankClasses; ++q) {
+        cls_base[q] = n_jobs;
+        n_jobs += ncls[ci][q];
+    }
+
+    // jobs: heaviest rank class first, slot order within a class
+    for (int base = 0; base < S; base += 32) {
+        const int k = base + lane;
+        const int c = k < S ? seg[k + 1] - seg[k] : 0;
+        const int cl = (k < S && c > 0) ? rank_class(rk[k]) : 0;
+        const int nj = c > 0 ? (c + jt - 1) / jt : 0;
+        int jo = 0;
+#pragma unroll
+        for (int q = 0; q < kPlanRankClasses; ++q) {
+            const int v = cl == q ? nj : 0;
+            const int inc = warp_incl_scan(v, lane);
+            if (cl == q) jo = cls_base[q] + inc - v;
+            cls_base[q] += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (c > 0) {
+            const int b = c / nj, rem = c % nj;
+            for (int j = 0; j < nj; ++j) {
+                const int cc = b + (j < rem ? 1 : 0);
+                const int q0 = seg[k] + j * b + min(j, rem);
+                int tk[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) tk[i] = i < cc ? perm_s[q0 + i] : -1;
+                out.jobs[2 * (jo + j)] = make_int4(k, cc, q0, 0);
+                out.jobs[2 * (jo + j) + 1] = make_int4(tk[0], tk[1], tk[2], tk[3]);
+            }
+        }
+    }
+    if (lane == 0) {
+        out.header->n_valid = n_valid;
+        out.header->n_seg = n_seg;
+        out.header->n_jobs = n_jobs;
+        out.header->n_tiles = 0;
+        out.header->T = T;
+        out.header->S = S;
+        out.header->job_tokens = jt;
+        out.header->long_thresh = long_thresh;
+    }
+}
+
 }  // namespace
 
 int launch_plan(const int32_t *ids, int T, const int32_t *ranks, int S, int long_thresh, int job_tokens,
@@ -481,6 +667,12 @@ int launch_plan(const int32_t *ids, int T, const int32_t *ranks, int S, int long
     int clusters = 1;
     if (int rc = gather_clusters(&clusters)) return rc;
     clusters = max(1, clusters / max(1, units_per_job));
+    const bool runs = long_thresh > 0 && T >= long_thresh;
+    if (!runs && T <= kSmallTokens && S <= kSmallSlots && opt_plan_kernel() != LORA_PLAN_GENERAL) {
+        plan_small_kernel<<<1, 32, 0, st>>>(ids, T, ranks, S, long_thresh, job_tokens, clusters, out, err_dev);
+        count_launch();
+        return cuda_check(cudaGetLastError());
+    }
     if (in_smem)
         plan_kernel<true><<<1, threads, smem, st>>>(ids, T, ranks, S, W, long_thresh, job_tokens, clusters, out, err_dev);
     else

@@ -394,6 +394,11 @@ int lora_slot_cache_stats(lora_slot_cache_t c, int64_t *hits, int64_t *misses, i
 #define LORA_GATHER_CLUSTER     1   /* one kernel: 4-CTA clusters exchange the shrink partials on chip */
 #define LORA_GATHER_SPLIT       2   /* a shrink kernel writes per-quarter partials to the workspace, an expand
                                         kernel adds them and updates Y; one pair per projection */
+#define LORA_OPT_PLAN_KERNEL    4   /* the plan's kernel: LORA_PLAN_AUTO (default) or LORA_PLAN_GENERAL; both
+                                        write the same plan, bit for bit */
+#define LORA_PLAN_AUTO          0   /* one warp for batches of at most 256 tokens, 128 slots and no long runs,
+                                        the block-wide kernel otherwise */
+#define LORA_PLAN_GENERAL       1   /* always the block-wide kernel */
 
 int lora_set_option(int key, int value);
 int lora_get_option(int key);
