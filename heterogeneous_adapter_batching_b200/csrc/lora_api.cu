@@ -4,6 +4,9 @@
 #include <atomic>
 #include <cstring>
 
+#include <mutex>
+#include <unordered_map>
+
 #include "lora_internal.cuh"
 
 namespace lora {
@@ -43,6 +46,22 @@ int opt_long_segment() { return g_long_segment.load(); }
 int opt_job_tokens() { return g_job_tokens.load(); }
 int opt_gather_path() { return g_gather_path.load(); }
 int opt_plan_kernel() { return g_plan_kernel.load(); }
+
+namespace {
+std::mutex g_last_mu;
+std::unordered_map<cudaStream_t, bool> g_plan_last;   // stream -> its last library launch was the plan
+}  // namespace
+
+bool plan_was_last_launch(cudaStream_t st) {
+    std::lock_guard<std::mutex> g(g_last_mu);
+    const auto it = g_plan_last.find(st);
+    return it != g_plan_last.end() && it->second;
+}
+
+void note_launch(cudaStream_t st, bool is_plan) {
+    std::lock_guard<std::mutex> g(g_last_mu);
+    g_plan_last[st] = is_plan;
+}
 
 int cuda_check(cudaError_t e) {
     if (e == cudaSuccess) return LORA_OK;

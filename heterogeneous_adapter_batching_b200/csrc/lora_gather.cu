@@ -129,6 +129,7 @@ struct KArgs {
     const int4 *jobs;
     const PlanHeader *hdr;
     int32_t *err;
+    int early;           // the plan was complete before this launch started (see plan_was_last_launch)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -328,14 +329,15 @@ __device__ __forceinline__ UnitGeom unit_geom(const Args &a, const GatherSmem &s
     return g;
 }
 
+// Plan data, read through L2 (it may come from a kernel before the one ahead).
 __device__ __forceinline__ int4 ld_v4_now(const int4 *p) {
     int4 v;
-    asm volatile("ld.global.v4.s32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    asm volatile("ld.global.cg.v4.s32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
     return v;
 }
 __device__ __forceinline__ int ld_s32_now(const int *p) {
     int v;
-    asm volatile("ld.global.s32 %0, [%1];" : "=r"(v) : "l"(p));
+    asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p));
     return v;
 }
 
@@ -407,12 +409,18 @@ gather_kernel(const __grid_constant__ GatherMaps<NP> maps, const __grid_constant
             sm.scales[i] = (MODE == kShrink) ? 0.f : pr.scales[k];
         }
     }
-    // The plan kernel runs before this one; wait for its output.  Then let the
-    // next kernel on the stream get its CTAs resident: it reads nothing the
-    // kernels write before its own wait, which returns only when this grid has
-    // completed.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;");
+    // Wait for the kernels ahead of this one, then let the next kernel on the
+    // stream get its CTAs resident (it reads nothing this grid writes before
+    // its own wait, which returns only when this grid has completed).  When
+    // the plan was complete before this launch started (a.early), only the
+    // consumer warps wait, before they read X and Y: the producer reads the
+    // plan and streams the adapter pages while the kernel ahead drains.
+    const bool early = a.early != 0;
+    auto wait_and_release = []() {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        asm volatile("griddepcontrol.launch_dependents;");
+    };
+    if (!early) wait_and_release();
 
     // Issue the first job record (a guess that holds whenever there are at
     // least half as many jobs as clusters) and the job count together, so
@@ -434,6 +442,7 @@ gather_kernel(const __grid_constant__ GatherMaps<NP> maps, const __grid_constant
     }
     __syncthreads();
     if (n_jobs <= 0) {   // uniform over the grid; no peer traffic has happened
+        if (early) wait_and_release();
         cluster_wait();
         return;
     }
@@ -451,7 +460,7 @@ gather_kernel(const __grid_constant__ GatherMaps<NP> maps, const __grid_constant
         int chunk = 0;
         for (int u = cluster_id; u < n_units; u += n_clusters) {
             const int ji = u / upj;
-            const int4 job = (ji == spec) ? spec_job : a.jobs[2 * ji];
+            const int4 job = (ji == spec) ? spec_job : ld_v4_now(a.jobs + 2 * ji);
             const int pj = (NP == 1) ? 0 : (u - ji * upj) / E, e = u - ji * upj - pj * E;
             const SlotMeta m = slot_meta<MODE>(a, sm, staged, pj, job.x);
             const UnitGeom g = unit_geom<MODE>(a, sm, pj, m.np, e, crank);
@@ -496,6 +505,7 @@ gather_kernel(const __grid_constant__ GatherMaps<NP> maps, const __grid_constant
     // ----------------------------------------------------------------------
     // Consumer warps.
     // ----------------------------------------------------------------------
+    if (early) wait_and_release();
     const int g8 = lane >> 2, tig = lane & 3;    // MMA fragment coordinates
     const int li = lane & 7, lj = lane >> 3;     // ldmatrix: row within a matrix, matrix index
     int chunk = 0;
@@ -860,6 +870,7 @@ int launch_mode(const GatherArgs &ga, lora_pool_s *const *pa, lora_pool_s *const
     a.X = ga.X; a.V = ga.V; a.T = ga.T; a.d_in = ga.d_in; a.S = ga.S; a.nproj = ga.nproj;
     for (int p = 0; p < NP; ++p) a.proj[p] = ga.proj[p < ga.nproj ? p : 0];
     a.perm = ga.perm; a.jobs = ga.jobs; a.hdr = ga.hdr; a.err = ga.err;
+    a.early = (pdl && !plan_was_last_launch(st)) ? 1 : 0;
     GatherMaps<NP> maps;
     int e_max = 1 << 30;
     for (int p = 0; p < a.nproj; ++p) {
@@ -910,6 +921,7 @@ int launch_mode(const GatherArgs &ga, lora_pool_s *const *pa, lora_pool_s *const
     cfg.numAttrs = pdl ? 2 : 1;
     if (int rc = cuda_check(cudaLaunchKernelEx(&cfg, gather_kernel<MODE, NP>, maps, a, e_max))) return rc;
     count_launch();
+    note_launch(st, false);
     return LORA_OK;
 }
 

@@ -105,6 +105,18 @@ int opt_plan_kernel();
 // Record a CUDA error and return LORA_ERR_CUDA, or LORA_OK.
 int cuda_check(cudaError_t e);
 
+// Programmatic launches.  Every library kernel that lets its dependents start
+// early (griddepcontrol.launch_dependents) does so only after its own
+// griddepcontrol.wait, and waits before it exits; the plan kernel, which
+// triggers at once, is launched without the programmatic attribute.  So when
+// a library kernel starts, everything launched on its stream before the
+// kernel just ahead of it has completed and is visible.  The library records,
+// per stream, whether its last launch there was the plan: if not, the plan
+// a launch reads is complete before the launch starts, and the kernel may
+// read it (and the adapter pages it names) before its own wait.
+bool plan_was_last_launch(cudaStream_t st);
+void note_launch(cudaStream_t st, bool is_plan);
+
 // Per-thread launch counter for diagnostics.
 void count_launch(int n = 1);
 void reset_launch_count();

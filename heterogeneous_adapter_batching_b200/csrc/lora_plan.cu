@@ -671,6 +671,7 @@ int launch_plan(const int32_t *ids, int T, const int32_t *ranks, int S, int long
     if (!runs && T <= kSmallTokens && S <= kSmallSlots && opt_plan_kernel() != LORA_PLAN_GENERAL) {
         plan_small_kernel<<<1, 32, 0, st>>>(ids, T, ranks, S, long_thresh, job_tokens, clusters, out, err_dev);
         count_launch();
+        note_launch(st, true);
         return cuda_check(cudaGetLastError());
     }
     if (in_smem)
@@ -678,6 +679,7 @@ int launch_plan(const int32_t *ids, int T, const int32_t *ranks, int S, int long
     else
         plan_kernel<false><<<1, threads, smem, st>>>(ids, T, ranks, S, W, long_thresh, job_tokens, clusters, out, err_dev);
     count_launch();
+    note_launch(st, true);
     return cuda_check(cudaGetLastError());
 }
 

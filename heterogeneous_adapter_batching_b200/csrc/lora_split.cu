@@ -913,6 +913,7 @@ int launch_split(const SplitArgs &s, lora_pool_s *pa, lora_pool_s *pb, cudaStrea
     cfg.dynamicSmemBytes = kExpandSmemBytes;
     if (int rc = cuda_check(cudaLaunchKernelEx(&cfg, expand_part_kernel, tmB, tmB4, k))) return rc;
     count_launch();
+    note_launch(st, false);
     return LORA_OK;
 }
 

@@ -828,6 +828,7 @@ int launch_np(const TileArgs &a, cudaStream_t st, bool pdl, int sms) {
     cfg.numAttrs = pdl ? 1 : 0;
     if (int rc = cuda_check(cudaLaunchKernelEx(&cfg, tiles_kernel<NP, MODE>, maps, k))) return rc;
     count_launch();
+    note_launch(st, false);
     return LORA_OK;
 }
 
