@@ -341,9 +341,11 @@ class Ring:
 
 # workload -> profile summary of its dominant kernel (each names the kernel source it was captured from)
 PROFILE_FOR = {
+    "sweep_8b_distinct_T1024": "profiles/split_kernels_sweep_8b_distinct_T1024.md",
     "decode_q_proj_7b": "profiles/gather_kernel_decode_q_proj_7b.md",
     "mixed_mlp_up": "profiles/gather_kernel_mixed_mlp_up.md",
-    "prefill": "profiles/tiles_kernel_prefill.md",
+    "prefill": "profiles/tiles_kernels_prefill.md",
+    "sweep_8b_one_T1024": "profiles/tiles_kernels_sweep_8b_one_T1024.md",
 }
 
 
