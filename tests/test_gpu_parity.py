@@ -345,3 +345,47 @@ def test_distinct_scales_reach_every_slot(H):
     d1 = Y1[rows].astype(np.float64) - wl.Y_base[rows]
     d2 = Y2[rows].astype(np.float64) - wl.Y_base[rows]
     assert np.abs(d2 - 3.0 * d1).max() <= 1e-4 * np.abs(d1).max() + 1e-6
+
+
+_PLANNED_CASES = {
+    "decode_q_proj_7b": lambda: W.by_name("decode_q_proj_7b"),
+    "mixed_mlp_up": lambda: W.by_name("mixed_mlp_up"),
+    "tiny": lambda: W.by_name("tiny"),
+    # long runs: the tile launches, whose per-tile quarter counters must be back
+    # at 0 for the next layer over the same plan
+    "segments": lambda: W.segments(8, [300, 7, 129, 40, 256], 512, 1024, S=6),
+}
+
+
+@pytest.mark.parametrize("name", sorted(_PLANNED_CASES))
+@pytest.mark.parametrize("path", ["cluster", "split"])
+def test_planned_layers_after_one_plan_bit_exact(H, name, path):
+    """One plan, then several layers on the same stream: every layer after the
+    first starts while the previous one drains and reads the plan (and, on the
+    cluster path, the adapter pages) before its grid-dependency wait.  Each layer
+    must equal the one-call lora_apply on its own inputs, bit for bit, and the
+    oracle."""
+    import torch
+    old = H.lora_get_option(H.OPT_GATHER_PATH)
+    H.lora_set_option(H.OPT_GATHER_PATH, H.GATHER_CLUSTER if path == "cluster" else H.GATHER_SPLIT)
+    try:
+        wl = _PLANNED_CASES[name]()
+        layers = [U.make_layer(wl) for _ in range(3)]
+        X, _, ids = U.dev_inputs(wl)
+        Ys = [U.dev_inputs(wl)[1] for _ in layers]
+        stream = torch.cuda.Stream()
+        with torch.cuda.stream(stream):
+            layers[0].plan(ids, stream=stream)
+            for lay, Y in zip(layers, Ys):
+                lay.apply_planned(X, Y, stream=stream, ws=layers[0].ws)
+        torch.cuda.synchronize()
+        ref_one, _, _ = _run_apply(H, wl)
+        oracle, _ = U.oracle_full(wl)
+        for lay, Y in zip(layers, Ys):
+            assert int(lay.err.item()) == 0
+            y = Y.cpu().numpy()
+            assert np.array_equal(y, ref_one)
+            U.assert_parity(y, oracle, wl.Y_base,
+                            delta_rel=U.DELTA_REL_TENSOR if name == "segments" else U.DELTA_REL_GATHER)
+    finally:
+        H.lora_set_option(H.OPT_GATHER_PATH, old)
