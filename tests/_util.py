@@ -6,7 +6,7 @@ import numpy as np
 
 import workloads as W
 
-# Spec tolerance per element (fp32 accumulate): |err| <= 2e-3 + 1e-2 |ref|.
+# Required tolerance per element (fp32 accumulate): |err| <= 2e-3 + 1e-2 |ref|.
 ATOL, RTOL = 2e-3, 1e-2
 # A stricter bound on the adapter delta alone, relative to its largest magnitude.
 # It separates a wrong rank row / adapter / scale (O(1) relative) from rounding.
