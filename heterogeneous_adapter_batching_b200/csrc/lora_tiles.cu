@@ -128,6 +128,12 @@ __device__ __forceinline__ void drain_wait(uint64_t *b, uint32_t par) {
     while (!mbar_try(a, par) && clock64() - t0 < kWaitLimit / 8) {
     }
 }
+// A plan field read through L2 (the plan may come from a kernel before the one ahead).
+__device__ __forceinline__ int ld_l2(const int *p) {
+    int v;
+    asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
 template <class Sm>
 __device__ __forceinline__ bool aborted(const Sm &sm) { return *(volatile const int *)&sm.abort != 0; }
 __device__ __forceinline__ void mbar_arrive(uint64_t *b) {
@@ -368,11 +374,23 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
     }
     asm volatile("" ::"l"(a.X), "r"(a.T), "r"(a.d_in), "l"(a.tiles), "l"(a.hdr), "l"(a.err));
     // The kernels before this one on the stream produce the plan (and, for
-    // kExpandV, v).  A batch without long runs has no tiles: leave before
-    // touching tensor memory.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int n_tiles = a.hdr->n_tiles;
-    if (n_tiles <= 0) return;   // uniform over the grid
+    // kExpandV, v).  The shrink launch lets its dependent (the expand launch)
+    // get resident once it has waited.  In the expand launch only the producer
+    // waits, after it has issued its first unit's B and Y loads and before it
+    // loads v: when it starts, every kernel before the shrink launch, the plan
+    // included, has completed (the shrink launch released it only after its
+    // own wait), and the shrink launch writes nothing else it reads.  A batch
+    // without long runs has no tiles: leave (after waiting) before touching
+    // tensor memory.
+    if (MODE != kExpandV) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        if (MODE == kShrinkQ) asm volatile("griddepcontrol.launch_dependents;");
+    }
+    const int n_tiles = ld_l2(&a.hdr->n_tiles);
+    if (n_tiles <= 0) {   // uniform over the grid
+        if (MODE == kExpandV) asm volatile("griddepcontrol.wait;" ::: "memory");
+        return;
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kSt; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], 1); }
@@ -451,25 +469,44 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
         // ---------------- expand operand producer: v (kExpandV), B and Y ----------------
         if constexpr (MODE != kShrinkQ) {
             int it = 0, itv = 0;
+            bool waited = MODE != kExpandV;
             UnitIter ur = unit_range(n_tiles, nj);
             UnitInfo ui;
-            while (next_unit(a, ur, ui) && !aborted(sm)) {
+            // kExpandV: the unit's v, high and low part, straight into the MMA's
+            // operand tiles (the first one after waiting for the shrink launch)
+            bool v_done = true;
+            auto issue_v = [&]() {
+                if (!waited) {
+                    asm volatile("griddepcontrol.wait;" ::: "memory");
+                    waited = true;
+                }
+                if (!mbar_wait(&sm.v_empty, (itv & 1) ^ 1, sm, a.err)) return false;
+                mbar_expect_tx(&sm.v_full, (uint32_t)(2 * kM * 64 * 2));
+                tma_load(sm.vs, &maps.V, 0, ui.row0, &sm.v_full);
+                tma_load(sm.vl, &maps.V, 64, ui.row0, &sm.v_full);
+                ++itv;
+                v_done = true;
+                return true;
+            };
+            bool ok = true;
+            while (ok && next_unit(a, ur, ui) && !aborted(sm)) {
                 if constexpr (MODE == kExpandV)
                     if (ui.bad && a.err) atomicOr(a.err, LORA_DEV_ERR_BAD_PAGE);
                 if (ui.skip) continue;
                 if constexpr (MODE == kExpandV) {
-                    // the unit's v, high and low part, straight into the MMA's operand tiles
-                    if (!mbar_wait(&sm.v_empty, (itv & 1) ^ 1, sm, a.err)) break;
-                    mbar_expect_tx(&sm.v_full, (uint32_t)(2 * kM * 64 * 2));
-                    tma_load(sm.vs, &maps.V, 0, ui.row0, &sm.v_full);
-                    tma_load(sm.vl, &maps.V, 64, ui.row0, &sm.v_full);
-                    ++itv;
+                    v_done = false;
+                    if (waited && !issue_v()) break;
                 }
                 int pg[4];
                 const int32_t *pt = a.proj[ui.p].pt;
                 for (int p = 0; p < 4; ++p) pg[p] = p < ui.np ? pt[ui.slot * 8 + 4 + p] : 0;
                 const CUtensorMap *tmB = &maps.B[ui.p], *tmY = &maps.Y[ui.p];
                 for (int j = ui.j0; j < ui.j1; ++j, ++it) {
+                    // the first unit's first kBuf items need nothing from the shrink launch
+                    if (!v_done && j - ui.j0 == kBuf && !issue_v()) {
+                        ok = false;
+                        break;
+                    }
                     const int b = it % kBuf;
                     const uint32_t par = ((it / kBuf) & 1) ^ 1;
                     if (!mbar_wait(&sm.bempty[b], par, sm, a.err)) break;
@@ -481,7 +518,9 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
                     tma_load(&sm.ys[b][0], tmY, j * kNB, ui.row0, &sm.yfull[b]);
                     tma_load(&sm.ys[b][kM * 32], tmY, j * kNB + 32, ui.row0, &sm.yfull[b]);
                 }
+                if (ok && !v_done && !issue_v()) ok = false;   // a first unit of at most kBuf items
             }
+            if (!waited) asm volatile("griddepcontrol.wait;" ::: "memory");   // before the CTA can finish
             for (int i = (it > kBuf ? it - kBuf : 0); i < it; ++i) {
                 drain_wait(&sm.bfull[i % kBuf], (i / kBuf) & 1);
                 drain_wait(&sm.yfull[i % kBuf], (i / kBuf) & 1);
