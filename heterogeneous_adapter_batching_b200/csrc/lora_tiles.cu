@@ -667,15 +667,16 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
                         float v[64];
 #pragma unroll
                         for (int c = 0; c < 64; ++c) v[c] = 0.f;
+                        // all four quarters' loads in flight at once; added in quarter order
+#pragma unroll
                         for (int q2 = 0; q2 < kSlicesQ; ++q2) {
                             int b0, b1;
                             quarter_blocks(nkb, q2, b0, b1);
-                            if (b1 <= b0) continue;
                             const float4 *src =
                                 reinterpret_cast<const float4 *>(a.vpart + ((size_t)q2 * a.T + ui.row0 + m) * LORA_MAX_RANK);
 #pragma unroll
                             for (int c = 0; c < 16; ++c) {
-                                if (c < ui.np * 4) {
+                                if (b1 > b0 && c < ui.np * 4) {
                                     const float4 w = __ldcg(src + c);
                                     v[4 * c] += w.x;
                                     v[4 * c + 1] += w.y;
