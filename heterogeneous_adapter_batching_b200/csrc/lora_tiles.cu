@@ -617,6 +617,7 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
         const int m = q * 32 + lane;         // tile row = accumulator lane
         const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
         const bool leader = (warp == 4 && lane == 0);
+        int pending = -1;   // Y buffer whose TMA store may still be reading it
         int ite = 0, itt = 0;
         // v (fp32, row m) -> bf16 high part and low part (v - high), the two
         // 16-significant-bit halves the expand multiplies by B
@@ -751,8 +752,11 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
                     mbar_arrive(&sm.v_ready);
                 }
                 // n-tiles: y = s * D2 + y on the Y tile in shared memory (row m
-                // per thread), then the rows of the unit's tokens go back with
-                // coalesced stores from all 128 threads
+                // per thread); a full tile goes back with two TMA stores issued by
+                // one thread (its buffer is released once the store has read it,
+                // one item later), a tile of fewer than 128 tokens with coalesced
+                // row stores of its tokens from all 128 threads
+                const bool full_tile = ui.ntok == kM;
                 for (int j = ui.j0; j < ui.j1; ++j, ++ite) {
                     const int b = ite % kBuf;
                     const uint32_t par = (ite / kBuf) & 1;
@@ -778,27 +782,53 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
                         y.w = fmaf(sc, acc[c * 4 + 3], y.w);
                         *yp = y;
                     }
-                    epi_sync();
-                    // 16 threads per row, one 16-byte group each: row r, group g
-                    const int tid = threadIdx.x - 128;
-#pragma unroll 4
-                    for (int i = 0; i < 16; ++i) {
-                        const int idx = tid + 128 * i, r = idx >> 4, g = idx & 15;
-                        const int col = j * kNB + 4 * g;
-                        if (r < ui.ntok && col < pr.d_out) {
-                            const int h = g >> 3, cc = g & 7;
-                            const float4 y =
-                                *reinterpret_cast<const float4 *>(yt + h * kM * 128 + r * 128 + ((cc ^ (r & 7)) << 4));
-                            *reinterpret_cast<float4 *>(pr.Y + (size_t)(ui.row0 + r) * pr.d_out + col) = y;
-                        }
-                    }
-                    // the tile was read and written through the generic proxy; order
-                    // that before the producer's next TMA load into it
+                    // the tile was written through the generic proxy; order that
+                    // before the TMA store or the producer's next TMA load into it
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     epi_sync();
-                    if (leader) mbar_arrive(&sm.yempty[b]);
+                    if (full_tile) {
+                        if (leader) {
+                            tma_store(&maps.Y[ui.p], j * kNB, ui.row0, &sm.ys[b][0]);
+                            tma_store(&maps.Y[ui.p], j * kNB + 32, ui.row0, &sm.ys[b][kM * 32]);
+                            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                            // the previous store has left its buffer once at most one
+                            // group (this one) is still reading
+                            asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                            if (pending >= 0) mbar_arrive(&sm.yempty[pending]);
+                            pending = b;
+                        }
+                    } else {
+                        // 16 threads per row, one 16-byte group each: row r, group g
+                        const int tid = threadIdx.x - 128;
+#pragma unroll 4
+                        for (int i = 0; i < 16; ++i) {
+                            const int idx = tid + 128 * i, r = idx >> 4, g = idx & 15;
+                            const int col = j * kNB + 4 * g;
+                            if (r < ui.ntok && col < pr.d_out) {
+                                const int h = g >> 3, cc = g & 7;
+                                const float4 y =
+                                    *reinterpret_cast<const float4 *>(yt + h * kM * 128 + r * 128 + ((cc ^ (r & 7)) << 4));
+                                *reinterpret_cast<float4 *>(pr.Y + (size_t)(ui.row0 + r) * pr.d_out + col) = y;
+                            }
+                        }
+                        epi_sync();
+                        if (leader) {
+                            // a buffer whose store is still pending would otherwise wait
+                            // for the next full tile, which may never come on this CTA
+                            if (pending >= 0) {
+                                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                                mbar_arrive(&sm.yempty[pending]);
+                                pending = -1;
+                            }
+                            mbar_arrive(&sm.yempty[b]);
+                        }
+                    }
                 }
                 ++itt;
+            }
+            if (leader) {
+                asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+                if (pending >= 0) mbar_arrive(&sm.yempty[pending]);
             }
         }
     }
