@@ -332,21 +332,37 @@ __device__ __forceinline__ bool next_unit(const KTile<NP> &a, UnitIter &u, UnitI
     return true;
 }
 
-// Units of the shrink-only launch: (tile, quarter q of the K blocks), handed
-// out round robin.  Quarter q covers K blocks [nkb q / 4, nkb (q + 1) / 4);
-// with fewer than four K blocks some quarters are empty and hold no partial.
+// Units of the shrink-only launch: (tile, quarter q of the K blocks), in
+// that order; every CTA takes an equal contiguous range, so a CTA mostly
+// holds all four quarters of its tiles and the reductions that finish the
+// tiles (done by whichever CTA completes a tile's last quarter) spread evenly
+// instead of piling up on CTAs that fell behind.  Quarter q covers K blocks
+// [nkb q / 4, nkb (q + 1) / 4); with fewer than four K blocks some quarters
+// are empty and hold no partial.
 __device__ __forceinline__ void quarter_blocks(int nkb, int q, int &kb0, int &kb1) {
     kb0 = nkb * q / kSlicesQ;
     kb1 = nkb * (q + 1) / kSlicesQ;
 }
 
+struct QIter {
+    int u, u1;   // next unit, end of this CTA's range
+};
+
+__device__ __forceinline__ QIter qunit_range(int n_tiles) {
+    const long long total = (long long)n_tiles * kSlicesQ;
+    QIter it;
+    it.u = (int)(total * blockIdx.x / gridDim.x);
+    it.u1 = (int)(total * (blockIdx.x + 1) / gridDim.x);
+    return it;
+}
+
 template <int NP>
-__device__ __forceinline__ bool next_qunit(const KTile<NP> &a, int n_tiles, int &u, UnitInfo &ui, int &q) {
-    if (u >= n_tiles * kSlicesQ) return false;
-    const int tile = u / kSlicesQ;
-    q = u - tile * kSlicesQ;
+__device__ __forceinline__ bool next_qunit(const KTile<NP> &a, QIter &it, UnitInfo &ui, int &q) {
+    if (it.u >= it.u1) return false;
+    const int tile = it.u / kSlicesQ;
+    q = it.u - tile * kSlicesQ;
     ui = unit_info(a, tile, 0, 0, 1);
-    u += gridDim.x;
+    ++it.u;
     return true;
 }
 
@@ -454,9 +470,10 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
                 if (!load_kblocks(ui, 0, nkb)) break;
             }
         } else if constexpr (MODE == kShrinkQ) {
-            int u = blockIdx.x, q = 0, kb0, kb1;
+            QIter u = qunit_range(n_tiles);
+            int q = 0, kb0, kb1;
             UnitInfo ui;
-            while (next_qunit(a, n_tiles, u, ui, q) && !aborted(sm)) {
+            while (next_qunit(a, u, ui, q) && !aborted(sm)) {
                 if (ui.bad && q == 0 && a.err) atomicOr(a.err, LORA_DEV_ERR_BAD_PAGE);
                 quarter_blocks(nkb, q, kb0, kb1);
                 if (ui.skip || kb1 <= kb0) continue;
@@ -587,9 +604,10 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
             return true;
         };
         if constexpr (MODE == kShrinkQ) {
-            int u = blockIdx.x, q = 0, kb0, kb1;
+            QIter u = qunit_range(n_tiles);
+            int q = 0, kb0, kb1;
             UnitInfo ui;
-            while (next_qunit(a, n_tiles, u, ui, q) && !aborted(sm)) {
+            while (next_qunit(a, u, ui, q) && !aborted(sm)) {
                 quarter_blocks(nkb, q, kb0, kb1);
                 if (ui.skip || kb1 <= kb0) continue;
                 if (!shrink(ui, q, q + 1, false)) break;
@@ -636,9 +654,10 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
             // D1 rows of the tile's tokens -> the quarter's fp32 partials; the
             // CTA that finishes a tile's last quarter adds the quarters in
             // order and leaves v (bf16 high, low) in quarter 0's rows
-            int u = blockIdx.x, qq = 0, kb0, kb1;
+            QIter u = qunit_range(n_tiles);
+            int qq = 0, kb0, kb1;
             UnitInfo ui;
-            while (next_qunit(a, n_tiles, u, ui, qq)) {
+            while (next_qunit(a, u, ui, qq)) {
                 if (!epi_all(!aborted(sm))) break;
                 quarter_blocks(nkb, qq, kb0, kb1);
                 if (ui.skip || kb1 <= kb0) continue;
