@@ -78,12 +78,12 @@ template <int MODE>
 struct SmemOf {
     using type = TileSmemT<MODE == kExpandV ? 1 : (MODE == kShrinkQ ? 6 : kStages), MODE == kShrinkQ ? 1 : (MODE == kExpandV ? 4 : 3)>;
 };
-// Tensor-memory columns: the shrink's D1 of quarter q at [64 q, 64 q + 64)
-// (kShrinkQ: its one quarter at [0, 64)); expand accumulator b at
+// Tensor-memory columns: the shrink's D1 of quarter q at [64 q, 64 q + 64);
+// expand accumulator b at
 // [kAccCol + 64 b, kAccCol + 64 b + 64).
 constexpr int kAccCol = 64 * kSlicesQ;
 template <int MODE>
-constexpr uint32_t tmem_cols() { return MODE == kShrinkQ ? 64u : 512u; }
+constexpr uint32_t tmem_cols() { return MODE == kShrinkQ ? 256u : 512u; }
 
 static_assert(sizeof(SmemOf<kFused>::type) + 1024 <= 227 * 1024, "tiles kernel: shared memory beyond the per-block limit");
 static_assert(sizeof(SmemOf<kShrinkQ>::type) + 1024 <= 227 * 1024, "tiles kernel: shared memory beyond the per-block limit");
@@ -345,13 +345,13 @@ __device__ __forceinline__ void quarter_blocks(int nkb, int q, int &kb0, int &kb
 }
 
 struct QIter {
-    int u, u1;   // next unit, end of this CTA's range
+    int u0, u, u1;   // start of this CTA's range, next unit, end of the range
 };
 
 __device__ __forceinline__ QIter qunit_range(int n_tiles) {
     const long long total = (long long)n_tiles * kSlicesQ;
     QIter it;
-    it.u = (int)(total * blockIdx.x / gridDim.x);
+    it.u0 = it.u = (int)(total * blockIdx.x / gridDim.x);
     it.u1 = (int)(total * (blockIdx.x + 1) / gridDim.x);
     return it;
 }
@@ -610,7 +610,7 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
             while (next_qunit(a, u, ui, q) && !aborted(sm)) {
                 quarter_blocks(nkb, q, kb0, kb1);
                 if (ui.skip || kb1 <= kb0) continue;
-                if (!shrink(ui, q, q + 1, false)) break;
+                if (!shrink(ui, q, q + 1, true)) break;
                 ++itt;
             }
         } else {
@@ -637,6 +637,28 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
         const bool leader = (warp == 4 && lane == 0);
         int pending = -1;   // Y buffer whose TMA store may still be reading it
         int ite = 0, itt = 0;
+        // row m of v (fp32) -> its bf16 high part (bytes 0..127 of quarter 0's
+        // workspace row) and low part (bytes 128..255), one 16-byte group of
+        // eight values at a time
+        auto store_v_row = [&](const float (&v)[64], int np, float *row) {
+            uint4 *dst = reinterpret_cast<uint4 *>(row);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                if (c < np * 2) {
+                    uint32_t hw[4], lw[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float f0 = v[c * 8 + 2 * e], f1 = v[c * 8 + 2 * e + 1];
+                        const __nv_bfloat162 h = __floats2bfloat162_rn(f0, f1);
+                        const __nv_bfloat162 l = __floats2bfloat162_rn(f0 - __low2float(h), f1 - __high2float(h));
+                        hw[e] = *reinterpret_cast<const uint32_t *>(&h);
+                        lw[e] = *reinterpret_cast<const uint32_t *>(&l);
+                    }
+                    dst[c] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    dst[8 + c] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                }
+            }
+        };
         // v (fp32, row m) -> bf16 high part and low part (v - high), the two
         // 16-significant-bit halves the expand multiplies by B
         auto split_v = [&](const float (&v)[64], int np, uint32_t (&hw)[32], uint32_t (&lw)[32]) {
@@ -651,11 +673,19 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
             }
         };
         if constexpr (MODE == kShrinkQ) {
-            // D1 rows of the tile's tokens -> the quarter's fp32 partials; the
-            // CTA that finishes a tile's last quarter adds the quarters in
-            // order and leaves v (bf16 high, low) in quarter 0's rows
+            // A tile whose four quarters all lie in this CTA's range keeps each
+            // quarter's D1 in its own tensor-memory block; at its last quarter
+            // the epilogue adds the blocks in quarter order and leaves v (bf16
+            // high, low) in quarter 0's rows of the workspace.  Any other tile:
+            // D1 rows of its tokens -> the quarter's fp32 partials, and the CTA
+            // that finishes the tile's last quarter adds the quarters in order
+            // from there.  Both give the same sums.
             QIter u = qunit_range(n_tiles);
-            int qq = 0, kb0, kb1;
+            int qq = 0, kb0, kb1, last_q = 0;
+            for (int q2 = 0; q2 < kSlicesQ; ++q2) {
+                quarter_blocks(nkb, q2, kb0, kb1);
+                if (kb1 > kb0) last_q = q2;
+            }
             UnitInfo ui;
             while (next_qunit(a, u, ui, qq)) {
                 if (!epi_all(!aborted(sm))) break;
@@ -663,10 +693,42 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
                 if (ui.skip || kb1 <= kb0) continue;
                 if (!epi_all(mbar_wait(&sm.shrink_done, itt & 1, sm, a.err))) break;
                 tc_fence_after();
+                const bool owned = ui.tile * kSlicesQ >= u.u0 && ui.tile * kSlicesQ + kSlicesQ <= u.u1;
+                if (owned) {
+                    if (qq == last_q) {
+                        float v[64];
+#pragma unroll
+                        for (int c = 0; c < 64; ++c) v[c] = 0.f;
+                        for (int q2 = 0; q2 < kSlicesQ; ++q2) {
+                            int b0, b1;
+                            quarter_blocks(nkb, q2, b0, b1);
+                            if (b1 <= b0) continue;
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                if (c < ui.np) {
+                                    float t16[16];
+                                    TMEM_LD16(trow + 64 * q2 + c * 16, t16);
+                                    tmem_wait_ld();
+#pragma unroll
+                                    for (int i = 0; i < 16; ++i) v[c * 16 + i] += t16[i];
+                                }
+                            }
+                        }
+                        tc_fence_before();
+                        mbar_arrive(&sm.d1_empty);
+                        if (m < ui.ntok) store_v_row(v, ui.np, a.vpart + ((size_t)ui.row0 + m) * LORA_MAX_RANK);
+                    } else {
+                        // the block stays until the tile's last quarter reads it
+                        tc_fence_before();
+                        mbar_arrive(&sm.d1_empty);
+                    }
+                    ++itt;
+                    continue;
+                }
                 float d1[64];
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
-                    if (c < ui.np) TMEM_LD16(trow + c * 16, (&d1[c * 16]));
+                    if (c < ui.np) TMEM_LD16(trow + 64 * qq + c * 16, (&d1[c * 16]));
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&sm.d1_empty);
@@ -705,16 +767,7 @@ tiles_kernel(const __grid_constant__ TileMaps<NP> maps, const __grid_constant__ 
                                 }
                             }
                         }
-                        uint32_t hw[32], lw[32];
-                        split_v(v, ui.np, hw, lw);
-                        uint4 *dst = reinterpret_cast<uint4 *>(a.vpart + ((size_t)ui.row0 + m) * LORA_MAX_RANK);
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            if (c < ui.np * 2) {
-                                dst[c] = make_uint4(hw[4 * c], hw[4 * c + 1], hw[4 * c + 2], hw[4 * c + 3]);
-                                dst[8 + c] = make_uint4(lw[4 * c], lw[4 * c + 1], lw[4 * c + 2], lw[4 * c + 3]);
-                            }
-                        }
+                        store_v_row(v, ui.np, a.vpart + ((size_t)ui.row0 + m) * LORA_MAX_RANK);
                     }
                     if (leader) a.tiles[ui.tile].w = 0;   // ready for the next launch over this plan
                 }
