@@ -58,6 +58,10 @@ def _apply(wl, H=None):
     (4, [513, 7, 1000], 1032, 520),
     (5, [90, 33, 256, 256, 12], 4096, 4096),
     (6, [5000], 256, 512),
+    # many tiles per CTA (whole tiles finished from tensor memory) with empty
+    # quarters of d_in: one K block (quarters 0-2 empty), three (quarter 0 empty)
+    (7, [20000], 64, 128),
+    (8, [20000], 192, 128),
 ])
 def test_tile_path_segments(H, thresh, seed, lens, d_in, d_out):
     H.lora_set_option(H.OPT_LONG_SEGMENT, thresh)
