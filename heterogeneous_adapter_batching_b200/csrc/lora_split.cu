@@ -793,41 +793,31 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
                     }
                 }
             }
-            // fragment (column g8 / g8 + 8, tokens 2 tig, 2 tig + 1) into the Y rows
+            // y = fmaf(s, acc, y) for column g8 / g8 + 8 and tokens 2 tig,
+            // 2 tig + 1, the old value from the staged Y rows, the new one
+            // straight to global memory (eight consecutive columns of a row per
+            // store)
 #pragma unroll
-            for (int q = 0; q < kTilesPerWarp; ++q) {
-                if (!has[q]) continue;
-                const int mt = mt0 + q * kCW;
+            for (int jj = 0; jj < kMaxNT; ++jj) {
+                if (jj < nt) {
+                    const int t0 = jj * kNTok + 2 * tig;
+                    const int tok0 = t0 < n ? h.tok[t0] : 0, tok1 = t0 + 1 < n ? h.tok[t0 + 1] : 0;
 #pragma unroll
-                for (int jj = 0; jj < kMaxNT; ++jj) {
-                    if (jj < nt) {
+                    for (int q = 0; q < kTilesPerWarp; ++q) {
+                        if (!has[q]) continue;
+                        const int mt = mt0 + q * kCW;
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            const int t = jj * kNTok + 2 * tig + (i & 1), cc = mt * 16 + g8 + 8 * (i >> 1);
-                            if (t < n && c0 + cc < hi) {
-                                float *y = ys + t * py4 + cc;
-                                *y = fmaf(sc, d[q][jj][i], *y);
-                            }
+                            const int t = t0 + (i & 1), cc = mt * 16 + g8 + 8 * (i >> 1);
+                            if (t < n && c0 + cc < hi)
+                                a.Y[(size_t)((i & 1) ? tok1 : tok0) * a.d_out + c0 + cc] =
+                                    fmaf(sc, d[q][jj][i], ys[t * py4 + cc]);
                         }
                     }
                 }
             }
-            __syncwarp();
-#pragma unroll
-            for (int q = 0; q < kTilesPerWarp; ++q) {
-                if (!has[q]) continue;
-                const int mt = mt0 + q * kCW;
-                for (int idx = lane; idx < n * 4; idx += 32) {
-                    const int t = idx >> 2, col = mt * 16 + 4 * (idx & 3);
-                    if (c0 + col < hi)
-                        *reinterpret_cast<float4 *>(a.Y + (size_t)h.tok[t] * a.d_out + c0 + col) =
-                            *reinterpret_cast<const float4 *>(ys + t * py4 + col);
-                }
-            }
         }
-        // the Y rows were written through the generic proxy; order that before
-        // the producer's next bulk copy into this stage
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        // the staged Y rows were only read
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.empty[st]);
         ++chunk;
