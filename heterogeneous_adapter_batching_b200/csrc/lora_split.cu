@@ -69,8 +69,9 @@ constexpr long long kWaitLimit = 2000000000LL;             // cycles (~1 s)
 constexpr int kVPartFloats = LORA_MAX_JOB_TOKENS * LORA_MAX_RANK;
 constexpr int kVTileBytes = LORA_MAX_JOB_TOKENS * LORA_MAX_RANK * 2;   // one bf16 part of v
 
-static_assert(kShrinkArena >= 3 * (16 * kBoxBytes + kRowRegion) && kExpandArena >= 2 * kMaxChunk,
-              "the rings hold at least three shrink or two expand chunks");
+static_assert(kShrinkArena / 2 >= kMaxPages * kBoxBytes + LORA_MAX_JOB_TOKENS * (kBoxCols * 2 + 16) &&
+                  kExpandArena >= 2 * kMaxChunk,
+              "the rings hold at least two chunks");
 static_assert(kMaxNT * kNTok == LORA_MAX_JOB_TOKENS, "job size must be a whole number of MMA tiles");
 
 // What the producer tells the consumers about one chunk.
@@ -365,7 +366,9 @@ shrink_part_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             const int nt = (n + kNTok - 1) / kNTok;
             const int in0 = 8 * (int)(Gi * s / kSlices), in1 = 8 * (int)(Gi * (s + 1) / kSlices);
             if (in1 <= in0) continue;
-            const int nb = min(16 / m.np, nt > 1 ? 8 : 16);
+            // as many 64-column blocks per page as keep two chunks in the ring
+            int nb = max(1, min(kMaxBoxes / m.np, nt > 1 ? 8 : 16));
+            while (nb > 1 && m.np * nb * kBoxBytes + nt * kNTok * (nb * kBoxCols * 2 + 16) > kShrinkArena / 2) --nb;
             const int cw = nb * kBoxCols, px = cw * 2 + 16;
             const int nch = (in1 - in0 + cw - 1) / cw;
             const int box_bytes = m.np * nb * kBoxBytes;
