@@ -625,7 +625,9 @@ expand_part_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constan
             if (out1 <= out0) continue;
             const int nt = (n + kNTok - 1) / kNTok;
             const int ylim = ((kRowRegion / n) - 16) / 4 / kBoxCols;   // Y rows of a chunk fit the row region
-            const int nb = max(1, min(min(kMaxBoxes / m.np, 16), ylim));
+            // as many 64-column blocks per page as keep two chunks in the ring
+            int nb = max(1, min(16, ylim));
+            while (nb > 1 && m.np * nb * kBoxBytes + n * (nb * kBoxCols * 4 + 16) > kExpandArena / 2) --nb;
             const int cw = nb * kBoxCols, py = cw * 4 + 16;
             const int nch = (out1 - out0 + cw - 1) / cw;
             const int vb = nv & 1;
