@@ -252,6 +252,18 @@ int lora_apply(const uint16_t *X, float *Y, int T, int d_in, int d_out, const in
  * options).  A model applies one plan to all of its adapted layers: a token's
  * adapter slot is the same in every layer, only the pools, page tables and
  * scales differ.  Launches only the compute kernels. */
+/* The compute half of lora_apply over the plan that lora_plan (or an earlier
+ * apply call on the same batch) left in ws: a model plans once per batch (a
+ * token's adapter is the same in every layer) and calls this for every
+ * adapted projection.  Arguments, layouts and errors as lora_apply without
+ * ids.  Ordering: the library's kernels let the next kernel on the stream
+ * start before they finish and release it only after their own wait, so when
+ * the plan was not the library's last launch on this stream, this call reads
+ * the plan and starts loading adapter pages before it waits for the kernel
+ * ahead (X and Y are read only after that wait).  Plain launches, events and
+ * CUDA graphs keep this safe; a caller's own kernel launched between lora_plan
+ * and this call with programmatic dependent launch that releases its
+ * dependents before its own wait does not. */
 int lora_apply_planned(const uint16_t *X, float *Y, int T, int d_in, int d_out, int num_slots,
                        const int32_t *ranks, const float *scales, const int32_t *page_table,
                        lora_pool_t pa, lora_pool_t pb, void *ws, size_t ws_bytes,
@@ -283,7 +295,7 @@ typedef struct {
  *   projection is skipped there).  Short segments of every projection are
  *   handled by one gather launch (on the split gather path: a shrink and an
  *   expand launch per projection); long runs by one tile launch for all
- *   projections.  ws as for lora_apply (lora_workspace_size(T, num_slots)).
+ *   projections (one projection: a tile shrink and a tile expand launch).  ws as for lora_apply (lora_workspace_size(T, num_slots)).
  * Each projection's result is bit-identical to lora_apply on that projection
  * alone.  Errors: as lora_apply, checked for every projection before any
  * work is enqueued; LORA_ERR_INVALID_ARG for num_projs out of range. */
