@@ -57,11 +57,12 @@ constexpr int kNTok = 8;                     // tokens per MMA (the N side)
 constexpr int kMaxNTiles = LORA_MAX_JOB_TOKENS / kNTok;
 constexpr int kMaxJobTokens = kMaxNTiles * kNTok;
 constexpr int kMaxPages = LORA_MAX_RANK / LORA_PAGE_ROWS;
-constexpr int kStages = 4;
+constexpr int kStages = 2;
 constexpr int kBoxCols = 64;                 // TMA box: 16 rows x 64 columns of bf16 = 2 KB, 128B swizzle
 constexpr int kBoxBytes = LORA_PAGE_ROWS * kBoxCols * 2;
-constexpr int kStageBoxes = 16;              // a stage holds 16 boxes = 32 KB
-constexpr int kMaxChunkCols = kStageBoxes * kBoxCols;   // chunk width with a single page
+constexpr int kStageBoxes = 32;              // a stage holds 32 boxes = 64 KB
+constexpr int kMaxPageBoxes = 16;            // 64-column blocks of one page in a chunk at most
+constexpr int kMaxChunkCols = kMaxPageBoxes * kBoxCols;   // widest chunk (1024 columns)
 constexpr int kTableSlots = 128;             // page tables up to this many slots live in shared memory
 constexpr long long kWaitLimit = 2000000000LL;   // cycles (~1 s)
 constexpr int kMaxSplit = 64;                // most parts d_out is split into
@@ -318,10 +319,11 @@ __device__ __forceinline__ UnitGeom unit_geom(const Args &a, const GatherSmem &s
     const unsigned ge0 = (unsigned)sm.ebound[pj][e], ge1 = (unsigned)sm.ebound[pj][e + 1];
     g.out0 = 8 * (int)(ge0 + (ge1 - ge0) * crank / kCS);
     g.out1 = 8 * (int)(ge0 + (ge1 - ge0) * (crank + 1) / kCS);
-    // As many boxes per page as fit in a stage: the chunk width depends on the
-    // rank only, so a token's fp32 summation order does not depend on which
-    // job it lands in.
-    g.nb = np > 0 ? kStageBoxes / np : 1;
+    // As many boxes per page as fit in a stage (at most 16 per page, the width
+    // of the X buffers): the chunk width depends on the rank only.  A token's
+    // fp32 summation order depends on neither the chunk width nor the job it
+    // lands in: 16-column steps and tiles are numbered across the whole slice.
+    g.nb = np > 0 ? min(kStageBoxes / np, kMaxPageBoxes) : 1;
     const int cw = g.nb * kBoxCols;
     const int win = g.in1 - g.in0, wout = g.out1 - g.out0;
     g.n_shrink = (MODE == kExpand || win <= 0 || np == 0) ? 0 : (win + cw - 1) / cw;
