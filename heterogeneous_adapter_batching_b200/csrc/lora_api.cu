@@ -360,10 +360,11 @@ static int run_tiles(const uint16_t *X, int T, int d_in, const lora_projection_t
 // (a pool of at least kSplitMinSlots slots and at least kSplitMinTokens
 // tokens, one projection).  Measured on B200 at the 7B/8B shapes, the cluster
 // kernel is faster with few gather jobs (decode over a small pool, one shared
-// adapter, mixed-rank MLPs over 128 slots: 10-35 % ahead), the split pair with
-// many (64 and 512 distinct rank-64 adapters at d_out 14336: 23 % and 36 %
+// adapter, mixed-rank MLPs over 128 slots: 30-45 % ahead), the split pair with
+// many (64 and 512 distinct rank-64 adapters at d_out 14336: 7 % and 26 %
 // ahead).  The job count itself is known only on the device, so the host
-// decides from the pool size and the token count.
+// decides from the pool size and the token count (one shared adapter over a
+// large pool at 64 tokens takes the split pair, 20 % behind).
 constexpr int kSplitMinSlots = 256;
 constexpr int kSplitMinTokens = 64;
 
