@@ -359,12 +359,12 @@ static int run_tiles(const uint16_t *X, int T, int d_in, const lora_projection_t
 // LORA_GATHER_AUTO: the split path where many distinct adapters are likely
 // (a pool of at least kSplitMinSlots slots and at least kSplitMinTokens
 // tokens, one projection).  Measured on B200 at the 7B/8B shapes, the cluster
-// kernel is faster with few gather jobs (decode over a small pool, one shared
-// adapter, mixed-rank MLPs over 128 slots: 30-45 % ahead), the split pair with
-// many (64 and 512 distinct rank-64 adapters at d_out 14336: 7 % and 26 %
-// ahead).  The job count itself is known only on the device, so the host
+// kernel takes 18-30 % less time with few gather jobs (decode over a small
+// pool, one shared adapter, mixed-rank MLPs over 128 slots), the split pair
+// with many (64 and 512 distinct rank-64 adapters at d_out 14336: 7 % and 26 %
+// less).  The job count itself is known only on the device, so the host
 // decides from the pool size and the token count (one shared adapter over a
-// large pool at 64 tokens takes the split pair, 20 % behind).
+// large pool at 64 tokens takes the split pair and 27 % longer).
 constexpr int kSplitMinSlots = 256;
 constexpr int kSplitMinTokens = 64;
 
