@@ -12,8 +12,10 @@
 // Work unit = one gather job (an adapter slot and up to 16 of its tokens, from
 // the plan kernel) times one projection (a launch may cover up to 8 that read
 // the same X) times one part e of an E-way split of d_out.  A cluster of kCS
-// CTAs (one per SM) runs one unit at a time and loops over the units
-// (persistent grid sized from the occupancy of the cluster shape).  Per CTA:
+// CTAs (one per SM) runs one unit at a time and loops over the units in
+// rounds of one unit per cluster, each round in the opposite direction to the
+// last (persistent grid sized from the occupancy of the cluster shape).  Per
+// CTA:
 //   * a producer warp streams the adapter's pages into a ring of shared-memory
 //     stages with 2D TMA loads of 16 rank rows x 64 columns (128-byte
 //     swizzled): first the CTA's 1/kCS slice of d_in (rows of A^T), then its
@@ -132,6 +134,14 @@ struct KArgs {
     int32_t *err;
     int early;           // the plan was complete before this launch started (see plan_was_last_launch)
 };
+
+// The unit a cluster runs in its round k.  Rounds alternate direction, so the
+// cluster that took one of the heaviest units first (jobs come heaviest rank
+// class first) takes one of the lightest in the next round.  Once a round's
+// unit is past the end, every later round's is too.
+__device__ __forceinline__ int unit_of(int k, int cluster_id, int n_clusters) {
+    return k * n_clusters + ((k & 1) ? n_clusters - 1 - cluster_id : cluster_id);
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -460,7 +470,7 @@ gather_kernel(const __grid_constant__ GatherMaps<NP> maps, const __grid_constant
         // the whole warp takes part in the cluster barriers.
         // ------------------------------------------------------------------
         int chunk = 0;
-        for (int u = cluster_id; u < n_units; u += n_clusters) {
+        for (int k = 0, u = cluster_id; u < n_units; ++k, u = unit_of(k, cluster_id, n_clusters)) {
             const int ji = u / upj;
             const int4 job = (ji == spec) ? spec_job : ld_v4_now(a.jobs + 2 * ji);
             const int pj = (NP == 1) ? 0 : (u - ji * upj) / E, e = u - ji * upj - pj * E;
@@ -513,7 +523,7 @@ gather_kernel(const __grid_constant__ GatherMaps<NP> maps, const __grid_constant
     int chunk = 0;
     int iter = 0;
     bool joined = false;   // passed the start-up cluster barrier
-    for (int u = cluster_id; u < n_units; u += n_clusters, ++iter) {
+    for (int u = cluster_id; u < n_units; ++iter, u = unit_of(iter, cluster_id, n_clusters)) {
         const int ji = u / upj;
         const int4 job = (ji == spec) ? spec_job : a.jobs[2 * ji];
         const int4 tk = (ji == spec) ? spec_tok : a.jobs[2 * ji + 1];
