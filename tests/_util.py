@@ -45,12 +45,6 @@ def oracle_full(wl: W.Workload, nthreads=0):
     return OC.lora_apply_c(wl.X, wl.Y_base, wl.ids, A, B, wl.scales_f32(), nthreads=nthreads)
 
 
-def oracle_tokens(wl: W.Workload, tokens, nthreads=0):
-    from oracle import build_oracle as OC
-    X, Yb, ids, A, B, sc = W.subset_for_tokens(wl, tokens)
-    return OC.lora_apply_c(X, Yb, ids, A, B, sc, nthreads=nthreads)
-
-
 def assert_parity(Y_dev: np.ndarray, Y_ref: np.ndarray, Y_base: np.ndarray, delta_rel=DELTA_REL_GATHER):
     Y_dev = np.asarray(Y_dev, np.float64)
     err = np.abs(Y_dev - Y_ref)

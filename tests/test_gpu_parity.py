@@ -107,13 +107,11 @@ def test_sweep_8b(H, regime, T):
     wl = W.sweep_8b(T=T, regime=regime)
     Y, err, _ = _run_apply(H, wl)
     assert err == 0
-    if T <= 64:
-        tokens = np.arange(T)
-    else:
-        tokens = np.sort(np.random.default_rng(T).choice(T, size=48, replace=False))
-    ref, rerr = U.oracle_tokens(wl, tokens)
+    # every token, every adapter's pages: at T = 1024 the fp64 oracle is about
+    # 2.4 GFLOP, a few seconds on the host's cores
+    ref, rerr = U.oracle_full(wl)
     assert rerr == 0
-    U.assert_parity(Y[tokens], ref, wl.Y_base[tokens], delta_rel=U.DELTA_REL_TENSOR)
+    U.assert_parity(Y, ref, wl.Y_base, delta_rel=U.DELTA_REL_TENSOR)
 
 
 # ---------------------------------------------------------------------------
